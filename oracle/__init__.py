@@ -1,0 +1,342 @@
+"""CPU oracle for MXFP8 quantisation and the MoE grouped GEMM (ctypes wrapper).
+
+TEST INFRASTRUCTURE ONLY: the tests, the package smoke check and the
+benchmark's CPU-baseline leg may import this module; the product path never
+does.  The arithmetic lives in ``mxfp8_oracle.c`` (plain C, fp64), which
+shares no source with the CUDA library.  This wrapper only marshals numpy
+arrays; bf16 tensors travel as their uint16 bit patterns.
+
+What each function follows is stated in the C file's header: MXFP8 = blocks
+of 32 elements sharing one power-of-two exponent (opensourcebeat.com,
+"Enabling up to 41% faster pre-training: MXFP8 and DeepEP ...", FAQ), with
+the OCP MX v1.0 E8M0/E4M3 rules; the grouped GEMM runs each expert on its
+real token count (iitak.ru, "NVIDIA ... JAX", Transformer Engine paragraph).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_vp = ctypes.c_void_p
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        L.orc_bf16_to_double.restype = ctypes.c_double
+        L.orc_bf16_to_double.argtypes = [ctypes.c_uint16]
+        L.orc_e4m3_decode.restype = ctypes.c_double
+        L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_encode.restype = ctypes.c_uint8
+        L.orc_e4m3_encode.argtypes = [ctypes.c_double]
+        L.orc_scale_exponent.restype = ctypes.c_int
+        L.orc_scale_exponent.argtypes = [ctypes.c_double]
+        L.orc_e4m3_encode_array.argtypes = [_vp, _i64, _vp]
+        L.orc_e4m3_decode_array.argtypes = [_vp, _i64, _vp]
+        L.orc_scale_exponent_array.argtypes = [_vp, _i64, _vp]
+        L.orc_quantize_block.argtypes = [_vp, ctypes.c_int, _i64, _vp, _i64, _vp]
+        L.orc_sf_offset.restype = _i64
+        L.orc_sf_offset.argtypes = [_i64, _i64, _i64]
+        L.orc_rowwise_pitch.restype = _i64
+        L.orc_rowwise_pitch.argtypes = [_i64]
+        L.orc_colwise_pitch.restype = _i64
+        L.orc_colwise_pitch.argtypes = [_i64, _i32]
+        L.orc_colwise_ld.restype = _i64
+        L.orc_colwise_ld.argtypes = [_i64, _i32]
+        L.orc_check_offsets.argtypes = [_vp, _i32, _i64]
+        for name in ("orc_quantize_rowwise", "orc_quantize_colwise"):
+            getattr(L, name).argtypes = [_vp, _i64, _i64, _vp, _i32, _vp, _vp]
+        for name in ("orc_dequantize_rowwise", "orc_dequantize_colwise"):
+            getattr(L, name).argtypes = [_vp, _vp, _i64, _i64, _vp, _i32, _vp]
+        for name in ("orc_gemm_fwd", "orc_gemm_dgrad", "orc_gemm_wgrad"):
+            getattr(L, name).argtypes = [_vp, _vp, _vp, _i32, _i64, _i64, _i64, _vp]
+        for name in ("orc_sample_fwd", "orc_sample_dgrad"):
+            getattr(L, name).argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64,
+                                         _i64, _vp, _vp, _vp]
+        L.orc_sample_wgrad.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64,
+                                       _i64, _vp, _vp, _vp, _vp]
+        for name in ("orc_baseline_fwd_f32", "orc_baseline_dgrad_f32", "orc_baseline_wgrad_f32"):
+            getattr(L, name).argtypes = [_vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _i64, _vp]
+        L.orc_baseline_quantize_rows.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp]
+        L.orc_threads.restype = ctypes.c_int
+        _LIB = L
+    return _LIB
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+def _u16(x) -> np.ndarray:
+    """bf16 bit patterns as a contiguous uint16 numpy array (torch or numpy input)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            assert x.dtype == torch.bfloat16
+            return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.ascontiguousarray(x)
+    assert x.dtype == np.uint16
+    return x
+
+
+def _offs(offs, rows):
+    if offs is None:
+        return None, 1
+    o = np.ascontiguousarray(np.asarray(offs, dtype=np.int32))
+    return o, len(o) - 1
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what}: invalid arguments (offsets or sizes)")
+
+
+# ---------------------------------------------------------------- scalars
+def bf16_to_double(b: int) -> float:
+    return lib().orc_bf16_to_double(b)
+
+
+def e4m3_decode(b) -> np.ndarray:
+    b = np.ascontiguousarray(np.asarray(b, dtype=np.uint8))
+    out = np.empty(b.shape, dtype=np.float64)
+    lib().orc_e4m3_decode_array(_p(b), b.size, _p(out))
+    return out
+
+
+def e4m3_encode(v) -> np.ndarray:
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().orc_e4m3_encode_array(_p(v), v.size, _p(out))
+    return out
+
+
+def scale_exponent(amax) -> np.ndarray:
+    a = np.ascontiguousarray(np.asarray(amax, dtype=np.float64))
+    out = np.empty(a.shape, dtype=np.int32)
+    lib().orc_scale_exponent_array(_p(a), a.size, _p(out))
+    return out
+
+
+def quantize_block(x_u16) -> tuple[np.ndarray, int]:
+    """One block (<= 32 values) -> (codes, scale byte)."""
+    x = _u16(x_u16).reshape(-1)
+    codes = np.empty(x.size, dtype=np.uint8)
+    sb = np.zeros(1, dtype=np.uint8)
+    lib().orc_quantize_block(_p(x), int(x.size), 1, _p(codes), 1, _p(sb))
+    return codes, int(sb[0])
+
+
+# ---------------------------------------------------------------- layouts
+def sf_offset(row: int, col: int, pitch: int) -> int:
+    return lib().orc_sf_offset(row, col, pitch)
+
+
+def rowwise_pitch(C: int) -> int:
+    return lib().orc_rowwise_pitch(C)
+
+
+def colwise_pitch(R: int, G: int) -> int:
+    return lib().orc_colwise_pitch(R, G)
+
+
+def colwise_ld(R: int, G: int) -> int:
+    return lib().orc_colwise_ld(R, G)
+
+
+def _nb128(R: int, G: int) -> int:
+    return 0 if R == 0 else (R + 127) // 128 + G - 1
+
+
+def rowwise_scale_bytes(R: int, C: int, G: int) -> int:
+    return _nb128(R, G) * rowwise_pitch(C) * 512
+
+
+def colwise_scale_bytes(R: int, C: int, G: int) -> int:
+    return ((C + 127) // 128) * colwise_pitch(R, G) * 512
+
+
+def group_blocks(offs, R):
+    """(RB_G, P_G): 128-row blocks and 32-padded rows over all groups."""
+    if offs is None:
+        return (R + 127) // 128, (R + 31) // 32 * 32
+    m = np.diff(np.asarray(offs, dtype=np.int64))
+    return int(((m + 127) // 128).sum()), int(((m + 31) // 32 * 32).sum())
+
+
+# ---------------------------------------------------------------- quantisers
+def quantize_rowwise(x, offs=None):
+    """x: bf16 [R, C] -> (q uint8 [R, C], sf uint8 [bound]); only the first
+    RB_G*pitch*512 scale bytes are defined."""
+    xu = _u16(x)
+    R, C = xu.shape
+    o, G = _offs(offs, R)
+    q = np.zeros((R, C), dtype=np.uint8)
+    sf = np.zeros(max(rowwise_scale_bytes(R, C, G), 512), dtype=np.uint8)
+    _check(lib().orc_quantize_rowwise(_p(xu), R, C, _p(o), G, _p(q), _p(sf)), "quantize_rowwise")
+    return q, sf
+
+
+def quantize_colwise(x, offs=None):
+    """x: bf16 [R, C] -> (qT uint8 [C, ldT], sfT uint8 [bound]); columns of qT
+    beyond P_G and atoms with block column >= RB_G are not defined."""
+    xu = _u16(x)
+    R, C = xu.shape
+    o, G = _offs(offs, R)
+    qT = np.zeros((C, colwise_ld(R, G)), dtype=np.uint8)
+    sf = np.zeros(max(colwise_scale_bytes(R, C, G), 512), dtype=np.uint8)
+    _check(lib().orc_quantize_colwise(_p(xu), R, C, _p(o), G, _p(qT), _p(sf)), "quantize_colwise")
+    return qT, sf
+
+
+def dequantize_rowwise(q, sf, offs=None) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    R, C = q.shape
+    o, G = _offs(offs, R)
+    out = np.zeros((R, C), dtype=np.float64)
+    _check(lib().orc_dequantize_rowwise(_p(q), _p(sf), R, C, _p(o), G, _p(out)), "dequantize_rowwise")
+    return out
+
+
+def dequantize_colwise(qT, sf, R: int, offs=None) -> np.ndarray:
+    qT = np.ascontiguousarray(qT, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    C = qT.shape[0]
+    o, G = _offs(offs, R)
+    assert qT.shape[1] == colwise_ld(R, G)
+    out = np.zeros((R, C), dtype=np.float64)
+    _check(lib().orc_dequantize_colwise(_p(qT), _p(sf), R, C, _p(o), G, _p(out)), "dequantize_colwise")
+    return out
+
+
+# ---------------------------------------------------------------- GEMMs (fp64)
+def gemm_fwd(X, W, offs) -> np.ndarray:
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    o, E = _offs(offs, X.shape[0])
+    M, K = X.shape
+    N = W.shape[1]
+    assert W.shape == (E, N, K)
+    Y = np.zeros((M, N), dtype=np.float64)
+    _check(lib().orc_gemm_fwd(_p(X), _p(W), _p(o), E, M, N, K, _p(Y)), "gemm_fwd")
+    return Y
+
+
+def gemm_dgrad(dY, W, offs) -> np.ndarray:
+    dY = np.ascontiguousarray(dY, dtype=np.float64)
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    o, E = _offs(offs, dY.shape[0])
+    M, N = dY.shape
+    K = W.shape[2]
+    assert W.shape == (E, N, K)
+    dX = np.zeros((M, K), dtype=np.float64)
+    _check(lib().orc_gemm_dgrad(_p(dY), _p(W), _p(o), E, M, N, K, _p(dX)), "gemm_dgrad")
+    return dX
+
+
+def gemm_wgrad(dY, X, offs) -> np.ndarray:
+    dY = np.ascontiguousarray(dY, dtype=np.float64)
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    o, E = _offs(offs, dY.shape[0])
+    M, N = dY.shape
+    K = X.shape[1]
+    dW = np.zeros((E, N, K), dtype=np.float64)
+    _check(lib().orc_gemm_wgrad(_p(dY), _p(X), _p(o), E, M, N, K, _p(dW)), "gemm_wgrad")
+    return dW
+
+
+# ---------------------------------------------------------------- sampled outputs
+def sample_fwd(xq, xs, wq, ws, offs, N, rows, cols) -> np.ndarray:
+    xq = np.ascontiguousarray(xq, np.uint8); xs = np.ascontiguousarray(xs, np.uint8)
+    wq = np.ascontiguousarray(wq, np.uint8); ws = np.ascontiguousarray(ws, np.uint8)
+    o, E = _offs(offs, xq.shape[0])
+    M, K = xq.shape
+    r = np.ascontiguousarray(rows, np.int64); c = np.ascontiguousarray(cols, np.int64)
+    out = np.zeros(r.size, dtype=np.float64)
+    _check(lib().orc_sample_fwd(_p(xq), _p(xs), _p(wq), _p(ws), _p(o), E, M, N, K, r.size,
+                                _p(r), _p(c), _p(out)), "sample_fwd")
+    return out
+
+
+def sample_dgrad(dyq, dys, wqT, wsT, offs, K, rows, cols) -> np.ndarray:
+    dyq = np.ascontiguousarray(dyq, np.uint8); dys = np.ascontiguousarray(dys, np.uint8)
+    wqT = np.ascontiguousarray(wqT, np.uint8); wsT = np.ascontiguousarray(wsT, np.uint8)
+    o, E = _offs(offs, dyq.shape[0])
+    M, N = dyq.shape
+    r = np.ascontiguousarray(rows, np.int64); c = np.ascontiguousarray(cols, np.int64)
+    out = np.zeros(r.size, dtype=np.float64)
+    _check(lib().orc_sample_dgrad(_p(dyq), _p(dys), _p(wqT), _p(wsT), _p(o), E, M, N, K, r.size,
+                                  _p(r), _p(c), _p(out)), "sample_dgrad")
+    return out
+
+
+def sample_wgrad(dyqT, dysT, xqT, xsT, offs, M, N, K, experts, rows, cols) -> np.ndarray:
+    dyqT = np.ascontiguousarray(dyqT, np.uint8); dysT = np.ascontiguousarray(dysT, np.uint8)
+    xqT = np.ascontiguousarray(xqT, np.uint8); xsT = np.ascontiguousarray(xsT, np.uint8)
+    o, E = _offs(offs, M)
+    e = np.ascontiguousarray(experts, np.int32)
+    r = np.ascontiguousarray(rows, np.int64); c = np.ascontiguousarray(cols, np.int64)
+    out = np.zeros(r.size, dtype=np.float64)
+    _check(lib().orc_sample_wgrad(_p(dyqT), _p(dysT), _p(xqT), _p(xsT), _p(o), E, M, N, K, r.size,
+                                  _p(e), _p(r), _p(c), _p(out)), "sample_wgrad")
+    return out
+
+
+# ---------------------------------------------------------------- CPU baseline (fp32 accumulate)
+def threads() -> int:
+    return lib().orc_threads()
+
+
+def baseline_fwd_f32(X_u16, W_u16, offs, N, row_lo, row_hi, out=None):
+    X = _u16(X_u16); W = _u16(W_u16)
+    o, E = _offs(offs, X.shape[0])
+    M, K = X.shape
+    Y = out if out is not None else np.zeros((M, N), dtype=np.float32)
+    _check(lib().orc_baseline_fwd_f32(_p(X), _p(W), _p(o), E, M, N, K, row_lo, row_hi, _p(Y)), "baseline_fwd")
+    return Y
+
+
+def baseline_dgrad_f32(dY_u16, W_u16, offs, K, row_lo, row_hi, out=None):
+    dY = _u16(dY_u16); W = _u16(W_u16)
+    o, E = _offs(offs, dY.shape[0])
+    M, N = dY.shape
+    dX = out if out is not None else np.zeros((M, K), dtype=np.float32)
+    _check(lib().orc_baseline_dgrad_f32(_p(dY), _p(W), _p(o), E, M, N, K, row_lo, row_hi, _p(dX)), "baseline_dgrad")
+    return dX
+
+
+def baseline_wgrad_f32(dY_u16, X_u16, offs, n_lo, n_hi, out=None):
+    dY = _u16(dY_u16); X = _u16(X_u16)
+    o, E = _offs(offs, dY.shape[0])
+    M, N = dY.shape
+    K = X.shape[1]
+    dW = out if out is not None else np.zeros((E, N, K), dtype=np.float32)
+    _check(lib().orc_baseline_wgrad_f32(_p(dY), _p(X), _p(o), E, M, N, K, n_lo, n_hi, _p(dW)), "baseline_wgrad")
+    return dW
+
+
+def baseline_quantize_rows(x_u16, row_lo, row_hi):
+    x = _u16(x_u16)
+    R, C = x.shape
+    q = np.zeros((R, C), dtype=np.uint8)
+    s = np.zeros((R, C // 32), dtype=np.uint8)
+    lib().orc_baseline_quantize_rows(_p(x), C, row_lo, row_hi, _p(q), _p(s))
+    return q, s
+
+
+__all__ = [n for n in dir() if not n.startswith("_") and n not in ("annotations", "ctypes", "np", "os")]

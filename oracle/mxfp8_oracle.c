@@ -1,0 +1,616 @@
+/*
+ * mxfp8_oracle.c -- plain, slow CPU oracle for MXFP8 quantisation and the
+ * dropless grouped GEMM of a Mixture-of-Experts expert layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only the tests, the package's smoke check and the CPU
+ * baseline leg of the benchmark use it.  It shares no source with the CUDA
+ * library (no headers, helpers or tables) and includes nothing from it.
+ *
+ * What it follows:
+ *   - MXFP8 is a microscaling format in which a block of 32 consecutive
+ *     elements shares one exponent (opensourcebeat.com, "Enabling up to 41%
+ *     faster pre-training: MXFP8 and DeepEP ...", FAQ "What is MXFP8?").
+ *     The block rules are those of the OCP Microscaling (MX) v1.0 format that
+ *     the benchmark spec names: E8M0 scale X = 2^(floor(log2(amax)) - emax),
+ *     emax = 8 for E4M3, clamped to the E8M0 range; element = E4M3(v / X)
+ *     with round-to-nearest-even and saturation to +-448.
+ *   - The grouped GEMM computes every expert on its real token count, with
+ *     no padding to a capacity (iitak.ru, "NVIDIA ... JAX", paragraph on the
+ *     Transformer Engine grouped GEMM): Y_e = X_e W_e^T, dX_e = dY_e W_e,
+ *     dW_e = dY_e^T X_e, each per expert e over rows offs[e]..offs[e+1]-1.
+ *
+ * Readings where the pages are silent (each is listed in the design doc):
+ *   - an all-zero block has scale exponent -127 (byte 0x00) and zero codes;
+ *   - the sign of zero survives quantisation (-0 and negative underflow
+ *     encode as 0x80), as IEEE round-to-nearest-even gives;
+ *   - a block whose amax is Inf or NaN is outside the contract; it gets the
+ *     NaN scale byte 0xFF and NaN codes 0x7F;
+ *   - colwise blocks restart at every group offset; a group's last block may
+ *     be short and its amax is over the real rows only.
+ *
+ * Data layouts (a format definition, restated here independently of the
+ * CUDA library):
+ *   rowwise: codes keep the [R, C] input layout.  Scales form a logical
+ *     matrix S[pr, j] (pr = padded row, j = 32-block index along C) in which
+ *     each group's rows start at a multiple of 128 (pr = 128*RB_g + t for
+ *     row offs[g] + t, RB_g = sum over h<g of ceil(m_h/128)).
+ *   colwise: codes are transposed, qT[c, P_g + t] for element (offs[g]+t, c),
+ *     P_g = sum over h<g of round_up(m_h, 32); the pad columns up to
+ *     round_up(m_g, 32) hold 0x00.  Scales form S^T[c, 4*RB_g + t/32].
+ *   Both scale matrices are stored in 512-byte atoms of 128 rows x 4 block
+ *     columns; atom (rb, cb) sits at byte (rb*pitch + cb)*512 and element
+ *     (row, col) inside it at (row%32)*16 + ((row%128)/32)*4 + col%4.  Pad
+ *     bytes inside a written atom are 0x00.  pitch = ceil(C/128) for rowwise,
+ *     ceil(R/128) + G - 1 for colwise.  The colwise code row stride is
+ *     ldT = round_up(round_up(R, 32) + 32*(G-1), 128), at least 128.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ */
+/* Scalars                                                              */
+/* ------------------------------------------------------------------ */
+
+/* bf16 is the top half of an IEEE binary32; widening to double is exact. */
+double orc_bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* E4M3 "fn": sign, 4 exponent bits with bias 7, 3 mantissa bits.  No
+ * infinities; S.1111.111 is NaN.  Normal: (1 + m/8) * 2^(e-7), e = 1..15
+ * (e = 15 only with m <= 6, max 448).  Subnormal: m * 2^-9. */
+double orc_e4m3_decode(uint8_t b)
+{
+    int s = b >> 7, e = (b >> 3) & 0xF, m = b & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Round v to the nearest E4M3 value, ties to the even mantissa, saturating
+ * finite overflow to +-448; the sign survives on zero. */
+uint8_t orc_e4m3_encode(double v)
+{
+    uint8_t sign;
+    double a, quantum, n, fl, rem, k, r, f;
+    int ex, e_biased, m;
+
+    if (isnan(v)) return 0x7F;
+    sign = signbit(v) ? 0x80 : 0x00;
+    a = fabs(v);
+    /* Values above 448 would round to 448 (below the 464 midpoint) or past
+     * the largest finite value; saturation maps both to 448. */
+    if (a > 448.0) return (uint8_t)(sign | 0x7E);
+    if (a < ldexp(1.0, -6)) {
+        quantum = ldexp(1.0, -9);                  /* subnormal spacing */
+    } else {
+        frexp(a, &ex);                             /* a = f*2^ex, f in [0.5,1) */
+        quantum = ldexp(1.0, (ex - 1) - 3);        /* 2^(floor(log2 a) - 3) */
+    }
+    n = a / quantum;                               /* exact: power-of-two divide */
+    fl = floor(n);
+    rem = n - fl;                                  /* exact */
+    if (rem > 0.5) k = fl + 1.0;
+    else if (rem < 0.5) k = fl;
+    else k = (fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;
+    r = k * quantum;                               /* exact, r <= 448 */
+    if (r == 0.0) return sign;
+    if (r < ldexp(1.0, -6)) {
+        m = (int)(r / ldexp(1.0, -9));
+        return (uint8_t)(sign | m);
+    }
+    f = frexp(r, &ex);
+    e_biased = (ex - 1) + 7;
+    m = (int)((f * 2.0 - 1.0) * 8.0);
+    return (uint8_t)(sign | (e_biased << 3) | m);
+}
+
+/* Shared block exponent s = floor(log2(amax)) - 8, clamped to [-127, 127];
+ * floor(log2) is read off the binary exponent, not a log function.  amax = 0
+ * gives -127.  Returns 128 for a non-finite amax (NaN scale). */
+int orc_scale_exponent(double amax)
+{
+    int ex, s;
+    if (isnan(amax) || isinf(amax)) return 128;
+    if (amax == 0.0) return -127;
+    frexp(amax, &ex);
+    s = (ex - 1) - 8;
+    if (s < -127) s = -127;
+    if (s > 127) s = 127;
+    return s;
+}
+
+uint8_t orc_scale_byte(int s) { return (uint8_t)(s + 127); }   /* 128 -> 0xFF */
+
+/* Array forms of the scalar rules, for exhaustive checks. */
+void orc_e4m3_encode_array(const double* v, int64_t n, uint8_t* out)
+{
+    int64_t i;
+    for (i = 0; i < n; ++i) out[i] = orc_e4m3_encode(v[i]);
+}
+
+void orc_e4m3_decode_array(const uint8_t* b, int64_t n, double* out)
+{
+    int64_t i;
+    for (i = 0; i < n; ++i) out[i] = orc_e4m3_decode(b[i]);
+}
+
+void orc_scale_exponent_array(const double* amax, int64_t n, int32_t* out)
+{
+    int64_t i;
+    for (i = 0; i < n; ++i) out[i] = orc_scale_exponent(amax[i]);
+}
+
+double orc_scale_value(uint8_t byte)
+{
+    if (byte == 0xFF) return NAN;
+    return ldexp(1.0, (int)byte - 127);
+}
+
+/* Quantise one block of n <= 32 bf16 values read at x[i*stride]. */
+void orc_quantize_block(const uint16_t* x, int n, int64_t stride, uint8_t* codes,
+                        int64_t code_stride, uint8_t* scale_byte)
+{
+    double amax = 0.0;
+    int i, s;
+    for (i = 0; i < n; ++i) {
+        double a = fabs(orc_bf16_to_double(x[i * stride]));
+        if (isnan(a)) { amax = NAN; break; }
+        if (a > amax) amax = a;
+    }
+    s = orc_scale_exponent(amax);
+    *scale_byte = orc_scale_byte(s);
+    for (i = 0; i < n; ++i) {
+        if (s == 128) codes[i * code_stride] = 0x7F;
+        else codes[i * code_stride] = orc_e4m3_encode(ldexp(orc_bf16_to_double(x[i * stride]), -s));
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Layout helpers                                                       */
+/* ------------------------------------------------------------------ */
+
+static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+static int64_t rup(int64_t a, int64_t b) { return cdiv(a, b) * b; }
+
+/* Byte offset of logical scale element (row, col) in the atom layout. */
+int64_t orc_sf_offset(int64_t row, int64_t col, int64_t pitch)
+{
+    int64_t atom = (row / 128) * pitch + col / 4;
+    return atom * 512 + (row % 32) * 16 + ((row % 128) / 32) * 4 + (col % 4);
+}
+
+int64_t orc_rowwise_pitch(int64_t C) { return cdiv(C, 128); }
+
+int64_t orc_colwise_pitch(int64_t R, int32_t G)
+{
+    return R == 0 ? 0 : cdiv(R, 128) + G - 1;
+}
+
+int64_t orc_colwise_ld(int64_t R, int32_t G)
+{
+    int64_t ld = rup(rup(R, 32) + 32 * (int64_t)(G - 1), 128);
+    return ld < 128 ? 128 : ld;
+}
+
+/* Default offsets: one group holding all rows. */
+static void group_bounds(const int32_t* offs, int32_t G, int64_t R, int32_t g,
+                         int64_t* lo, int64_t* hi)
+{
+    if (offs) { *lo = offs[g]; *hi = offs[g + 1]; }
+    else { *lo = 0; *hi = R; }
+}
+
+/* Prefixes RB_g (128-row blocks before group g) and P_g (32-padded rows). */
+static void group_prefixes(const int32_t* offs, int32_t G, int64_t R, int64_t* RB, int64_t* P)
+{
+    int32_t g;
+    RB[0] = 0; P[0] = 0;
+    for (g = 0; g < G; ++g) {
+        int64_t lo, hi;
+        group_bounds(offs, G, R, g, &lo, &hi);
+        RB[g + 1] = RB[g] + cdiv(hi - lo, 128);
+        P[g + 1] = P[g] + rup(hi - lo, 32);
+    }
+}
+
+/* Returns 0 if offs[0] = 0, offs non-decreasing and offs[G] = R. */
+int orc_check_offsets(const int32_t* offs, int32_t G, int64_t R)
+{
+    int32_t g;
+    if (!offs) return 0;
+    if (offs[0] != 0 || offs[G] != R) return 1;
+    for (g = 0; g < G; ++g) if (offs[g + 1] < offs[g]) return 1;
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Whole-tensor quantisers in the library layout                        */
+/* ------------------------------------------------------------------ */
+
+/* x: bf16 [R, C] row-major, C % 32 == 0.  q: [R, C].  sf: scale atoms,
+ * at least RB_G * pitch * 512 bytes; only that prefix is written. */
+int orc_quantize_rowwise(const uint16_t* x, int64_t R, int64_t C, const int32_t* offs,
+                         int32_t G, uint8_t* q, uint8_t* sf)
+{
+    int64_t pitch = orc_rowwise_pitch(C), nb = C / 32;
+    int64_t *RB, *P;
+    int32_t g;
+    if (C % 32 != 0 || G < 1 || orc_check_offsets(offs, G, R)) return 1;
+    RB = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
+    P = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
+    group_prefixes(offs, G, R, RB, P);
+    memset(sf, 0, (size_t)(RB[G] * pitch * 512));
+    for (g = 0; g < G; ++g) {
+        int64_t lo, hi, r, j;
+        group_bounds(offs, G, R, g, &lo, &hi);
+        for (r = lo; r < hi; ++r) {
+            int64_t pr = 128 * RB[g] + (r - lo);
+            for (j = 0; j < nb; ++j) {
+                uint8_t sb;
+                orc_quantize_block(x + r * C + 32 * j, 32, 1, q + r * C + 32 * j, 1, &sb);
+                sf[orc_sf_offset(pr, j, pitch)] = sb;
+            }
+        }
+    }
+    free(RB); free(P);
+    return 0;
+}
+
+/* x: bf16 [R, C].  qT: [C, ldT] with ldT = orc_colwise_ld(R, G); columns
+ * P_G..ldT-1 are not written.  sfT: pitch = orc_colwise_pitch(R, G); atoms
+ * (rb, cb) with cb < RB_G are written, for rb < ceil(C/128). */
+int orc_quantize_colwise(const uint16_t* x, int64_t R, int64_t C, const int32_t* offs,
+                         int32_t G, uint8_t* qT, uint8_t* sfT)
+{
+    int64_t ldT = orc_colwise_ld(R, G), pitch = orc_colwise_pitch(R, G);
+    int64_t *RB, *P, c, rb, cb;
+    int32_t g;
+    if (C % 32 != 0 || G < 1 || orc_check_offsets(offs, G, R)) return 1;
+    RB = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
+    P = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
+    group_prefixes(offs, G, R, RB, P);
+    for (rb = 0; rb < cdiv(C, 128); ++rb)
+        for (cb = 0; cb < RB[G]; ++cb)
+            memset(sfT + (rb * pitch + cb) * 512, 0, 512);
+    for (g = 0; g < G; ++g) {
+        int64_t lo, hi, m, t0;
+        group_bounds(offs, G, R, g, &lo, &hi);
+        m = hi - lo;
+        for (c = 0; c < C; ++c) {
+            for (t0 = 0; t0 < m; t0 += 32) {
+                int n = (int)(m - t0 < 32 ? m - t0 : 32);
+                uint8_t sb;
+                orc_quantize_block(x + (lo + t0) * C + c, n, C, qT + c * ldT + P[g] + t0, 1, &sb);
+                sfT[orc_sf_offset(c, 4 * RB[g] + t0 / 32, pitch)] = sb;
+            }
+            for (t0 = m; t0 < rup(m, 32); ++t0) qT[c * ldT + P[g] + t0] = 0;
+        }
+    }
+    free(RB); free(P);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Dequantisation from the library layout                               */
+/* ------------------------------------------------------------------ */
+
+/* out: fp64 [R, C] = code * 2^s for every element. */
+int orc_dequantize_rowwise(const uint8_t* q, const uint8_t* sf, int64_t R, int64_t C,
+                           const int32_t* offs, int32_t G, double* out)
+{
+    int64_t pitch = orc_rowwise_pitch(C);
+    int64_t *RB, *P;
+    int32_t g;
+    if (C % 32 != 0 || G < 1 || orc_check_offsets(offs, G, R)) return 1;
+    RB = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
+    P = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
+    group_prefixes(offs, G, R, RB, P);
+    for (g = 0; g < G; ++g) {
+        int64_t lo, hi, r, c;
+        group_bounds(offs, G, R, g, &lo, &hi);
+        for (r = lo; r < hi; ++r) {
+            int64_t pr = 128 * RB[g] + (r - lo);
+            for (c = 0; c < C; ++c)
+                out[r * C + c] = orc_e4m3_decode(q[r * C + c]) *
+                                 orc_scale_value(sf[orc_sf_offset(pr, c / 32, pitch)]);
+        }
+    }
+    free(RB); free(P);
+    return 0;
+}
+
+/* out: fp64 [R, C] (un-transposed) from the colwise layout. */
+int orc_dequantize_colwise(const uint8_t* qT, const uint8_t* sfT, int64_t R, int64_t C,
+                           const int32_t* offs, int32_t G, double* out)
+{
+    int64_t ldT = orc_colwise_ld(R, G), pitch = orc_colwise_pitch(R, G);
+    int64_t *RB, *P;
+    int32_t g;
+    if (C % 32 != 0 || G < 1 || orc_check_offsets(offs, G, R)) return 1;
+    RB = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
+    P = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
+    group_prefixes(offs, G, R, RB, P);
+    for (g = 0; g < G; ++g) {
+        int64_t lo, hi, t, c;
+        group_bounds(offs, G, R, g, &lo, &hi);
+        for (t = 0; t < hi - lo; ++t)
+            for (c = 0; c < C; ++c)
+                out[(lo + t) * C + c] = orc_e4m3_decode(qT[c * ldT + P[g] + t]) *
+                                        orc_scale_value(sfT[orc_sf_offset(c, 4 * RB[g] + t / 32, pitch)]);
+    }
+    free(RB); free(P);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Grouped GEMMs: the plain definition in fp64 on dense operands        */
+/* ------------------------------------------------------------------ */
+
+/* Y[i, n] = sum_k X[i, k] * W[e, n, k] for rows i of expert e. */
+int orc_gemm_fwd(const double* X, const double* W, const int32_t* offs, int32_t E,
+                 int64_t M, int64_t N, int64_t K, double* Y)
+{
+    int32_t e;
+    if (orc_check_offsets(offs, E, M)) return 1;
+    for (e = 0; e < E; ++e) {
+        int64_t i, n, k;
+        for (i = offs[e]; i < offs[e + 1]; ++i)
+            for (n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (k = 0; k < K; ++k) acc += X[i * K + k] * W[((int64_t)e * N + n) * K + k];
+                Y[i * N + n] = acc;
+            }
+    }
+    return 0;
+}
+
+/* dX[i, k] = sum_n dY[i, n] * W[e, n, k] for rows i of expert e. */
+int orc_gemm_dgrad(const double* dY, const double* W, const int32_t* offs, int32_t E,
+                   int64_t M, int64_t N, int64_t K, double* dX)
+{
+    int32_t e;
+    if (orc_check_offsets(offs, E, M)) return 1;
+    for (e = 0; e < E; ++e) {
+        int64_t i, n, k;
+        for (i = offs[e]; i < offs[e + 1]; ++i)
+            for (k = 0; k < K; ++k) {
+                double acc = 0.0;
+                for (n = 0; n < N; ++n) acc += dY[i * N + n] * W[((int64_t)e * N + n) * K + k];
+                dX[i * K + k] = acc;
+            }
+    }
+    return 0;
+}
+
+/* dW[e, n, k] = sum over rows i of expert e of dY[i, n] * X[i, k]; zero
+ * for an expert with no rows. */
+int orc_gemm_wgrad(const double* dY, const double* X, const int32_t* offs, int32_t E,
+                   int64_t M, int64_t N, int64_t K, double* dW)
+{
+    int32_t e;
+    if (orc_check_offsets(offs, E, M)) return 1;
+    for (e = 0; e < E; ++e) {
+        int64_t i, n, k;
+        for (n = 0; n < N; ++n)
+            for (k = 0; k < K; ++k) {
+                double acc = 0.0;
+                for (i = offs[e]; i < offs[e + 1]; ++i) acc += dY[i * N + n] * X[i * K + k];
+                dW[((int64_t)e * N + n) * K + k] = acc;
+            }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Sampled outputs straight from quantised operands (full-size checks)  */
+/* ------------------------------------------------------------------ */
+
+/* The group g with offs[g] <= r < offs[g+1]: the last g with offs[g] <= r
+ * (empty groups before it share its offset and are skipped). */
+static int32_t group_of_row(const int32_t* offs, int32_t G, int64_t r)
+{
+    int32_t lo = 0, hi = G - 1;
+    while (lo < hi) {
+        int32_t mid = (lo + hi + 1) / 2;
+        if (offs[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+typedef struct {
+    const uint8_t* q; const uint8_t* sf; int64_t R, C; const int32_t* offs; int32_t G;
+    int64_t pitch, ldT; int64_t *RB, *P; int colwise;
+} orc_operand;
+
+static void operand_init(orc_operand* o, const uint8_t* q, const uint8_t* sf, int64_t R,
+                         int64_t C, const int32_t* offs, int32_t G, int colwise)
+{
+    o->q = q; o->sf = sf; o->R = R; o->C = C; o->offs = offs; o->G = G; o->colwise = colwise;
+    o->pitch = colwise ? orc_colwise_pitch(R, G) : orc_rowwise_pitch(C);
+    o->ldT = orc_colwise_ld(R, G);
+    o->RB = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
+    o->P = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
+    group_prefixes(offs, G, R, o->RB, o->P);
+}
+
+static void operand_free(orc_operand* o) { free(o->RB); free(o->P); }
+
+/* Dequantised logical element (r, c) of an operand of logical shape [R, C]. */
+static double operand_at(const orc_operand* o, int64_t r, int64_t c)
+{
+    int32_t g = o->offs ? group_of_row(o->offs, o->G, r) : 0;
+    int64_t lo = o->offs ? o->offs[g] : 0, t = r - lo;
+    if (!o->colwise)
+        return orc_e4m3_decode(o->q[r * o->C + c]) *
+               orc_scale_value(o->sf[orc_sf_offset(128 * o->RB[g] + t, c / 32, o->pitch)]);
+    return orc_e4m3_decode(o->q[c * o->ldT + o->P[g] + t]) *
+           orc_scale_value(o->sf[orc_sf_offset(c, 4 * o->RB[g] + t / 32, o->pitch)]);
+}
+
+/* fwd sample: Y[rows[s], cols[s]]; X rowwise [M, K] grouped by offs, W
+ * rowwise [E*N, K] quantised as one group. */
+int orc_sample_fwd(const uint8_t* xq, const uint8_t* xs, const uint8_t* wq, const uint8_t* ws,
+                   const int32_t* offs, int32_t E, int64_t M, int64_t N, int64_t K,
+                   int64_t ns, const int64_t* rows, const int64_t* cols, double* out)
+{
+    orc_operand X, W;
+    int64_t s;
+    if (orc_check_offsets(offs, E, M)) return 1;
+    operand_init(&X, xq, xs, M, K, offs, E, 0);
+    operand_init(&W, wq, ws, (int64_t)E * N, K, NULL, 1, 0);
+    for (s = 0; s < ns; ++s) {
+        int64_t i = rows[s], n = cols[s], k;
+        int32_t e = group_of_row(offs, E, i);
+        double acc = 0.0;
+        for (k = 0; k < K; ++k) acc += operand_at(&X, i, k) * operand_at(&W, (int64_t)e * N + n, k);
+        out[s] = acc;
+    }
+    operand_free(&X); operand_free(&W);
+    return 0;
+}
+
+/* dgrad sample: dX[rows[s], cols[s]]; dY rowwise [M, N] grouped by offs,
+ * W colwise (logical [E*N, K], one group). */
+int orc_sample_dgrad(const uint8_t* dyq, const uint8_t* dys, const uint8_t* wqT,
+                     const uint8_t* wsT, const int32_t* offs, int32_t E, int64_t M, int64_t N,
+                     int64_t K, int64_t ns, const int64_t* rows, const int64_t* cols, double* out)
+{
+    orc_operand D, W;
+    int64_t s;
+    if (orc_check_offsets(offs, E, M)) return 1;
+    operand_init(&D, dyq, dys, M, N, offs, E, 0);
+    operand_init(&W, wqT, wsT, (int64_t)E * N, K, NULL, 1, 1);
+    for (s = 0; s < ns; ++s) {
+        int64_t i = rows[s], k = cols[s], n;
+        int32_t e = group_of_row(offs, E, i);
+        double acc = 0.0;
+        for (n = 0; n < N; ++n) acc += operand_at(&D, i, n) * operand_at(&W, (int64_t)e * N + n, k);
+        out[s] = acc;
+    }
+    operand_free(&D); operand_free(&W);
+    return 0;
+}
+
+/* wgrad sample: dW[experts[s], rows[s], cols[s]]; dY and X colwise, both
+ * grouped by offs. */
+int orc_sample_wgrad(const uint8_t* dyqT, const uint8_t* dysT, const uint8_t* xqT,
+                     const uint8_t* xsT, const int32_t* offs, int32_t E, int64_t M, int64_t N,
+                     int64_t K, int64_t ns, const int32_t* experts, const int64_t* rows,
+                     const int64_t* cols, double* out)
+{
+    orc_operand D, X;
+    int64_t s;
+    if (orc_check_offsets(offs, E, M)) return 1;
+    operand_init(&D, dyqT, dysT, M, N, offs, E, 1);
+    operand_init(&X, xqT, xsT, M, K, offs, E, 1);
+    for (s = 0; s < ns; ++s) {
+        int32_t e = experts[s];
+        int64_t n = rows[s], k = cols[s], i;
+        double acc = 0.0;
+        for (i = offs[e]; i < offs[e + 1]; ++i) acc += operand_at(&D, i, n) * operand_at(&X, i, k);
+        out[s] = acc;
+    }
+    operand_free(&D); operand_free(&X);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* CPU baseline: bf16 inputs, fp32 accumulation, rows split over threads */
+/* ------------------------------------------------------------------ */
+
+static float bf16f(uint16_t b) { uint32_t u = (uint32_t)b << 16; float f; memcpy(&f, &u, 4); return f; }
+
+int orc_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Y = X_e W_e^T for rows [row_lo, row_hi) only (a bounded sample). */
+int orc_baseline_fwd_f32(const uint16_t* X, const uint16_t* W, const int32_t* offs, int32_t E,
+                         int64_t M, int64_t N, int64_t K, int64_t row_lo, int64_t row_hi, float* Y)
+{
+    int64_t i;
+    if (orc_check_offsets(offs, E, M)) return 1;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (i = row_lo; i < row_hi; ++i) {
+        int32_t e = group_of_row(offs, E, i);
+        int64_t n, k;
+        for (n = 0; n < N; ++n) {
+            float acc = 0.0f;
+            for (k = 0; k < K; ++k) acc += bf16f(X[i * K + k]) * bf16f(W[((int64_t)e * N + n) * K + k]);
+            Y[i * N + n] = acc;
+        }
+    }
+    return 0;
+}
+
+/* dX = dY_e W_e for rows [row_lo, row_hi). */
+int orc_baseline_dgrad_f32(const uint16_t* dY, const uint16_t* W, const int32_t* offs, int32_t E,
+                           int64_t M, int64_t N, int64_t K, int64_t row_lo, int64_t row_hi, float* dX)
+{
+    int64_t i;
+    if (orc_check_offsets(offs, E, M)) return 1;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (i = row_lo; i < row_hi; ++i) {
+        int32_t e = group_of_row(offs, E, i);
+        int64_t n, k;
+        for (k = 0; k < K; ++k) dX[i * K + k] = 0.0f;
+        for (n = 0; n < N; ++n) {
+            float d = bf16f(dY[i * N + n]);
+            for (k = 0; k < K; ++k) dX[i * K + k] += d * bf16f(W[((int64_t)e * N + n) * K + k]);
+        }
+    }
+    return 0;
+}
+
+/* dW_e = dY_e^T X_e for output rows n in [n_lo, n_hi) of every expert. */
+int orc_baseline_wgrad_f32(const uint16_t* dY, const uint16_t* X, const int32_t* offs, int32_t E,
+                           int64_t M, int64_t N, int64_t K, int64_t n_lo, int64_t n_hi, float* dW)
+{
+    int64_t en;
+    if (orc_check_offsets(offs, E, M)) return 1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (en = 0; en < (int64_t)E * (n_hi - n_lo); ++en) {
+        int32_t e = (int32_t)(en / (n_hi - n_lo));
+        int64_t n = n_lo + en % (n_hi - n_lo), i, k;
+        float* out = dW + ((int64_t)e * N + n) * K;
+        for (k = 0; k < K; ++k) out[k] = 0.0f;
+        for (i = offs[e]; i < offs[e + 1]; ++i) {
+            float d = bf16f(dY[i * N + n]);
+            for (k = 0; k < K; ++k) out[k] += d * bf16f(X[i * K + k]);
+        }
+    }
+    return 0;
+}
+
+/* Whole-tensor quantiser timing helper for the CPU baseline: rowwise over
+ * rows [row_lo, row_hi) of a single-group tensor (codes and logical scales). */
+int orc_baseline_quantize_rows(const uint16_t* x, int64_t C, int64_t row_lo, int64_t row_hi,
+                               uint8_t* q, uint8_t* s_logical)
+{
+    int64_t r;
+#pragma omp parallel for schedule(static)
+    for (r = row_lo; r < row_hi; ++r) {
+        int64_t j;
+        for (j = 0; j < C / 32; ++j)
+            orc_quantize_block(x + r * C + 32 * j, 32, 1, q + r * C + 32 * j, 1, s_logical + r * (C / 32) + j);
+    }
+    return 0;
+}
