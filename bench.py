@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Benchmark of the MXFP8 MoE expert-layer hot path on B200.
+
+One step = one pass of the whole path over one synthetic routed batch of the
+DeepSeek-V3-16B-like MoE layer (64 experts, top-6 of 8192 tokens = 49152
+rows; gate/up N = 2816, K = 2048; down N = 2048, K = 1408): for each of the
+two grouped linears, rowwise + colwise MXFP8 quantisation of X, W and dY,
+then the forward, dgrad and wgrad grouped GEMMs.  The metric is algorithmic
+GEMM TFLOP/s (3 passes x 2*M*N*K per linear over real tokens) per step.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+N > 1 (launched by torchrun): every rank runs its own copy of the layer on its
+own GPU (experts are independent; no data-path collective), torch.distributed
+is used only for the barrier and the max over ranks of the timings.
+``--impl reference`` times the CPU oracle (bf16 inputs, fp32 accumulation)
+on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mxfp8_grouped_gemm_quantize_b200 import workloads as wl  # noqa: E402
+
+METRIC = "MoE grouped-GEMM MXFP8 TFLOP/s (fwd+dgrad+wgrad) and % of B200 FP8 peak"
+UNIT = "TFLOP/s"
+WORKLOAD = "ds-v3-16b"
+FP8_OVER_BF16 = 2.0   # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"], "bf16_sust": d.get("bf16_tflops_sustained"),
+                "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sust": 1400.0, "src": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks (NVML reads only)
+class ClockSampler:
+    BAD = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+    def __init__(self, device_index: int, period_s=0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self.stop_evt, self.thread = period_s, threading.Event(), None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _reason_names(self, mask):
+        nv = self.nv
+        names = {"hw_slowdown": getattr(nv, "nvmlClocksThrottleReasonHwSlowdown", 0x8),
+                 "hw_thermal_slowdown": getattr(nv, "nvmlClocksThrottleReasonHwThermalSlowdown", 0x40),
+                 "sw_thermal_slowdown": getattr(nv, "nvmlClocksThrottleReasonSwThermalSlowdown", 0x20),
+                 "sw_power_cap": getattr(nv, "nvmlClocksThrottleReasonSwPowerCap", 0x4)}
+        return {k for k, bit in names.items() if mask & bit}
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_evt.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                self.reasons |= self._reason_names(fn(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.thread:
+            self.stop_evt.set()
+            self.thread.join()
+
+    def summary(self):
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- one grouped linear on the GPU
+class Linear:
+    """Device buffers and launches for one grouped linear (all three passes)."""
+
+    def __init__(self, mx, w: wl.Workload, layer: wl.Layer, device):
+        self.mx = mx
+        self.name = layer.name
+        self.M, self.N, self.K, self.E = w.M, layer.N, layer.K, w.E
+        self.X, W, self.dY = wl.layer_tensors(w, layer, device=device)
+        self.W2 = W.reshape(self.E * self.N, self.K)
+        self.offs = torch.from_numpy(w.offsets).to(device)
+        M, N, K, E = self.M, self.N, self.K, self.E
+        u8 = lambda n: torch.empty(max(int(n), 16), dtype=torch.uint8, device=device)  # noqa: E731
+        self.xq, self.xs = torch.empty((M, K), dtype=torch.uint8, device=device), u8(mx.mxfp8_rowwise_scale_bytes(M, K, E))
+        self.wq, self.ws = torch.empty((E * N, K), dtype=torch.uint8, device=device), u8(mx.mxfp8_rowwise_scale_bytes(E * N, K, 1))
+        self.dyq, self.dys = torch.empty((M, N), dtype=torch.uint8, device=device), u8(mx.mxfp8_rowwise_scale_bytes(M, N, E))
+        self.wqT = torch.empty((K, mx.mxfp8_colwise_ld(E * N, 1)), dtype=torch.uint8, device=device)
+        self.wsT = u8(mx.mxfp8_colwise_scale_bytes(E * N, K, 1))
+        ldm = mx.mxfp8_colwise_ld(M, E)
+        self.dyqT, self.dysT = torch.empty((N, ldm), dtype=torch.uint8, device=device), u8(mx.mxfp8_colwise_scale_bytes(M, N, E))
+        self.xqT, self.xsT = torch.empty((K, ldm), dtype=torch.uint8, device=device), u8(mx.mxfp8_colwise_scale_bytes(M, K, E))
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        self.dx = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+        self.dw = torch.empty((E, N, K), dtype=torch.bfloat16, device=device)
+        self.work = mx.new_workspace(E, M, N, K, device)
+
+    def flops_per_pass(self):
+        return 2 * self.M * self.N * self.K
+
+    def quant_bytes(self):
+        """Algorithmic bytes of the six quantisations: 2 B read, 1 + 1/32 B written per element."""
+        el = 2 * (self.M * self.K + self.E * self.N * self.K + self.M * self.N)
+        return el * (2 + 1 + 1 / 32)
+
+    def launches(self):
+        """(kind, callable) for one pass of the path; kind is 'quant' or 'gemm:<pass>'."""
+        mx = self.mx
+        return [
+            ("quant", lambda: mx.mxfp8_quantize_rowwise(self.X, self.offs, q=self.xq, scales=self.xs)),
+            ("quant", lambda: mx.mxfp8_quantize_rowwise(self.W2, None, q=self.wq, scales=self.ws)),
+            ("gemm:fwd", lambda: mx.mxfp8_grouped_gemm_fwd(self.xq, self.xs, self.wq, self.ws, self.offs, self.N,
+                                                           out=self.y, work=self.work)),
+            ("quant", lambda: mx.mxfp8_quantize_rowwise(self.dY, self.offs, q=self.dyq, scales=self.dys)),
+            ("quant", lambda: mx.mxfp8_quantize_colwise(self.W2, None, qT=self.wqT, scales=self.wsT)),
+            ("gemm:dgrad", lambda: mx.mxfp8_grouped_gemm_dgrad(self.dyq, self.dys, self.wqT, self.wsT, self.offs,
+                                                               self.K, out=self.dx, work=self.work)),
+            ("quant", lambda: mx.mxfp8_quantize_colwise(self.dY, self.offs, qT=self.dyqT, scales=self.dysT)),
+            ("quant", lambda: mx.mxfp8_quantize_colwise(self.X, self.offs, qT=self.xqT, scales=self.xsT)),
+            ("gemm:wgrad", lambda: mx.mxfp8_grouped_gemm_wgrad(self.dyqT, self.dysT, self.xqT, self.xsT, self.offs,
+                                                               self.M, out=self.dw, work=self.work)),
+        ]
+
+
+def run_ours(args, rank, world, local_rank):
+    import mxfp8_grouped_gemm_quantize_b200 as mx
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if not mx.mxfp8_device_supported():
+        raise SystemExit("bench: the current device is not sm_100")
+    w = wl.WORKLOADS[args.workload]()
+    layers = [Linear(mx, w, L, dev) for L in w.layers]
+    calls = [c for L in layers for c in L.launches()]
+    step_flops = 3 * sum(L.flops_per_pass() for L in layers)
+    quant_bytes = sum(L.quant_bytes() for L in layers)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for _, fn in calls:
+            fn()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    for L in layers:
+        st = mx.mxfp8_get_status(L.work)
+        if st != 0:
+            raise SystemExit(f"bench: device status {st} after warm-up")
+
+    # per-launch events inside the timed region (same stream as the launches)
+    K = args.steps
+    n_calls = len(calls)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_calls + 1)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        start.record(stream)
+        for s in range(K):
+            e = ev[s]
+            e[0].record(stream)
+            for i, (_, fn) in enumerate(calls):
+                fn()
+                e[i + 1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = start.elapsed_time(end)
+    per_kind = {}
+    for s in range(K):
+        for i, (kind, _) in enumerate(calls):
+            per_kind.setdefault(kind, []).append(ev[s][i].elapsed_time(ev[s][i + 1]))
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / K
+    value = world * step_flops / (ms_step * 1e-3) / 1e12
+
+    pk = peaks()
+    fp8_peak = pk["bf16"] * FP8_OVER_BF16
+    gemm_ms = sum(sum(v) for k, v in per_kind.items() if k.startswith("gemm")) / K
+    gemm_launches = sum(len(v) for k, v in per_kind.items() if k.startswith("gemm"))
+    gemm_tflops = step_flops / (gemm_ms * 1e-3) / 1e12
+    quant_ms = sum(per_kind["quant"]) / K
+    quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+    breakdown = {}
+    for kind, v in per_kind.items():
+        if kind.startswith("gemm"):
+            p = kind.split(":")[1]
+            breakdown[p] = {"ms_per_step": round(sum(v) / K, 4),
+                            "tflops": round((step_flops / 3) / (sum(v) / K * 1e-3) / 1e12, 1)}
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": f"{w.name}-like MoE layer", "experts": w.E, "routed_rows": w.M,
+                   "layers": [{"name": L.name, "N": L.N, "K": L.K} for L in w.layers],
+                   "routing": "top-6 of 8192 tokens, N(0,1) logits + N(0,0.5) expert bias" if w.name == "ds-v3-16b" else w.name,
+                   "l2": "inputs larger than L2 (step touches > 2 GB)", "parallelism": f"replica x{world}"},
+        "fraction_of_fp8_peak": round(value / world / fp8_peak, 4),
+        "roofline": {"kernel": "grouped_gemm_kernel (fwd+dgrad+wgrad launches)", "bound": "tensor",
+                     "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(gemm_tflops / fp8_peak, 4), "traffic": None,
+                     "peak_source": f"{pk['src']} bf16 burst x {FP8_OVER_BF16} (nominal FP8/BF16)",
+                     "launches_timed": gemm_launches},
+        "quantiser": {"achieved_gbs": round(quant_gbs, 1), "peak_gbs": pk["hbm_gbs"],
+                      "frac": round(quant_gbs / pk["hbm_gbs"], 4), "ms_per_step": round(quant_ms, 4)},
+        "breakdown": breakdown,
+        "gpu_launches": K * n_calls,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline(w, budget_s=12.0)
+    out["e2e"] = e2e(args, mx, w, layers, dev, world)
+    return out
+
+
+def e2e(args, mx, w, layers, dev, world):
+    """Same metric through the public API with host buffers: every step copies
+    the bf16 inputs (X, W, dY of both linears) and the offsets from pinned host
+    memory, runs the path and copies Y, dX and dW back to pinned host memory."""
+    stream = torch.cuda.current_stream()
+    host_in, host_out = [], []
+    for L in layers:
+        host_in += [(L.X, L.X.cpu().pin_memory()), (L.W2, L.W2.cpu().pin_memory()),
+                    (L.dY, L.dY.cpu().pin_memory()), (L.offs, L.offs.cpu().pin_memory())]
+        host_out += [(L.y, torch.empty_like(L.y, device="cpu").pin_memory()),
+                     (L.dx, torch.empty_like(L.dx, device="cpu").pin_memory()),
+                     (L.dw, torch.empty_like(L.dw, device="cpu").pin_memory())]
+    calls = [fn for L in layers for _, fn in L.launches()]
+    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
+    d2h = sum(h.numel() * h.element_size() for _, h in host_out)
+
+    def step():
+        for d, h in host_in:
+            d.copy_(h, non_blocking=True)
+        for fn in calls:
+            fn()
+        for d, h in host_out:
+            h.copy_(d, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    K = max(1, args.e2e_steps)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    a.record(stream)
+    for _ in range(K):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / K
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    flops = 3 * sum(L.flops_per_pass() for L in layers)
+    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": UNIT, "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": K}
+
+
+# ---------------------------------------------------------------- CPU oracle baseline / reference arm
+def _cpu_sample(w: wl.Workload, budget_s: float):
+    """Times the oracle's bf16-input fp32-accumulate fwd, dgrad and wgrad on
+    a bounded sample of the first linear (rows / output rows chosen so the
+    sample takes about budget_s); returns (flops, seconds, description)."""
+    import oracle
+    layer = w.layers[0]
+    X, W, dY = wl.layer_tensors(w, layer)
+    W2 = W.reshape(w.E * layer.N, layer.K)
+    offs = w.offsets
+    N, K, M = layer.N, layer.K, w.M
+    t0 = time.perf_counter()
+    oracle.baseline_fwd_f32(X, W2, offs, N, 0, 8)
+    rate = 2 * 8 * N * K / max(time.perf_counter() - t0, 1e-6)      # FLOP/s estimate
+    rows = int(max(1, min(M, budget_s / 3 * rate / (2 * N * K))))
+    # wgrad sample: output rows n in [0, nr) for every expert (work 2*M*nr*K)
+    nr = int(max(1, min(N, budget_s / 3 * rate / (2 * M * K))))
+    Y = np.zeros((M, N), dtype=np.float32)
+    dX = np.zeros((M, K), dtype=np.float32)
+    dW = np.zeros((w.E, N, K), dtype=np.float32)
+    t0 = time.perf_counter()
+    oracle.baseline_fwd_f32(X, W2, offs, N, 0, rows, out=Y)
+    oracle.baseline_dgrad_f32(dY, W2, offs, K, 0, rows, out=dX)
+    oracle.baseline_wgrad_f32(dY, X, offs, 0, nr, out=dW)
+    secs = time.perf_counter() - t0
+    flops = 2 * rows * N * K * 2 + 2 * M * nr * K
+    desc = (f"{layer.name} linear of {w.name}: fwd+dgrad on rows 0..{rows - 1} of {M}, "
+            f"wgrad on output rows 0..{nr - 1} of {N} for all {w.E} experts")
+    return flops, secs, desc
+
+
+def cpu_baseline(w, budget_s=12.0):
+    import oracle
+    flops, secs, desc = _cpu_sample(w, budget_s)
+    return {"value": round(flops / secs / 1e12, 5), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": desc, "seconds": round(secs, 2)}
+
+
+def run_reference(args):
+    import oracle
+    w = wl.WORKLOADS[args.workload]()
+    steps, warm = max(1, args.steps), max(0, args.warmup)
+    per_step = max(0.05, min(2.0, 120.0 / (steps + warm)))
+    for _ in range(warm):
+        _cpu_sample(w, per_step)
+    tot_f, tot_s, desc = 0, 0.0, ""
+    for _ in range(steps):
+        f, s, desc = _cpu_sample(w, per_step)
+        tot_f += f
+        tot_s += s
+    value = tot_f / tot_s / 1e12
+    return {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": args.gpus, "steps": steps,
+            "warmup": warm, "ms_per_step": round(1e3 * tot_s / steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 inputs)", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": f"{w.name}-like MoE layer", "experts": w.E, "routed_rows": w.M,
+                       "layers": [{"name": L.name, "N": L.N, "K": L.K} for L in w.layers]},
+            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                             "sample": desc + f"; {per_step:.2f} s per step"},
+            "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

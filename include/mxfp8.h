@@ -1,0 +1,194 @@
+/*
+ * mxfp8.h -- C ABI of the B200 (sm_100a) MXFP8 quantisers and the dropless
+ * grouped GEMM of a Mixture-of-Experts expert layer.
+ *
+ * What is computed
+ *   MXFP8: every block of 32 consecutive elements shares one power-of-two
+ *   scale (opensourcebeat.com, "Enabling up to 41% faster pre-training: MXFP8
+ *   and DeepEP for DeepSeek-V3 on B200 with TorchTitan", FAQ "What is
+ *   MXFP8?"; the same page, section "Двухсторонняя атака", says Blackwell's
+ *   5th-generation tensor cores run it natively).  The block rules are OCP MX
+ *   v1.0: the E8M0 scale byte is s + 127 with s = floor(log2(amax)) - 8
+ *   clamped to [-127, 127] (amax = 0 gives byte 0x00); each element becomes
+ *   the E4M3 code of x * 2^-s, rounded to nearest even and saturated to
+ *   +-448; the sign survives on zero.  A block with a non-finite element is
+ *   outside the contract and gets scale 0xFF and codes 0x7F.
+ *
+ *   Grouped GEMM: all experts run in one launch, each on its real token count,
+ *   with no padding to a capacity and no dropped tokens (iitak.ru, "NVIDIA
+ *   в 10 раз ускорила обучение моделей-«смесей экспертов» на JAX", paragraphs
+ *   on dropless routing and the Transformer Engine grouped GEMM; the two
+ *   all-to-alls around it are on opensourcebeat.com, section "Двухсторонняя
+ *   атака").  For expert e owning rows offs[e] .. offs[e+1]-1:
+ *     forward  Y_e  = X_e  W_e^T     Y  [M, N]
+ *     dgrad    dX_e = dY_e W_e       dX [M, K]
+ *     wgrad    dW_e = dY_e^T X_e     dW [E, N, K]  (zero when m_e = 0)
+ *   Products of dequantised operands are accumulated in fp32 (tensor memory)
+ *   and written as bf16 (round to nearest even).
+ *
+ * Conventions
+ *   - Every pointer except the `stream` is a DEVICE pointer owned by the
+ *     caller; the library allocates nothing and keeps no pointer after a call.
+ *   - bf16 data is passed as its uint16 bit pattern.  All matrices are
+ *     row-major.  Data and scale pointers must be 16-byte aligned.
+ *   - `d_offs` is an int32 device array of num_groups + 1 exclusive prefix
+ *     offsets: d_offs[0] = 0, non-decreasing, d_offs[num_groups] = rows.  A
+ *     NULL `d_offs` means one group holding every row.  The quantisers never
+ *     read or write out of bounds for any offsets (they clamp them); the GEMMs
+ *     check them on the device and report MXF8_ERR_BAD_OFFSETS through the
+ *     workspace status without touching the output.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous: a return of MXF8_OK means the launch was accepted.
+ *   - Only sm_100 devices (B200/GB200) are supported.
+ *
+ * Layouts (shared by the quantisers' outputs and the GEMMs' inputs)
+ *   Scale atoms: scales are stored in 512-byte atoms covering 128 rows x 4
+ *   32-blocks; atom (rb, cb) starts at byte 512*(rb*pitch + cb) and logical
+ *   scale (row, blk) sits at byte (row%32)*16 + ((row%128)/32)*4 + blk%4 inside
+ *   it.  This is the scale-factor layout tcgen05 block-scaled MMA reads from
+ *   tensor memory after a 32x128-bit copy; pad bytes inside a written atom
+ *   are 0x00.
+ *   Rowwise (blocks along the last dimension): codes keep the [rows, cols]
+ *   layout; scale rows of group g start at a multiple of 128 (padded row
+ *   128*RB_g + t for row d_offs[g] + t, RB_g = sum over h < g of
+ *   ceil(m_h/128)); pitch = ceil(cols/128).
+ *   Colwise (blocks along rows, restarting at every group offset; a short
+ *   last block covers the real rows only): codes are transposed, qT[c, P_g + t]
+ *   holds element (d_offs[g] + t, c) with P_g = sum over h < g of
+ *   round_up(m_h, 32), and the pad columns up to round_up(m_g, 32) are 0x00;
+ *   the row stride is ldT = mxfp8_colwise_ld(rows, num_groups).  The scales
+ *   form the matrix S^T[c, 4*RB_g + t/32] with pitch
+ *   mxfp8_colwise_pitch(rows, num_groups).  Every GEMM operand is then K-major.
+ */
+#ifndef MXFP8_H
+#define MXFP8_H
+
+#include <stdint.h>
+
+/* Symbols of the shared library are exported explicitly (it is built with
+ * hidden visibility). */
+#if defined(__GNUC__)
+#define MXF8_API __attribute__((visibility("default")))
+#else
+#define MXF8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MXF8_OK = 0,
+    MXF8_ERR_INVALID_ARG = 1,  /* null pointer, bad size, buffer too small, too many groups */
+    MXF8_ERR_ALIGNMENT = 2,    /* a pointer is not 16-byte aligned */
+    MXF8_ERR_UNSUPPORTED = 3,  /* the current device is not sm_100 */
+    MXF8_ERR_CUDA = 4,         /* a CUDA call failed; see mxfp8_last_cuda_error() */
+    MXF8_ERR_BAD_OFFSETS = 5,  /* device side: d_offs is not a valid prefix of `rows` */
+    MXF8_ERR_TIMEOUT = 6       /* device side: a pipeline wait ran past its limit */
+} mxf8_status;
+
+/* Largest num_groups (experts) a grouped GEMM accepts. */
+#define MXF8_GEMM_MAX_GROUPS 256
+
+/* ---------------------------------------------------------------- sizes */
+
+/* Bytes the rowwise scale buffer needs for a [rows, cols] input split into
+ * num_groups groups: (ceil(rows/128) + num_groups - 1) * ceil(cols/128) * 512
+ * (0 when rows = 0).  Only the prefix used by the actual offsets is written. */
+MXF8_API int64_t mxfp8_rowwise_scale_bytes(int64_t rows, int64_t cols, int32_t num_groups);
+
+/* Atom pitch of the colwise scale matrix: ceil(rows/128) + num_groups - 1. */
+MXF8_API int64_t mxfp8_colwise_pitch(int64_t rows, int32_t num_groups);
+
+/* Bytes the colwise scale buffer needs: ceil(cols/128) * pitch * 512. */
+MXF8_API int64_t mxfp8_colwise_scale_bytes(int64_t rows, int64_t cols, int32_t num_groups);
+
+/* Row stride (bytes) of the transposed colwise codes:
+ * round_up(round_up(rows, 32) + 32*(num_groups-1), 128), at least 128. */
+MXF8_API int64_t mxfp8_colwise_ld(int64_t rows, int32_t num_groups);
+
+/* Bytes of the workspace a grouped GEMM needs (a status word and reserve). */
+MXF8_API int64_t mxfp8_workspace_bytes(int32_t num_groups, int64_t M, int64_t N, int64_t K);
+
+/* ---------------------------------------------------------------- quantisers */
+
+/* Rowwise MXFP8 quantisation (32-blocks along `cols`).
+ *   x       bf16 [rows, cols], cols % 32 == 0, rows >= 0
+ *   d_offs  num_groups + 1 row offsets (NULL: one group)
+ *   q       uint8 [rows, cols] E4M3 codes
+ *   scales  uint8 [scale_bytes] E8M0 atoms, scale_bytes >=
+ *           mxfp8_rowwise_scale_bytes(rows, cols, num_groups)
+ * Errors: INVALID_ARG (null x/q/scales -- x and q may be NULL when rows = 0 --,
+ * cols % 32, num_groups < 1, buffer too small), ALIGNMENT, UNSUPPORTED, CUDA.
+ * Nothing is launched on error. */
+MXF8_API mxf8_status mxfp8_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols,
+                                   const int32_t* d_offs, int32_t num_groups,
+                                   uint8_t* q, uint8_t* scales, int64_t scale_bytes,
+                                   void* stream);
+
+/* Colwise MXFP8 quantisation (32-blocks along `rows`, restarting at every
+ * group offset), written transposed.
+ *   x        bf16 [rows, cols], cols % 32 == 0
+ *   qT       uint8 [cols, ldT], ldT == mxfp8_colwise_ld(rows, num_groups);
+ *            columns past the last group's padded end are not written
+ *   scalesT  uint8 [scale_bytes] >= mxfp8_colwise_scale_bytes(...)
+ * Errors as mxfp8_quantize_rowwise, plus INVALID_ARG for a wrong ldT. */
+MXF8_API mxf8_status mxfp8_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols,
+                                   const int32_t* d_offs, int32_t num_groups,
+                                   uint8_t* qT, int64_t ldT, uint8_t* scalesT,
+                                   int64_t scale_bytes, void* stream);
+
+/* ---------------------------------------------------------------- grouped GEMMs
+ * Shared arguments: E = num_groups (1..MXF8_GEMM_MAX_GROUPS); M = total rows
+ * (d_offs[E]); N % 128 == 0; K % 32 == 0; N, K > 0.  `work` is a device
+ * workspace of work_bytes >= mxfp8_workspace_bytes(E, M, N, K) that one call
+ * at a time may use; when M = 0 the row-indexed operand and output may be NULL
+ * (wgrad still writes dW = 0).  The status word is cleared at the start of every call
+ * and set by the device on BAD_OFFSETS or TIMEOUT (read it with
+ * mxfp8_get_status).  Errors returned directly: INVALID_ARG, ALIGNMENT,
+ * UNSUPPORTED, CUDA; nothing is launched on error. */
+
+/* Forward: y[M, N] bf16.  xq/xs: rowwise(X [M, K], d_offs);
+ * wq/ws: rowwise(W viewed as [E*N, K], one group). */
+MXF8_API mxf8_status mxfp8_grouped_gemm_fwd(const uint8_t* xq, const uint8_t* xs, int64_t xs_bytes,
+                                   const uint8_t* wq, const uint8_t* ws, int64_t ws_bytes,
+                                   const int32_t* d_offs, int32_t E, int64_t M, int64_t N,
+                                   int64_t K, uint16_t* y, void* work, int64_t work_bytes,
+                                   void* stream);
+
+/* Dgrad: dx[M, K] bf16.  dyq/dys: rowwise(dY [M, N], d_offs);
+ * wqT/wsT: colwise(W viewed as [E*N, K], one group), ldT = mxfp8_colwise_ld(E*N, 1). */
+MXF8_API mxf8_status mxfp8_grouped_gemm_dgrad(const uint8_t* dyq, const uint8_t* dys, int64_t dys_bytes,
+                                     const uint8_t* wqT, const uint8_t* wsT, int64_t wsT_bytes,
+                                     const int32_t* d_offs, int32_t E, int64_t M, int64_t N,
+                                     int64_t K, uint16_t* dx, void* work, int64_t work_bytes,
+                                     void* stream);
+
+/* Wgrad: dw[E, N, K] bf16.  dyqT/dysT: colwise(dY [M, N], d_offs);
+ * xqT/xsT: colwise(X [M, K], d_offs); both with ldT = mxfp8_colwise_ld(M, E).
+ * Experts with no rows get dW_e = 0. */
+MXF8_API mxf8_status mxfp8_grouped_gemm_wgrad(const uint8_t* dyqT, const uint8_t* dysT, int64_t dysT_bytes,
+                                     const uint8_t* xqT, const uint8_t* xsT, int64_t xsT_bytes,
+                                     const int32_t* d_offs, int32_t E, int64_t M, int64_t N,
+                                     int64_t K, uint16_t* dw, void* work, int64_t work_bytes,
+                                     void* stream);
+
+/* ---------------------------------------------------------------- status */
+
+/* Synchronises `stream`, then stores the device status of the last GEMM that
+ * used `work` (an mxf8_status value, MXF8_OK if none) in *device_status. */
+MXF8_API mxf8_status mxfp8_get_status(const void* work, void* stream, int32_t* device_status);
+
+/* Static description of a status code. */
+MXF8_API const char* mxfp8_status_string(int32_t status);
+
+/* Text of the last CUDA error seen by this thread ("" if none). */
+MXF8_API const char* mxfp8_last_cuda_error(void);
+
+/* 1 if the current device is sm_100 (the only target), else 0. */
+MXF8_API int32_t mxfp8_device_supported(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MXFP8_H */

@@ -1,1 +1,200 @@
-"""MXFP8 quantisation and dropless grouped GEMM for B200 (sm_100a)."""
+"""MXFP8 quantisation and dropless grouped GEMM for B200 (sm_100a).
+
+A thin ctypes binding over ``libmxfp8.so`` (the C ABI in ``include/mxfp8.h``).
+The functions carry the C names and only marshal arguments: PyTorch supplies
+device memory and the current stream, every step runs in the library's CUDA
+kernels.  There is no fallback: if the library is missing or the device is not
+sm_100 the calls raise.
+
+MXFP8 = 32-element blocks sharing one power-of-two scale (opensourcebeat.com,
+"Enabling up to 41% faster pre-training: MXFP8 and DeepEP ...", FAQ), with the
+OCP MX v1.0 E8M0/E4M3 rules; the grouped GEMM runs every expert on its real
+token count (iitak.ru, "NVIDIA ... JAX", Transformer Engine paragraph).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmxfp8.so")
+_LIB = None
+
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_vp = ctypes.c_void_p
+
+MXF8_OK = 0
+MXF8_GEMM_MAX_GROUPS = 256
+STATUS_NAMES = {0: "MXF8_OK", 1: "MXF8_ERR_INVALID_ARG", 2: "MXF8_ERR_ALIGNMENT", 3: "MXF8_ERR_UNSUPPORTED",
+                4: "MXF8_ERR_CUDA", 5: "MXF8_ERR_BAD_OFFSETS", 6: "MXF8_ERR_TIMEOUT"}
+
+EXPORTED = ("mxfp8_rowwise_scale_bytes", "mxfp8_colwise_pitch", "mxfp8_colwise_scale_bytes", "mxfp8_colwise_ld",
+            "mxfp8_workspace_bytes", "mxfp8_quantize_rowwise", "mxfp8_quantize_colwise",
+            "mxfp8_grouped_gemm_fwd", "mxfp8_grouped_gemm_dgrad", "mxfp8_grouped_gemm_wgrad",
+            "mxfp8_get_status", "mxfp8_status_string", "mxfp8_last_cuda_error", "mxfp8_device_supported")
+
+
+class MXFP8Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        detail = ""
+        if _LIB is not None:
+            detail = _LIB.mxfp8_status_string(status).decode()
+            if status == 4:
+                detail += ": " + _LIB.mxfp8_last_cuda_error().decode()
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({detail})")
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libmxfp8.so; raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m mxfp8_grouped_gemm_quantize_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for n in ("mxfp8_rowwise_scale_bytes", "mxfp8_colwise_scale_bytes"):
+            getattr(L, n).restype = _i64
+            getattr(L, n).argtypes = [_i64, _i64, _i32]
+        for n in ("mxfp8_colwise_pitch", "mxfp8_colwise_ld"):
+            getattr(L, n).restype = _i64
+            getattr(L, n).argtypes = [_i64, _i32]
+        L.mxfp8_workspace_bytes.restype = _i64
+        L.mxfp8_workspace_bytes.argtypes = [_i32, _i64, _i64, _i64]
+        L.mxfp8_quantize_rowwise.restype = _i32
+        L.mxfp8_quantize_rowwise.argtypes = [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _i64, _vp]
+        L.mxfp8_quantize_colwise.restype = _i32
+        L.mxfp8_quantize_colwise.argtypes = [_vp, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _i64, _vp]
+        for n in ("mxfp8_grouped_gemm_fwd", "mxfp8_grouped_gemm_dgrad", "mxfp8_grouped_gemm_wgrad"):
+            getattr(L, n).restype = _i32
+            getattr(L, n).argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp, _vp, _i64, _vp]
+        L.mxfp8_get_status.restype = _i32
+        L.mxfp8_get_status.argtypes = [_vp, _vp, ctypes.POINTER(_i32)]
+        L.mxfp8_status_string.restype = ctypes.c_char_p
+        L.mxfp8_status_string.argtypes = [_i32]
+        L.mxfp8_last_cuda_error.restype = ctypes.c_char_p
+        L.mxfp8_device_supported.restype = _i32
+        _LIB = L
+    return _LIB
+
+
+def _check(status: int, where: str):
+    if status != MXF8_OK:
+        raise MXFP8Error(status, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    assert t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors"
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _groups(offs: torch.Tensor | None) -> int:
+    if offs is None:
+        return 1
+    assert offs.dtype == torch.int32 and offs.is_cuda
+    return offs.numel() - 1
+
+
+# ------------------------------------------------------------------ sizes
+def mxfp8_rowwise_scale_bytes(rows: int, cols: int, num_groups: int = 1) -> int:
+    return lib().mxfp8_rowwise_scale_bytes(rows, cols, num_groups)
+
+
+def mxfp8_colwise_pitch(rows: int, num_groups: int = 1) -> int:
+    return lib().mxfp8_colwise_pitch(rows, num_groups)
+
+
+def mxfp8_colwise_scale_bytes(rows: int, cols: int, num_groups: int = 1) -> int:
+    return lib().mxfp8_colwise_scale_bytes(rows, cols, num_groups)
+
+
+def mxfp8_colwise_ld(rows: int, num_groups: int = 1) -> int:
+    return lib().mxfp8_colwise_ld(rows, num_groups)
+
+
+def mxfp8_workspace_bytes(num_groups: int, M: int, N: int, K: int) -> int:
+    return lib().mxfp8_workspace_bytes(num_groups, M, N, K)
+
+
+def _u8(n: int, device) -> torch.Tensor:
+    return torch.empty(max(int(n), 16), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------ quantisers
+def mxfp8_quantize_rowwise(x: torch.Tensor, offs: torch.Tensor | None = None, q=None, scales=None, stream=None):
+    """x: bf16 [rows, cols] -> (q uint8 [rows, cols], scales uint8 atoms)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    R, C = x.shape
+    G = _groups(offs)
+    q = q if q is not None else torch.empty((R, C), dtype=torch.uint8, device=x.device)
+    scales = scales if scales is not None else _u8(mxfp8_rowwise_scale_bytes(R, C, G), x.device)
+    _check(lib().mxfp8_quantize_rowwise(_ptr(x), R, C, _ptr(offs), G, _ptr(q), _ptr(scales), scales.numel(),
+                                        _stream(stream)), "mxfp8_quantize_rowwise")
+    return q, scales
+
+
+def mxfp8_quantize_colwise(x: torch.Tensor, offs: torch.Tensor | None = None, qT=None, scales=None, stream=None):
+    """x: bf16 [rows, cols] -> (qT uint8 [cols, ldT], scales uint8 atoms)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    R, C = x.shape
+    G = _groups(offs)
+    ld = mxfp8_colwise_ld(R, G)
+    qT = qT if qT is not None else torch.empty((C, ld), dtype=torch.uint8, device=x.device)
+    scales = scales if scales is not None else _u8(mxfp8_colwise_scale_bytes(R, C, G), x.device)
+    _check(lib().mxfp8_quantize_colwise(_ptr(x), R, C, _ptr(offs), G, _ptr(qT), ld, _ptr(scales), scales.numel(),
+                                        _stream(stream)), "mxfp8_quantize_colwise")
+    return qT, scales
+
+
+# ------------------------------------------------------------------ grouped GEMMs
+def new_workspace(E: int, M: int, N: int, K: int, device="cuda") -> torch.Tensor:
+    return torch.zeros(mxfp8_workspace_bytes(E, M, N, K), dtype=torch.uint8, device=device)
+
+
+def _gemm(fn: str, a, as_, b, bs, offs, M, N, K, out, work, stream):
+    E = _groups(offs)
+    work = work if work is not None else new_workspace(E, M, N, K, out.device)
+    _check(getattr(lib(), fn)(_ptr(a), _ptr(as_), as_.numel(), _ptr(b), _ptr(bs), bs.numel(), _ptr(offs), E,
+                              M, N, K, _ptr(out), _ptr(work), work.numel(), _stream(stream)), fn)
+    return out
+
+
+def mxfp8_grouped_gemm_fwd(xq, xs, wq, ws, offs, N: int, out=None, work=None, stream=None):
+    """Y[M, N] = X_e W_e^T per expert.  xq/xs rowwise(X, offs); wq/ws rowwise(W as [E*N, K])."""
+    M, K = xq.shape
+    out = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    return _gemm("mxfp8_grouped_gemm_fwd", xq, xs, wq, ws, offs, M, N, K, out, work, stream)
+
+
+def mxfp8_grouped_gemm_dgrad(dyq, dys, wqT, wsT, offs, K: int, out=None, work=None, stream=None):
+    """dX[M, K] = dY_e W_e.  dyq/dys rowwise(dY, offs); wqT/wsT colwise(W as [E*N, K])."""
+    M, N = dyq.shape
+    out = out if out is not None else torch.empty((M, K), dtype=torch.bfloat16, device=dyq.device)
+    return _gemm("mxfp8_grouped_gemm_dgrad", dyq, dys, wqT, wsT, offs, M, N, K, out, work, stream)
+
+
+def mxfp8_grouped_gemm_wgrad(dyqT, dysT, xqT, xsT, offs, M: int, out=None, work=None, stream=None):
+    """dW[E, N, K] = dY_e^T X_e.  dyqT/dysT colwise(dY, offs); xqT/xsT colwise(X, offs)."""
+    N, K = dyqT.shape[0], xqT.shape[0]
+    E = _groups(offs)
+    out = out if out is not None else torch.empty((E, N, K), dtype=torch.bfloat16, device=dyqT.device)
+    return _gemm("mxfp8_grouped_gemm_wgrad", dyqT, dysT, xqT, xsT, offs, M, N, K, out, work, stream)
+
+
+def mxfp8_get_status(work: torch.Tensor, stream=None) -> int:
+    st = _i32(0)
+    _check(lib().mxfp8_get_status(_ptr(work), _stream(stream), ctypes.byref(st)), "mxfp8_get_status")
+    return int(st.value)
+
+
+def mxfp8_device_supported() -> bool:
+    return bool(lib().mxfp8_device_supported())

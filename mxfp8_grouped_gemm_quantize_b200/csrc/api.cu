@@ -1,0 +1,245 @@
+// api.cu -- the extern "C" entry points declared in include/mxfp8.h: argument
+// checks, workspace status handling and kernel launches.  No entry point
+// allocates device memory.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+
+#include "launch.h"
+#include "mxfp8.h"
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;   // a pipeline wait gives up after 2 s
+constexpr int64_t kWorkspaceBytes = 256;                 // status word + reserve
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t round_up(int64_t a, int64_t b) { return cdiv(a, b) * b; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t blocks128_bound(int64_t rows, int32_t G) { return rows <= 0 ? 0 : cdiv(rows, 128) + G - 1; }
+
+mxf8_status cuda_fail(cudaError_t e, const char* where, const char* detail = nullptr) {
+  std::snprintf(g_last_error, sizeof g_last_error, "%s: %s%s%s", where, cudaGetErrorString(e),
+                detail ? " -- " : "", detail ? detail : "");
+  return MXF8_ERR_CUDA;
+}
+
+// Only sm_100 parts carry the tcgen05 instructions this library is built for.
+mxf8_status check_device() {
+  static int cached[64];   // 0 unknown, 1 supported, 2 unsupported
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return MXF8_ERR_UNSUPPORTED;
+  if (cached[dev] == 0) {
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return cached[dev] == 1 ? MXF8_OK : MXF8_ERR_UNSUPPORTED;
+}
+
+mxf8_status check_quant_args(const uint16_t* x, int64_t rows, int64_t cols, int32_t G, const void* q,
+                             const void* scales, int64_t scale_bytes, int64_t need) {
+  if (rows < 0 || cols <= 0 || cols % 32 != 0 || G < 1) return MXF8_ERR_INVALID_ARG;
+  if ((rows > 0 && (!x || !q)) || !scales) return MXF8_ERR_INVALID_ARG;   // no rows: x and q may be empty
+  if (rows > (int64_t(1) << 31) - 1 || cols > int64_t(65535) * 128) return MXF8_ERR_INVALID_ARG;
+  if (scale_bytes < need) return MXF8_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(scales)) return MXF8_ERR_ALIGNMENT;
+  return MXF8_OK;
+}
+
+struct GemmCheck {
+  const uint8_t* a; const uint8_t* as; int64_t as_bytes;
+  const uint8_t* b; const uint8_t* bs; int64_t bs_bytes;
+  const int32_t* offs; int32_t E; int64_t M, N, K;
+  const void* out; void* work; int64_t work_bytes;
+};
+
+mxf8_status check_gemm_args(const GemmCheck& c) {
+  // With no rows the row-indexed buffers (a for fwd/dgrad, out) may be empty.
+  if ((c.M > 0 && (!c.a || !c.out)) || !c.as || !c.b || !c.bs || !c.offs || !c.work) return MXF8_ERR_INVALID_ARG;
+  if (c.E < 1 || c.E > MXF8_GEMM_MAX_GROUPS) return MXF8_ERR_INVALID_ARG;
+  if (c.M < 0 || c.M > (int64_t(1) << 30) || c.N <= 0 || c.K <= 0) return MXF8_ERR_INVALID_ARG;
+  if (c.N % 128 != 0 || c.K % 32 != 0) return MXF8_ERR_INVALID_ARG;
+  if (int64_t(c.E) * c.N > (int64_t(1) << 30) || c.K > (int64_t(1) << 30)) return MXF8_ERR_INVALID_ARG;
+  if (c.work_bytes < kWorkspaceBytes) return MXF8_ERR_INVALID_ARG;
+  if (!aligned16(c.a) || !aligned16(c.as) || !aligned16(c.b) || !aligned16(c.bs) || !aligned16(c.out) ||
+      !aligned16(c.work))
+    return MXF8_ERR_ALIGNMENT;
+  return MXF8_OK;
+}
+
+mxf8_status run_gemm(mxf8::GemmArgs& g, void* work, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  g.status = static_cast<int32_t*>(work);
+  g.timeout_ns = kDefaultTimeoutNs;
+  cudaError_t e = cudaMemsetAsync(work, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  const char* detail = nullptr;
+  e = mxf8::launch_grouped_gemm(g, st, &detail);
+  if (e != cudaSuccess) return cuda_fail(e, "grouped_gemm launch", detail);
+  return MXF8_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t mxfp8_rowwise_scale_bytes(int64_t rows, int64_t cols, int32_t num_groups) {
+  if (rows < 0 || cols <= 0 || num_groups < 1) return 0;
+  return blocks128_bound(rows, num_groups) * cdiv(cols, 128) * 512;
+}
+
+int64_t mxfp8_colwise_pitch(int64_t rows, int32_t num_groups) {
+  if (rows < 0 || num_groups < 1) return 0;
+  return blocks128_bound(rows, num_groups);
+}
+
+int64_t mxfp8_colwise_scale_bytes(int64_t rows, int64_t cols, int32_t num_groups) {
+  if (rows < 0 || cols <= 0 || num_groups < 1) return 0;
+  return cdiv(cols, 128) * mxfp8_colwise_pitch(rows, num_groups) * 512;
+}
+
+int64_t mxfp8_colwise_ld(int64_t rows, int32_t num_groups) {
+  if (rows < 0 || num_groups < 1) return 0;
+  const int64_t ld = round_up(round_up(rows, 32) + 32 * int64_t(num_groups - 1), 128);
+  return ld < 128 ? 128 : ld;
+}
+
+int64_t mxfp8_workspace_bytes(int32_t num_groups, int64_t M, int64_t N, int64_t K) {
+  (void)num_groups; (void)M; (void)N; (void)K;
+  return kWorkspaceBytes;
+}
+
+mxf8_status mxfp8_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols, const int32_t* d_offs,
+                                   int32_t num_groups, uint8_t* q, uint8_t* scales, int64_t scale_bytes,
+                                   void* stream) {
+  mxf8_status s = check_quant_args(x, rows, cols, num_groups, q, scales, scale_bytes,
+                                   mxfp8_rowwise_scale_bytes(rows, cols, num_groups));
+  if (s != MXF8_OK) return s;
+  if (!d_offs && num_groups != 1) return MXF8_ERR_INVALID_ARG;
+  if ((s = check_device()) != MXF8_OK) return s;
+  cudaError_t e = mxf8::launch_quantize_rowwise(x, rows, cols, d_offs, num_groups, q, scales,
+                                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "quantize_rowwise launch");
+}
+
+mxf8_status mxfp8_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols, const int32_t* d_offs,
+                                   int32_t num_groups, uint8_t* qT, int64_t ldT, uint8_t* scalesT,
+                                   int64_t scale_bytes, void* stream) {
+  mxf8_status s = check_quant_args(x, rows, cols, num_groups, qT, scalesT, scale_bytes,
+                                   mxfp8_colwise_scale_bytes(rows, cols, num_groups));
+  if (s != MXF8_OK) return s;
+  if (!d_offs && num_groups != 1) return MXF8_ERR_INVALID_ARG;
+  if (ldT != mxfp8_colwise_ld(rows, num_groups)) return MXF8_ERR_INVALID_ARG;
+  if ((s = check_device()) != MXF8_OK) return s;
+  cudaError_t e = mxf8::launch_quantize_colwise(x, rows, cols, d_offs, num_groups, qT, ldT, scalesT,
+                                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "quantize_colwise launch");
+}
+
+mxf8_status mxfp8_grouped_gemm_fwd(const uint8_t* xq, const uint8_t* xs, int64_t xs_bytes, const uint8_t* wq,
+                                   const uint8_t* ws, int64_t ws_bytes, const int32_t* d_offs, int32_t E,
+                                   int64_t M, int64_t N, int64_t K, uint16_t* y, void* work,
+                                   int64_t work_bytes, void* stream) {
+  mxf8_status s = check_gemm_args({xq, xs, xs_bytes, wq, ws, ws_bytes, d_offs, E, M, N, K, y, work, work_bytes});
+  if (s != MXF8_OK) return s;
+  if (xs_bytes < mxfp8_rowwise_scale_bytes(M, K, E) || ws_bytes < mxfp8_rowwise_scale_bytes(E * N, K, 1))
+    return MXF8_ERR_INVALID_ARG;
+  if ((s = check_device()) != MXF8_OK) return s;
+  if (M == 0) return cudaMemsetAsync(work, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) == cudaSuccess
+                         ? MXF8_OK : cuda_fail(cudaGetLastError(), "cudaMemsetAsync(status)");
+  mxf8::GemmArgs g{};
+  g.mode = mxf8::kFwd; g.E = E; g.M = M; g.N = N; g.K = K; g.offs = d_offs;
+  g.a = xq; g.lda = K; g.a_rows = M; g.a_cols = K;
+  g.b = wq; g.ldb = K; g.b_rows = E * N; g.b_cols = K;
+  g.sfa = xs; g.sfa_pitch = cdiv(K, 128); g.sfa_atoms = xs_bytes / 512;
+  g.sfb = ws; g.sfb_pitch = cdiv(K, 128); g.sfb_atoms = ws_bytes / 512;
+  g.out = y;
+  return run_gemm(g, work, stream);
+}
+
+mxf8_status mxfp8_grouped_gemm_dgrad(const uint8_t* dyq, const uint8_t* dys, int64_t dys_bytes,
+                                     const uint8_t* wqT, const uint8_t* wsT, int64_t wsT_bytes,
+                                     const int32_t* d_offs, int32_t E, int64_t M, int64_t N, int64_t K,
+                                     uint16_t* dx, void* work, int64_t work_bytes, void* stream) {
+  mxf8_status s =
+      check_gemm_args({dyq, dys, dys_bytes, wqT, wsT, wsT_bytes, d_offs, E, M, N, K, dx, work, work_bytes});
+  if (s != MXF8_OK) return s;
+  if (dys_bytes < mxfp8_rowwise_scale_bytes(M, N, E) || wsT_bytes < mxfp8_colwise_scale_bytes(E * N, K, 1))
+    return MXF8_ERR_INVALID_ARG;
+  if ((s = check_device()) != MXF8_OK) return s;
+  if (M == 0) return cudaMemsetAsync(work, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) == cudaSuccess
+                         ? MXF8_OK : cuda_fail(cudaGetLastError(), "cudaMemsetAsync(status)");
+  const int64_t ldw = mxfp8_colwise_ld(E * N, 1);
+  mxf8::GemmArgs g{};
+  g.mode = mxf8::kDgrad; g.E = E; g.M = M; g.N = N; g.K = K; g.offs = d_offs;
+  g.a = dyq; g.lda = N; g.a_rows = M; g.a_cols = N;
+  g.b = wqT; g.ldb = ldw; g.b_rows = K; g.b_cols = ldw;
+  g.sfa = dys; g.sfa_pitch = cdiv(N, 128); g.sfa_atoms = dys_bytes / 512;
+  g.sfb = wsT; g.sfb_pitch = mxfp8_colwise_pitch(E * N, 1); g.sfb_atoms = wsT_bytes / 512;
+  g.out = dx;
+  return run_gemm(g, work, stream);
+}
+
+mxf8_status mxfp8_grouped_gemm_wgrad(const uint8_t* dyqT, const uint8_t* dysT, int64_t dysT_bytes,
+                                     const uint8_t* xqT, const uint8_t* xsT, int64_t xsT_bytes,
+                                     const int32_t* d_offs, int32_t E, int64_t M, int64_t N, int64_t K,
+                                     uint16_t* dw, void* work, int64_t work_bytes, void* stream) {
+  mxf8_status s =
+      check_gemm_args({dyqT, dysT, dysT_bytes, xqT, xsT, xsT_bytes, d_offs, E, M, N, K, dw, work, work_bytes});
+  if (s != MXF8_OK) return s;
+  if (dysT_bytes < mxfp8_colwise_scale_bytes(M, N, E) || xsT_bytes < mxfp8_colwise_scale_bytes(M, K, E))
+    return MXF8_ERR_INVALID_ARG;
+  if ((s = check_device()) != MXF8_OK) return s;
+  const int64_t ldt = mxfp8_colwise_ld(M, E);
+  mxf8::GemmArgs g{};
+  g.mode = mxf8::kWgrad; g.E = E; g.M = M; g.N = N; g.K = K; g.offs = d_offs;
+  g.a = dyqT; g.lda = ldt; g.a_rows = N; g.a_cols = ldt;
+  g.b = xqT; g.ldb = ldt; g.b_rows = K; g.b_cols = ldt;
+  const int64_t pitch = mxfp8_colwise_pitch(M, E);
+  g.sfa = dysT; g.sfa_pitch = pitch; g.sfa_atoms = dysT_bytes / 512;
+  g.sfb = xsT; g.sfb_pitch = pitch; g.sfb_atoms = xsT_bytes / 512;
+  g.out = dw;
+  if (g.sfa_atoms < 1 || g.sfb_atoms < 1) {
+    // M = 0: no scale atoms exist; point at the (unread) code buffers instead.
+    g.sfa = dyqT; g.sfb = xqT; g.sfa_atoms = g.sfb_atoms = 1;
+  }
+  return run_gemm(g, work, stream);
+}
+
+mxf8_status mxfp8_get_status(const void* work, void* stream, int32_t* device_status) {
+  if (!work || !device_status) return MXF8_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  e = cudaMemcpy(device_status, work, sizeof(int32_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
+  return MXF8_OK;
+}
+
+const char* mxfp8_status_string(int32_t status) {
+  switch (status) {
+    case MXF8_OK: return "ok";
+    case MXF8_ERR_INVALID_ARG: return "invalid argument";
+    case MXF8_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case MXF8_ERR_UNSUPPORTED: return "device is not sm_100";
+    case MXF8_ERR_CUDA: return "CUDA error";
+    case MXF8_ERR_BAD_OFFSETS: return "group offsets are not a valid prefix";
+    case MXF8_ERR_TIMEOUT: return "device pipeline wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* mxfp8_last_cuda_error(void) { return g_last_error; }
+
+int32_t mxfp8_device_supported(void) { return check_device() == MXF8_OK ? 1 : 0; }
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// groups.cuh -- on-device reading of the ragged group offsets.
+//
+// Every kernel derives what it needs from the int32 offsets itself (no host
+// round trip): offsets are clamped to [0, rows] and made non-decreasing, so
+// that any input, valid or not, keeps every access in bounds.  Per group g
+// (m_g = offs'[g+1] - offs'[g]):
+//   RB_g = sum over h < g of ceil(m_h / 128)   (128-row blocks; scale atoms)
+//   P_g  = sum over h < g of round_up(m_h, 32) (32-padded rows; colwise codes)
+#pragma once
+#include <cstdint>
+
+namespace mxf8 {
+
+struct GroupBlock {
+  int32_t g;       // group index, -1 if the block index is past the last block
+  int64_t lo;      // first row of the group
+  int64_t m;       // rows in the group
+  int64_t rb;      // RB_g
+  int64_t p;       // P_g
+};
+
+__device__ __forceinline__ int64_t clamp_off(const int32_t* offs, int32_t h, int64_t rows) {
+  int64_t v = offs ? static_cast<int64_t>(__ldg(offs + h)) : (h == 0 ? 0 : rows);
+  return v < 0 ? 0 : (v > rows ? rows : v);
+}
+
+// Warp-cooperative lookup of the group owning padded 128-row block `pb`
+// (blocks ordered group by group).  Every lane returns the same result.
+__device__ __forceinline__ GroupBlock warp_find_block(const int32_t* offs, int32_t G, int64_t rows,
+                                                      int64_t pb) {
+  const int lane = threadIdx.x & 31;
+  int64_t o_prev = clamp_off(offs, 0, rows);
+  int64_t carry_rb = 0, carry_p = 0;
+  for (int32_t base = 0; base < G; base += 32) {
+    const int32_t h = base + lane;
+    int64_t v = (h < G) ? clamp_off(offs, h + 1, rows) : 0;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      int64_t t = __shfl_up_sync(0xffffffffu, v, d);
+      if (lane >= d) v = v > t ? v : t;
+    }
+    const int64_t hi = v > o_prev ? v : o_prev;           // offs'[h + 1]
+    int64_t lo = __shfl_up_sync(0xffffffffu, hi, 1);
+    if (lane == 0) lo = o_prev;                           // offs'[h]
+    const int64_t m = (h < G) ? hi - lo : 0;
+    const int64_t nb = (m + 127) / 128, np = (m + 31) / 32 * 32;
+    int64_t snb = nb, snp = np;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      int64_t a = __shfl_up_sync(0xffffffffu, snb, d);
+      int64_t b = __shfl_up_sync(0xffffffffu, snp, d);
+      if (lane >= d) { snb += a; snp += b; }
+    }
+    const int64_t rb0 = carry_rb + snb - nb, p0 = carry_p + snp - np;
+    const bool found = (h < G) && nb > 0 && pb >= rb0 && pb < rb0 + nb;
+    const uint32_t ball = __ballot_sync(0xffffffffu, found);
+    if (ball) {
+      const int src = __ffs(ball) - 1;
+      GroupBlock r;
+      r.g = __shfl_sync(0xffffffffu, h, src);
+      r.lo = __shfl_sync(0xffffffffu, lo, src);
+      r.m = __shfl_sync(0xffffffffu, m, src);
+      r.rb = __shfl_sync(0xffffffffu, rb0, src);
+      r.p = __shfl_sync(0xffffffffu, p0, src);
+      return r;
+    }
+    carry_rb = __shfl_sync(0xffffffffu, carry_rb + snb, 31);
+    carry_p = __shfl_sync(0xffffffffu, carry_p + snp, 31);
+    o_prev = __shfl_sync(0xffffffffu, hi, 31);
+  }
+  GroupBlock none;
+  none.g = -1; none.lo = 0; none.m = 0; none.rb = 0; none.p = 0;
+  return none;
+}
+
+}  // namespace mxf8

@@ -1,0 +1,62 @@
+"""The C-ABI library loads and exports every entry point include/mxfp8.h
+declares (CPU only: no compute call is made); host-side size helpers agree
+with the layout definition."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(mxfp8_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mxfp8_grouped_gemm_quantize_b200 import build
+    build.build()
+    import mxfp8_grouped_gemm_quantize_b200 as m
+    return m.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("mxfp8_quantize_rowwise", "mxfp8_quantize_colwise", "mxfp8_grouped_gemm_fwd",
+              "mxfp8_grouped_gemm_dgrad", "mxfp8_grouped_gemm_wgrad", "mxfp8_get_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_python_binding_names_match_the_header():
+    import mxfp8_grouped_gemm_quantize_b200 as m
+    assert set(m.EXPORTED) == set(_declared())
+
+
+@pytest.mark.parametrize("R,C,G", [(0, 32, 1), (64, 256, 4), (49152, 2048, 64), (16384, 7168, 32), (1, 32, 1)])
+def test_size_helpers_agree_with_the_layout_definition(lib, R, C, G):
+    import mxfp8_grouped_gemm_quantize_b200 as m
+    assert m.mxfp8_colwise_ld(R, G) == oracle.colwise_ld(R, G)
+    assert m.mxfp8_colwise_pitch(R, G) == oracle.colwise_pitch(R, G)
+    assert m.mxfp8_rowwise_scale_bytes(R, C, G) == oracle.rowwise_scale_bytes(R, C, G)
+    assert m.mxfp8_colwise_scale_bytes(R, C, G) == oracle.colwise_scale_bytes(R, C, G)
+
+
+def test_status_strings(lib):
+    import mxfp8_grouped_gemm_quantize_b200 as m
+    for code in range(7):
+        assert m.lib().mxfp8_status_string(code)
