@@ -319,9 +319,11 @@ def _cpu_sample(w: wl.Workload, budget_s: float):
     W2 = W.reshape(w.E * layer.N, layer.K)
     offs = w.offsets
     N, K, M = layer.N, layer.K, w.M
+    cal = min(M, 512)
+    oracle.baseline_fwd_f32(X, W2, offs, N, 0, 16)                    # thread start-up
     t0 = time.perf_counter()
-    oracle.baseline_fwd_f32(X, W2, offs, N, 0, 8)
-    rate = 2 * 8 * N * K / max(time.perf_counter() - t0, 1e-6)      # FLOP/s estimate
+    oracle.baseline_fwd_f32(X, W2, offs, N, 0, cal)
+    rate = 2 * cal * N * K / max(time.perf_counter() - t0, 1e-6)      # FLOP/s estimate
     rows = int(max(1, min(M, budget_s / 3 * rate / (2 * N * K))))
     # wgrad sample: output rows n in [0, nr) for every expert (work 2*M*nr*K)
     nr = int(max(1, min(N, budget_s / 3 * rate / (2 * M * K))))
