@@ -173,6 +173,31 @@ MXF8_API mxf8_status mxfp8_grouped_gemm_wgrad(const uint8_t* dyqT, const uint8_t
                                      int64_t K, uint16_t* dw, void* work, int64_t work_bytes,
                                      void* stream);
 
+/* Forward grouped GEMM that allocates nothing and takes no workspace.
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot call cudaMalloc (for example a plugin inside an engine that owns
+ * the device-memory budget, or a path where an allocation's implicit device
+ * synchronisation is not acceptable).  Arguments and results are those of
+ * mxfp8_grouped_gemm_fwd without work/work_bytes; the scratch is a static
+ * device array of MXF8_NOALLOC_SCRATCH_BYTES inside the library, held by
+ * every GPU that loads the library until the process exits.
+ *   - The first call on a device looks up that array's device address (with
+ *     the device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array; its status word is cleared
+ *     at the start of each call, but calls that overlap on the GPU (other
+ *     streams, other host threads) race on it.
+ *   - host_status (nullable, HOST pointer): when given, the call synchronises
+ *     `stream` and stores the device status (an mxf8_status) there.
+ *   - Returns MXF8_ERR_INVALID_ARG if the call would need more scratch than
+ *     MXF8_NOALLOC_SCRATCH_BYTES, plus every error mxfp8_grouped_gemm_fwd
+ *     returns.  It calls no allocating routine. */
+#define MXF8_NOALLOC_SCRATCH_BYTES 4096
+MXF8_API mxf8_status mxfp8_grouped_gemm_fwd_noalloc(const uint8_t* xq, const uint8_t* xs, int64_t xs_bytes,
+                                                    const uint8_t* wq, const uint8_t* ws, int64_t ws_bytes,
+                                                    const int32_t* d_offs, int32_t E, int64_t M, int64_t N,
+                                                    int64_t K, uint16_t* y, int32_t* host_status,
+                                                    void* stream);
+
 /* ---------------------------------------------------------------- status */
 
 /* Synchronises `stream`, then stores the device status of the last GEMM that

@@ -34,7 +34,8 @@ STATUS_NAMES = {0: "MXF8_OK", 1: "MXF8_ERR_INVALID_ARG", 2: "MXF8_ERR_ALIGNMENT"
 EXPORTED = ("mxfp8_rowwise_scale_bytes", "mxfp8_colwise_pitch", "mxfp8_colwise_scale_bytes", "mxfp8_colwise_ld",
             "mxfp8_workspace_bytes", "mxfp8_quantize_rowwise", "mxfp8_quantize_colwise",
             "mxfp8_grouped_gemm_fwd", "mxfp8_grouped_gemm_dgrad", "mxfp8_grouped_gemm_wgrad",
-            "mxfp8_get_status", "mxfp8_status_string", "mxfp8_last_cuda_error", "mxfp8_device_supported")
+            "mxfp8_get_status", "mxfp8_status_string", "mxfp8_last_cuda_error", "mxfp8_device_supported",
+            "mxfp8_grouped_gemm_fwd_noalloc")
 
 
 class MXFP8Error(RuntimeError):
@@ -70,6 +71,9 @@ def lib() -> ctypes.CDLL:
         for n in ("mxfp8_grouped_gemm_fwd", "mxfp8_grouped_gemm_dgrad", "mxfp8_grouped_gemm_wgrad"):
             getattr(L, n).restype = _i32
             getattr(L, n).argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp, _vp, _i64, _vp]
+        L.mxfp8_grouped_gemm_fwd_noalloc.restype = _i32
+        L.mxfp8_grouped_gemm_fwd_noalloc.argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp,
+                                                     ctypes.POINTER(_i32), _vp]
         L.mxfp8_get_status.restype = _i32
         L.mxfp8_get_status.argtypes = [_vp, _vp, ctypes.POINTER(_i32)]
         L.mxfp8_status_string.restype = ctypes.c_char_p
@@ -188,6 +192,21 @@ def mxfp8_grouped_gemm_wgrad(dyqT, dysT, xqT, xsT, offs, M: int, out=None, work=
     E = _groups(offs)
     out = out if out is not None else torch.empty((E, N, K), dtype=torch.bfloat16, device=dyqT.device)
     return _gemm("mxfp8_grouped_gemm_wgrad", dyqT, dysT, xqT, xsT, offs, M, N, K, out, work, stream)
+
+
+def mxfp8_grouped_gemm_fwd_noalloc(xq, xs, wq, ws, offs, N: int, out=None, stream=None, want_status=False):
+    """Forward grouped GEMM with the library's static scratch instead of a
+    workspace, for callers that cannot allocate device memory.  With
+    want_status the call synchronises the stream and returns (out, status)."""
+    M, K = xq.shape
+    E = _groups(offs)
+    out = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    st = _i32(-1)
+    _check(lib().mxfp8_grouped_gemm_fwd_noalloc(_ptr(xq), _ptr(xs), xs.numel(), _ptr(wq), _ptr(ws), ws.numel(),
+                                                _ptr(offs), E, M, N, K, _ptr(out),
+                                                ctypes.byref(st) if want_status else None, _stream(stream)),
+           "mxfp8_grouped_gemm_fwd_noalloc")
+    return (out, int(st.value)) if want_status else out
 
 
 def mxfp8_get_status(work: torch.Tensor, stream=None) -> int:
