@@ -12,27 +12,31 @@
 // FAQ), so one block-scaled MMA instruction (kind::mxf8f6f4, K = 32) applies
 // the scales in hardware and accumulates in fp32 tensor memory.
 //
-// Structure (one CTA per SM, 192 threads):
-//   warp 0   TMA producer: per 128-wide K block, A 128x128 and B 256x128 code
-//            tiles (128-byte swizzle) and three 512-byte scale atoms into a
-//            4-stage shared-memory ring.
-//   warp 1   allocates 512 tensor-memory columns; one thread copies the scale
-//            atoms to tensor memory (tcgen05.cp 32x128b.warpx4) and issues the
-//            128x256x32 MMAs; tcgen05.commit releases ring stages and signals
-//            a finished accumulator.
-//   warps 2-5 epilogue: tensor memory -> registers -> bf16 -> shared (swizzled)
-//            -> coalesced 16-byte global stores, masked to the group's real
-//            rows and the matrix columns.
-// Two 128x256 fp32 accumulators overlap in 64 columns (0..255 and 192..447),
-// which leaves columns 448..511 for per-stage scale factors; the epilogue
-// drains the shared 64 columns first and then releases the accumulator, so
-// the next tile's MMAs overlap the rest of the epilogue.
+// One kernel template, CG = CTAs per MMA:
+//   CG = 2: CTA pairs (clusters of 2) issue 256x256x32 MMAs
+//     (cta_group::2).  Each CTA stages its own 128 rows of A, half of B's 256
+//     rows and all 256 rows of B's scales; the pair computes a 256x256 output
+//     tile, 128 rows in each CTA's tensor memory.  Per CTA this moves 2/3 of
+//     the operand bytes per FLOP of a 1-CTA 128x256 tile.
+//   CG = 1: 128x256x32 MMAs (cta_group::1), one CTA per tile.
+// Roles per CTA (192 threads): warp 0 TMA producer; warp 1 allocates the 512
+// tensor-memory columns, and (in the leader CTA) one thread copies scale
+// atoms to tensor memory and issues the MMAs; warps 2-5 drain the
+// accumulator: tcgen05.ld -> bf16 -> 128-byte-swizzled shared stage -> TMA
+// bulk-tensor store (plain masked stores only for a group's ragged slice).
+// Two 128x256 fp32 accumulators overlap in 64 columns (0..255 and 192..447);
+// the epilogue drains the shared columns first and releases the accumulator,
+// so the next tile's MMAs overlap the rest of the drain.  Columns 448.. hold
+// one scale-factor set per pipeline stage.
 // The tile schedule is built on the device from the group offsets at kernel
-// start (no host synchronisation); tiles are dealt round-robin to the CTAs.
-// Every wait is bounded: on timeout the kernel records MXF8_ERR_TIMEOUT,
-// drains its in-flight copies and MMAs, frees tensor memory and exits.
+// start (no host synchronisation); tiles are dealt round-robin.  Every wait is
+// bounded: on timeout the kernel records MXF8_ERR_TIMEOUT, drains its
+// in-flight copies and MMAs, frees tensor memory and exits.
 #include <cuda.h>
 #include <cuda_runtime.h>
+
+#include <cstdlib>
+#include <cstring>
 
 #include "launch.h"
 #include "mxfp8.h"
@@ -41,36 +45,42 @@
 namespace mxf8 {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 128, STAGES = 4;
-constexpr int A_TILE = BM * BK;            // 16 KB of E4M3 codes
-constexpr int B_TILE = BN * BK;            // 32 KB
+constexpr int BM = 128, BN = 256, BK = 128;
 constexpr int SFA_TILE = 512, SFB_TILE = 1024;
-constexpr uint32_t STAGE_TX = A_TILE + B_TILE + SFA_TILE + SFB_TILE;
 constexpr int NUM_THREADS = 192;
-constexpr int EPI_STAGE = 32 * 128;        // per epilogue warp: 32 rows x 64 bf16
+constexpr int EPI_STAGE = 32 * 128;        // one epilogue buffer: 32 rows x 64 bf16, 128B-swizzled
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_STRIDE = 192;       // accumulator 1 starts at column 192
-constexpr uint32_t SF_COL = 448;           // stage s: SFA at 448 + 16 s (4 columns), SFB at +4 (8 columns)
-constexpr uint32_t SF_STRIDE = 16;
+constexpr uint32_t SF_COL = 448;           // stage s: SFA at 448 + 12 s (4 columns), SFB at +4 (8 columns)
+constexpr uint32_t SF_STRIDE = 12;
 constexpr int MAXG = MXF8_GEMM_MAX_GROUPS;
-
-// Shared-memory map (offsets from a 1024-byte aligned base).
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + STAGES * A_TILE;
-constexpr int OFF_SFA = OFF_B + STAGES * B_TILE;
-constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_TILE;
-constexpr int OFF_EPI = OFF_SFB + STAGES * SFB_TILE;
-constexpr int OFF_BAR = OFF_EPI + 4 * EPI_STAGE;
-constexpr int NUM_BARS = 2 * STAGES + 3;   // full[S], empty[S], acc_full, acc_empty, drain
-constexpr int OFF_MISC = OFF_BAR + 128;
-constexpr int OFF_SCHED = OFF_MISC + 64;
+constexpr int PF_DIST = 8;                 // K blocks of L2 prefetch ahead of the TMA loads
 constexpr int SCHED_INTS = 4 * (MAXG + 1);
-constexpr int SMEM_USED = OFF_SCHED + SCHED_INTS * 4;
-constexpr int SMEM_BYTES = SMEM_USED + 1024;   // slack for aligning the base
-static_assert(NUM_BARS * 8 <= 128, "barrier area");
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-static_assert(OFF_B % 1024 == 0 && OFF_SFA % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-static_assert(SF_COL + SF_STRIDE * (STAGES - 1) + 12 <= TMEM_COLS, "scale columns");
+
+constexpr int round_up_c(int a, int b) { return (a + b - 1) / b * b; }
+
+template <int CG>
+struct Cfg {
+  static constexpr int STAGES = CG == 2 ? 5 : 4;
+  static constexpr int B_ROWS = BN / CG;               // B rows staged by each CTA
+  static constexpr int A_TILE = BM * BK;               // 16 KB of E4M3 codes
+  static constexpr int B_TILE = B_ROWS * BK;
+  static constexpr int EPI_BUFS = CG == 2 ? 2 : 1;
+  static constexpr uint32_t STAGE_TX = CG * (A_TILE + B_TILE + SFA_TILE + SFB_TILE);
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_TILE;
+  static constexpr int OFF_SFA = OFF_B + STAGES * B_TILE;
+  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_TILE;
+  static constexpr int OFF_EPI = round_up_c(OFF_SFB + STAGES * SFB_TILE, 1024);
+  static constexpr int OFF_BAR = OFF_EPI + 4 * EPI_BUFS * EPI_STAGE;
+  static constexpr int OFF_MISC = OFF_BAR + 128;
+  static constexpr int OFF_SCHED = OFF_MISC + 64;
+  static constexpr int SMEM_BYTES = OFF_SCHED + SCHED_INTS * 4 + 1024;   // + slack to align the base
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(OFF_B % 1024 == 0 && B_TILE % 1024 == 0 && OFF_EPI % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static_assert(SF_COL + SF_STRIDE * (STAGES - 1) + 12 <= TMEM_COLS, "scale columns");
+  static_assert((2 * STAGES + 3) * 8 <= 128, "barrier area");
+};
 static_assert(ACC_STRIDE + BN <= SF_COL, "accumulators must not reach the scale columns");
 
 struct Params {
@@ -78,10 +88,9 @@ struct Params {
   int32_t E;
   int64_t M, N, K;
   const int32_t* offs;
-  const uint8_t* sfa;
-  const uint8_t* sfb;
-  int64_t sfa_pitch, sfb_pitch, sfa_atoms, sfb_atoms;
-  uint16_t* out;
+  int64_t sfa_pitch, sfb_pitch;        // atoms per atom row of the A / B scale matrices
+  uint16_t* out;                       // output (fwd [M,N], dgrad [M,K], wgrad [E*N,K])
+  int64_t out_ld;                      // output row stride (elements)
   int32_t* status;
   uint64_t timeout_ns;
 };
@@ -95,30 +104,31 @@ struct Sched {
   int32_t* p;       // [E]   P_e: 32-padded rows before group e (colwise code column)
 };
 
+// One CTA's share of a tile.
 struct Tile {
-  int32_t e, mt, nt;
   int32_t kblocks;       // 128-wide K blocks (0: nothing to accumulate)
   int32_t ksteps_last;   // 32-wide MMA steps in the last K block
-  int32_t a_x, a_y, b_x, b_y;           // TMA coordinates of the first K block
-  int64_t sfa_row, sfa_col, sfb_row, sfb_col;   // scale atom (row, column) of the first K block
-  uint16_t* out;         // output element (0, 0) of the tile
-  int64_t ld;            // output row stride (elements)
-  int32_t rows, cols;    // valid rows (<= 128) and columns (<= 256) of the tile
+  int32_t a_x, a_y, b_x, b_y;           // TMA coordinates of the first K block (this CTA's rows)
+  int64_t sfa_atom, sfb_atom0, sfb_atom1;   // scale atoms of the first K block
+  int64_t out_row, out_col;             // output element (row, col) of this CTA's tile corner
+  int32_t rows, cols;    // valid rows (0..128) and columns (<= 256) of this CTA's tile
 };
 
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
-
 __device__ __forceinline__ int32_t cdiv32(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
 
-__device__ __forceinline__ int32_t group_m_tiles(const Params& p, int32_t m) {
-  return p.mode == kWgrad ? cdiv32(p.N, BM) : cdiv32(m, BM);
+template <int CG>
+__device__ __forceinline__ int32_t group_m_units(const Params& p, int32_t m) {
+  return cdiv32(p.mode == kWgrad ? cdiv32(p.N, BM) : cdiv32(m, BM), CG);
 }
 
 __device__ __forceinline__ int32_t n_tiles(const Params& p) {
   return p.mode == kFwd ? cdiv32(p.N, BN) : cdiv32(p.K, BN);
 }
 
-__device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int32_t t) {
+// Tile t (a pair tile when CG = 2) as seen by CTA `rank` of its pair.
+template <int CG>
+__device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int32_t t, uint32_t rank) {
   int32_t lo = 0, hi = p.E - 1;   // last group whose first tile is <= t
   while (lo < hi) {
     const int32_t mid = (lo + hi + 1) >> 1;
@@ -127,52 +137,47 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int
   Tile tl;
   const int32_t e = lo;
   const int32_t row0 = s.off[e], m = s.off[e + 1] - s.off[e];
-  const int32_t mtiles = group_m_tiles(p, m);
+  const int32_t munits = group_m_units<CG>(p, m);
   const int32_t local = t - s.tile0[e];
-  tl.e = e;
-  tl.mt = local % mtiles;
-  tl.nt = local / mtiles;
+  const int32_t mt = CG * (local % munits) + static_cast<int32_t>(rank);   // this CTA's 128-row block
+  const int32_t nt = local / munits;
+  const int32_t b_half = (CG == 2) ? BN / 2 * static_cast<int32_t>(rank) : 0;
   const int64_t L = p.mode == kFwd ? p.K : (p.mode == kDgrad ? p.N : m);
   tl.kblocks = static_cast<int32_t>((L + BK - 1) / BK);
   tl.ksteps_last = tl.kblocks > 0 ? static_cast<int32_t>((L - int64_t(BK) * (tl.kblocks - 1) + 31) / 32) : 0;
+  int64_t sfa_row, sfa_col, sfb_row, sfb_col, out_cols;
   if (p.mode == kFwd) {
-    tl.a_x = 0;            tl.a_y = row0 + BM * tl.mt;
-    tl.b_x = 0;            tl.b_y = static_cast<int32_t>(e * p.N) + BN * tl.nt;
-    tl.sfa_row = s.rb[e] + tl.mt;                 tl.sfa_col = 0;
-    tl.sfb_row = e * (p.N / 128) + 2 * tl.nt;     tl.sfb_col = 0;
-    tl.out = p.out + (int64_t(row0) + BM * tl.mt) * p.N + BN * tl.nt;
-    tl.ld = p.N;
-    tl.rows = min(BM, m - BM * tl.mt);
-    tl.cols = static_cast<int32_t>(min64(BN, p.N - int64_t(BN) * tl.nt));
+    tl.a_x = 0;                              tl.a_y = row0 + BM * mt;
+    tl.b_x = 0;                              tl.b_y = static_cast<int32_t>(e * p.N) + BN * nt + b_half;
+    sfa_row = s.rb[e] + mt;                  sfa_col = 0;
+    sfb_row = e * (p.N / 128) + 2 * nt;      sfb_col = 0;
+    tl.out_row = int64_t(row0) + BM * mt;
+    tl.rows = static_cast<int32_t>(min64(BM, m - BM * mt));
+    out_cols = p.N;
   } else if (p.mode == kDgrad) {
-    tl.a_x = 0;                                   tl.a_y = row0 + BM * tl.mt;
-    tl.b_x = static_cast<int32_t>(e * p.N);       tl.b_y = BN * tl.nt;
-    tl.sfa_row = s.rb[e] + tl.mt;                 tl.sfa_col = 0;
-    tl.sfb_row = 2 * tl.nt;                       tl.sfb_col = e * (p.N / 128);
-    tl.out = p.out + (int64_t(row0) + BM * tl.mt) * p.K + BN * tl.nt;
-    tl.ld = p.K;
-    tl.rows = min(BM, m - BM * tl.mt);
-    tl.cols = static_cast<int32_t>(min64(BN, p.K - int64_t(BN) * tl.nt));
+    tl.a_x = 0;                              tl.a_y = row0 + BM * mt;
+    tl.b_x = static_cast<int32_t>(e * p.N);  tl.b_y = BN * nt + b_half;
+    sfa_row = s.rb[e] + mt;                  sfa_col = 0;
+    sfb_row = 2 * nt;                        sfb_col = e * (p.N / 128);
+    tl.out_row = int64_t(row0) + BM * mt;
+    tl.rows = static_cast<int32_t>(min64(BM, m - BM * mt));
+    out_cols = p.K;
   } else {
-    tl.a_x = s.p[e];       tl.a_y = BM * tl.mt;
-    tl.b_x = s.p[e];       tl.b_y = BN * tl.nt;
-    tl.sfa_row = tl.mt;                           tl.sfa_col = s.rb[e];
-    tl.sfb_row = 2 * tl.nt;                       tl.sfb_col = s.rb[e];
-    tl.out = p.out + int64_t(e) * p.N * p.K + int64_t(BM) * tl.mt * p.K + BN * tl.nt;
-    tl.ld = p.K;
-    tl.rows = static_cast<int32_t>(min64(BM, p.N - int64_t(BM) * tl.mt));
-    tl.cols = static_cast<int32_t>(min64(BN, p.K - int64_t(BN) * tl.nt));
+    tl.a_x = s.p[e];                         tl.a_y = BM * mt;
+    tl.b_x = s.p[e];                         tl.b_y = BN * nt + b_half;
+    sfa_row = mt;                            sfa_col = s.rb[e];
+    sfb_row = 2 * nt;                        sfb_col = s.rb[e];
+    tl.out_row = int64_t(e) * p.N + BM * mt;
+    tl.rows = static_cast<int32_t>(min64(BM, p.N - int64_t(BM) * mt));
+    out_cols = p.K;
   }
+  if (tl.rows < 0) tl.rows = 0;
+  tl.out_col = int64_t(BN) * nt;
+  tl.cols = static_cast<int32_t>(min64(BN, out_cols - tl.out_col));
+  tl.sfa_atom = sfa_row * p.sfa_pitch + sfa_col;
+  tl.sfb_atom0 = sfb_row * p.sfb_pitch + sfb_col;
+  tl.sfb_atom1 = (sfb_row + 1) * p.sfb_pitch + sfb_col;
   return tl;
-}
-
-// Scale atom address, clamped into the buffer: atoms that fall outside it
-// only ever feed masked output rows/columns.
-__device__ __forceinline__ const uint8_t* atom_ptr(const uint8_t* base, int64_t row, int64_t col,
-                                                   int64_t pitch, int64_t atoms) {
-  int64_t a = row * pitch + col;
-  a = a < 0 ? 0 : (a >= atoms ? atoms - 1 : a);
-  return base + a * 512;
 }
 
 __device__ __forceinline__ void record_error(int32_t* status, int32_t code, volatile int* abort) {
@@ -182,6 +187,7 @@ __device__ __forceinline__ void record_error(int32_t* status, int32_t code, vola
 
 // Warp 0: validate the offsets and build the schedule.  Returns the total
 // tile count (0 if the offsets are invalid).
+template <int CG>
 __device__ int32_t build_schedule(const Params& p, const Sched& s) {
   const int lane = threadIdx.x & 31;
   const int32_t ntl = n_tiles(p);
@@ -196,7 +202,7 @@ __device__ int32_t build_schedule(const Params& p, const Sched& s) {
     if (h == p.E - 1 && int64_t(b) != p.M) lbad = true;
     bad |= __any_sync(0xffffffffu, lbad);
     const int32_t m = (h < p.E && !lbad) ? b - a : 0;
-    const int32_t tiles = (h < p.E) ? group_m_tiles(p, m) * ntl : 0;
+    const int32_t tiles = (h < p.E) ? group_m_units<CG>(p, m) * ntl : 0;
     const int32_t nb = (m + BM - 1) / BM, np = (m + 31) / 32 * 32;
     int32_t st = tiles, sr = nb, sp = np;
 #pragma unroll
@@ -224,23 +230,44 @@ __device__ int32_t build_schedule(const Params& p, const Sched& s) {
   return carry_t;
 }
 
+// tcgen05.wait::ld, tied to the registers the outstanding loads write so that
+// no use of them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_regs(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                 "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+                 "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+                 "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
+template <int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const Params p) {
+                    const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
+                    const __grid_constant__ CUtensorMap tmOut, const Params p) {
+  using C = Cfg<CG>;
+  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int32_t unit0 = (CG == 2) ? static_cast<int32_t>(blockIdx.x >> 1) : static_cast<int32_t>(blockIdx.x);
+  const int32_t nunits = (CG == 2) ? static_cast<int32_t>(gridDim.x >> 1) : static_cast<int32_t>(gridDim.x);
 
-  const uint32_t bar0 = smem_addr(smem + OFF_BAR);
+  const uint32_t bar0 = smem_addr(smem + C::OFF_BAR);
   auto full_bar = [&](uint32_t s) { return bar0 + 8 * s; };
   auto empty_bar = [&](uint32_t s) { return bar0 + 8 * (STAGES + s); };
   const uint32_t acc_full = bar0 + 8 * (2 * STAGES);
-  const uint32_t acc_empty = bar0 + 8 * (2 * STAGES + 1);
+  const uint32_t acc_empty = bar0 + 8 * (2 * STAGES + 1);   // used in the leader CTA
   const uint32_t drain_bar = bar0 + 8 * (2 * STAGES + 2);
-  volatile int32_t* misc = reinterpret_cast<volatile int32_t*>(smem + OFF_MISC);
+  volatile int32_t* misc = reinterpret_cast<volatile int32_t*>(smem + C::OFF_MISC);
   // misc[0]: tensor-memory base, misc[1]: abort flag, misc[2]: total tiles
   Sched sc;
-  int32_t* sched = reinterpret_cast<int32_t*>(smem + OFF_SCHED);
+  int32_t* sched = reinterpret_cast<int32_t*>(smem + C::OFF_SCHED);
   sc.tile0 = sched;
   sc.off = sched + (MAXG + 1);
   sc.rb = sched + 2 * (MAXG + 1);
@@ -250,21 +277,30 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     if (lane == 0) {
       for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
       mbar_init(acc_full, 1);
-      mbar_init(acc_empty, 4 * 32);
+      mbar_init(acc_empty, CG * 4 * 32);
       mbar_init(drain_bar, 1);
       fence_barrier_init();
       prefetch_tmap(&tmA);
       prefetch_tmap(&tmB);
+      prefetch_tmap(&tmSFA);
+      prefetch_tmap(&tmSFB);
+      prefetch_tmap(&tmOut);
       misc[1] = 0;
     }
-    const int32_t total = build_schedule(p, sc);
+    const int32_t total = build_schedule<CG>(p, sc);
     if (lane == 0) misc[2] = total;
   } else if (warp == 1) {
-    tmem_alloc(smem_addr(const_cast<int32_t*>(misc)), TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (CG == 2) {
+      tmem_alloc_pair(smem_addr(const_cast<int32_t*>(misc)), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_addr(const_cast<int32_t*>(misc)), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) cluster_sync();   // peer barriers initialised before any cross-CTA signal
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = static_cast<uint32_t>(misc[0]);
   const int32_t total = misc[2];
@@ -274,12 +310,33 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------------------ producer
+      // ------------------------------------------------------------ producer (every CTA)
       uint32_t it = 0;
       bool failed = false;
-      for (int32_t t = blockIdx.x; t < total && !failed; t += gridDim.x) {
-        const Tile tl = decode_tile(p, sc, t);
+      // L2 prefetch cursor running PF_DIST K blocks ahead of the loads, across
+      // tile boundaries, so first touches of A/B tiles (DRAM misses) overlap
+      // the ring's in-flight loads.
+      int32_t pf_t = unit0, pf_kb = 0;
+      Tile pf_tl;
+      if (pf_t < total) pf_tl = decode_tile<CG>(p, sc, pf_t, rank);
+      auto advance_prefetch = [&]() {
+        while (pf_t < total) {
+          if (pf_kb < pf_tl.kblocks) {
+            tma_prefetch_2d(&tmA, pf_tl.a_x + BK * pf_kb, pf_tl.a_y);
+            tma_prefetch_2d(&tmB, pf_tl.b_x + BK * pf_kb, pf_tl.b_y);
+            ++pf_kb;
+            return;
+          }
+          pf_t += nunits;
+          pf_kb = 0;
+          if (pf_t < total) pf_tl = decode_tile<CG>(p, sc, pf_t, rank);
+        }
+      };
+      for (int i = 0; i < PF_DIST; ++i) advance_prefetch();
+      for (int32_t t = unit0; t < total && !failed; t += nunits) {
+        const Tile tl = decode_tile<CG>(p, sc, t, rank);
         for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
+          advance_prefetch();
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
           if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, lim)) {
             record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
@@ -287,35 +344,54 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             break;
           }
           const uint32_t fb = full_bar(s);
-          mbar_arrive_expect_tx(fb, STAGE_TX);
-          tma_load_2d(smem_addr(smem + OFF_A + s * A_TILE), &tmA, tl.a_x + BK * kb, tl.a_y, fb);
-          tma_load_2d(smem_addr(smem + OFF_B + s * B_TILE), &tmB, tl.b_x + BK * kb, tl.b_y, fb);
-          bulk_load(smem_addr(smem + OFF_SFA + s * SFA_TILE),
-                    atom_ptr(p.sfa, tl.sfa_row, tl.sfa_col + kb, p.sfa_pitch, p.sfa_atoms), 512, fb);
-          bulk_load(smem_addr(smem + OFF_SFB + s * SFB_TILE),
-                    atom_ptr(p.sfb, tl.sfb_row, tl.sfb_col + kb, p.sfb_pitch, p.sfb_atoms), 512, fb);
-          bulk_load(smem_addr(smem + OFF_SFB + s * SFB_TILE + 512),
-                    atom_ptr(p.sfb, tl.sfb_row + 1, tl.sfb_col + kb, p.sfb_pitch, p.sfb_atoms), 512, fb);
+          const uint32_t sa = smem_addr(smem + C::OFF_A + s * C::A_TILE);
+          const uint32_t sb = smem_addr(smem + C::OFF_B + s * C::B_TILE);
+          const uint32_t ssa = smem_addr(smem + C::OFF_SFA + s * SFA_TILE);
+          const uint32_t ssb = smem_addr(smem + C::OFF_SFB + s * SFB_TILE);
+          // Scale atoms are 4 rows of 128 bytes in the scale maps; atoms past
+          // the buffer read as zero (they only ever feed masked outputs).
+          const int32_t ya = static_cast<int32_t>(4 * (tl.sfa_atom + kb));
+          const int32_t yb0 = static_cast<int32_t>(4 * (tl.sfb_atom0 + kb));
+          const int32_t yb1 = static_cast<int32_t>(4 * (tl.sfb_atom1 + kb));
+          if constexpr (CG == 2) {
+            if (leader) mbar_arrive_expect_tx(fb, C::STAGE_TX);   // both CTAs' bytes land here
+            tma_load_2d_pair(sa, &tmA, tl.a_x + BK * kb, tl.a_y, fb);
+            tma_load_2d_pair(sb, &tmB, tl.b_x + BK * kb, tl.b_y, fb);
+            tma_load_2d_pair(ssa, &tmSFA, 0, ya, fb);
+            tma_load_2d_pair(ssb, &tmSFB, 0, yb0, fb);
+            tma_load_2d_pair(ssb + 512, &tmSFB, 0, yb1, fb);
+          } else {
+            mbar_arrive_expect_tx(fb, C::STAGE_TX);
+            tma_load_2d(sa, &tmA, tl.a_x + BK * kb, tl.a_y, fb);
+            tma_load_2d(sb, &tmB, tl.b_x + BK * kb, tl.b_y, fb);
+            tma_load_2d(ssa, &tmSFA, 0, ya, fb);
+            tma_load_2d(ssb, &tmSFB, 0, yb0, fb);
+            tma_load_2d(ssb + 512, &tmSFB, 0, yb1, fb);
+          }
           ++it;
         }
       }
       if (failed) {
         // Let every copy already issued land before the CTA can exit.
-        for (uint32_t j = it > STAGES ? it - STAGES : 0; j < it; ++j)
-          mbar_wait(full_bar(j % STAGES), (j / STAGES) & 1, &never, lim);
+        if (leader) {
+          for (uint32_t j = it > STAGES ? it - STAGES : 0; j < it; ++j)
+            mbar_wait(full_bar(j % STAGES), (j / STAGES) & 1, &never, lim);
+        } else {
+          for (int i = 0; i < 100; ++i) __nanosleep(1000);
+        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (leader CTA)
       // Instruction descriptor: E4M3 x E4M3, E8M0 scales, K-major A and B,
-      // M = 128, N = 256; the scale-factor ids (bits 4-5 for B, 29-30 for A)
-      // select the byte of the 32-bit scale column used by each K step.
-      const uint32_t idesc0 = (1u << 23) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+      // M = 128*CG, N = 256; the scale-factor ids (bits 4-5 for B, 29-30 for
+      // A) select the byte of the 32-bit scale column used by each K step.
+      const uint32_t idesc0 = (1u << 23) | (uint32_t(BN >> 3) << 17) | (uint32_t((BM * CG) >> 4) << 24);
       uint32_t it = 0, j = 0;
       bool failed = false;
-      for (int32_t t = blockIdx.x; t < total && !failed; t += gridDim.x) {
-        const Tile tl = decode_tile(p, sc, t);
+      for (int32_t t = unit0; t < total && !failed; t += nunits) {
+        const Tile tl = decode_tile<CG>(p, sc, t, 0);
         if (tl.kblocks == 0) continue;
         const uint32_t d_tmem = tmem + (j & 1) * ACC_STRIDE;
         if (!mbar_wait(acc_empty, (j & 1) ^ 1, abort_flag, lim)) {
@@ -333,47 +409,65 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           }
           tc_fence_after();
           const uint32_t sfa_t = tmem + SF_COL + SF_STRIDE * s, sfb_t = sfa_t + 4;
-          tc_cp_32x128b_x4(sfa_t, desc_sf_32x16(smem_addr(smem + OFF_SFA + s * SFA_TILE)));
-          tc_cp_32x128b_x4(sfb_t, desc_sf_32x16(smem_addr(smem + OFF_SFB + s * SFB_TILE)));
-          tc_cp_32x128b_x4(sfb_t + 4, desc_sf_32x16(smem_addr(smem + OFF_SFB + s * SFB_TILE + 512)));
-          const uint64_t da = desc_kmajor_sw128(smem_addr(smem + OFF_A + s * A_TILE));
-          const uint64_t db = desc_kmajor_sw128(smem_addr(smem + OFF_B + s * B_TILE));
+          const uint64_t dsa = desc_sf_32x16(smem_addr(smem + C::OFF_SFA + s * SFA_TILE));
+          const uint64_t dsb0 = desc_sf_32x16(smem_addr(smem + C::OFF_SFB + s * SFB_TILE));
+          const uint64_t dsb1 = desc_sf_32x16(smem_addr(smem + C::OFF_SFB + s * SFB_TILE + 512));
+          const uint64_t da = desc_kmajor_sw128(smem_addr(smem + C::OFF_A + s * C::A_TILE));
+          const uint64_t db = desc_kmajor_sw128(smem_addr(smem + C::OFF_B + s * C::B_TILE));
           const int32_t nk = (kb == tl.kblocks - 1) ? tl.ksteps_last : BK / 32;
+          if constexpr (CG == 2) {
+            tc_cp_32x128b_x4_pair(sfa_t, dsa);
+            tc_cp_32x128b_x4_pair(sfb_t, dsb0);
+            tc_cp_32x128b_x4_pair(sfb_t + 4, dsb1);
+          } else {
+            tc_cp_32x128b_x4(sfa_t, dsa);
+            tc_cp_32x128b_x4(sfb_t, dsb0);
+            tc_cp_32x128b_x4(sfb_t + 4, dsb1);
+          }
           for (int32_t k = 0; k < nk; ++k) {
             const uint32_t idesc = idesc0 | (uint32_t(k) << 4) | (uint32_t(k) << 29);
             // +2 per step: the start-address field counts 16-byte units, one step is 32 bytes of K
-            tc_mma_mxf8(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
-                        sfb_t | (uint32_t(k) << 30), (kb | k) != 0);
+            if constexpr (CG == 2)
+              tc_mma_mxf8_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
+                               sfb_t | (uint32_t(k) << 30), (kb | k) != 0);
+            else
+              tc_mma_mxf8(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
+                          sfb_t | (uint32_t(k) << 30), (kb | k) != 0);
           }
-          tc_commit(empty_bar(s));
+          if constexpr (CG == 2) tc_commit_pair(empty_bar(s), 0x3);
+          else tc_commit(empty_bar(s));
           ++it;
         }
         if (failed) break;
-        tc_commit(acc_full);
+        if constexpr (CG == 2) tc_commit_pair(acc_full, 0x3);
+        else tc_commit(acc_full);
         ++j;
       }
       if (failed) {
         // Wait for the MMAs and copies already issued before freeing tensor memory.
-        tc_commit(drain_bar);
+        if constexpr (CG == 2) tc_commit_pair(drain_bar, 0x1);
+        else tc_commit(drain_bar);
         mbar_wait(drain_bar, 0, &never, lim);
       }
     }
   } else {
-    // -------------------------------------------------------------- epilogue
+    // -------------------------------------------------------------- epilogue (every CTA)
     const uint32_t quarter = warp & 3;   // tensor-memory lanes 32*quarter .. +31
-    uint4* stage = reinterpret_cast<uint4*>(smem + OFF_EPI + (warp - 2) * EPI_STAGE);
+    uint8_t* stage_base = smem + C::OFF_EPI + (warp - 2) * C::EPI_BUFS * EPI_STAGE;
     const int srow = lane >> 3, schunk = lane & 7;
-    uint32_t j = 0;
-    for (int32_t t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile tl = decode_tile(p, sc, t);
-      const int32_t row_base = 32 * quarter;
+    const int32_t row_base = 32 * static_cast<int32_t>(quarter);
+    uint32_t j = 0, ec = 0;
+    for (int32_t t = unit0; t < total; t += nunits) {
+      const Tile tl = decode_tile<CG>(p, sc, t, rank);
+      const int32_t vr = max(0, min(32, tl.rows - row_base));       // valid rows of this warp's slice
+      uint16_t* out_tile = p.out + tl.out_row * p.out_ld + tl.out_col;
       if (tl.kblocks == 0) {
         // An expert without tokens: dW_e = 0.
         for (int c = 0; c < 4; ++c)
           for (int i = 0; i < 8; ++i) {
-            const int r = row_base + 4 * i + srow, col = 64 * c + 8 * schunk;
-            if (r < tl.rows && col < tl.cols)
-              *reinterpret_cast<uint4*>(tl.out + int64_t(r) * tl.ld + col) = make_uint4(0, 0, 0, 0);
+            const int rr = 4 * i + srow, col = 64 * c + 8 * schunk;
+            if (rr < vr && col < tl.cols)
+              *reinterpret_cast<uint4*>(out_tile + int64_t(row_base + rr) * p.out_ld + col) = make_uint4(0, 0, 0, 0);
           }
         continue;
       }
@@ -383,46 +477,85 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       }
       tc_fence_after();
       const uint32_t buf = j & 1;
+      const uint32_t tbase = tmem + ((32 * quarter) << 16) + buf * ACC_STRIDE;
+      // Buffer 0 shares its last 64 columns with buffer 1's first 64: drain them first.
+      auto chunk_of = [&](int ci) { return buf == 0 ? (ci + 3) & 3 : ci; };
+      uint32_t ra0[32], ra1[32], rb0[32], rb1[32];
+      tmem_ld_32x32b_x32(tbase + 64 * chunk_of(0), ra0);
+      tmem_ld_32x32b_x32(tbase + 64 * chunk_of(0) + 32, ra1);
+      tmem_wait_regs(ra0);
+      tmem_wait_regs(ra1);
+      tc_fence_before();
+      if constexpr (CG == 2) {
+        if (leader) mbar_arrive(acc_empty); else mbar_arrive_cluster(acc_empty, 0);
+      } else {
+        mbar_arrive(acc_empty);
+      }
+#pragma unroll
       for (int ci = 0; ci < 4; ++ci) {
-        // Buffer 0 shares its last 64 columns with buffer 1's first 64: drain them first.
-        const int c = buf == 0 ? (ci + 3) & 3 : ci;
-        const uint32_t taddr = tmem + ((32 * quarter) << 16) + buf * ACC_STRIDE + 64 * c;
-        uint32_t r0[32], r1[32];
-        tmem_ld_32x32b_x32(taddr, r0);
-        tmem_ld_32x32b_x32(taddr + 32, r1);
-        tmem_ld_wait();
-        if (ci == 0) {
-          tc_fence_before();
-          mbar_arrive(acc_empty);
+        uint32_t(&c0)[32] = (ci & 1) ? rb0 : ra0;
+        uint32_t(&c1)[32] = (ci & 1) ? rb1 : ra1;
+        uint32_t(&n0)[32] = (ci & 1) ? ra0 : rb0;
+        uint32_t(&n1)[32] = (ci & 1) ? ra1 : rb1;
+        if (ci < 3) {   // next chunk's tensor-memory load overlaps this chunk's conversion and store
+          tmem_ld_32x32b_x32(tbase + 64 * chunk_of(ci + 1), n0);
+          tmem_ld_32x32b_x32(tbase + 64 * chunk_of(ci + 1) + 32, n1);
         }
-        uint32_t pk[32];
+        const int c = chunk_of(ci);
+        if (vr > 0 && 64 * c < tl.cols) {
+          uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          pk[i] = cvt_bf16x2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
-          pk[16 + i] = cvt_bf16x2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
+          for (int i = 0; i < 16; ++i) {
+            pk[i] = cvt_bf16x2(__uint_as_float(c0[2 * i]), __uint_as_float(c0[2 * i + 1]));
+            pk[16 + i] = cvt_bf16x2(__uint_as_float(c1[2 * i]), __uint_as_float(c1[2 * i + 1]));
+          }
+          uint8_t* stg = stage_base + (ec % C::EPI_BUFS) * EPI_STAGE;
+          uint4* st4 = reinterpret_cast<uint4*>(stg);
+          if (lane == 0) bulk_wait_read<C::EPI_BUFS - 1>();   // the buffer's previous store has read it
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 8; ++q)   // 128-byte swizzle: chunk q of row `lane` at q ^ (lane % 8)
+            st4[lane * 8 + (q ^ (lane & 7))] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          if (vr == 32) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmOut, static_cast<int32_t>(tl.out_col + 64 * c),
+                           static_cast<int32_t>(tl.out_row + row_base), smem_addr(stg));
+              bulk_commit_group();
+            }
+          } else {
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int rr = 4 * i + srow, col = 64 * c + 8 * schunk;
+              if (rr < vr && col < tl.cols)
+                *reinterpret_cast<uint4*>(out_tile + int64_t(row_base + rr) * p.out_ld + col) =
+                    st4[rr * 8 + (schunk ^ (rr & 7))];
+            }
+          }
+          __syncwarp();
+          ++ec;
         }
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          stage[lane * 8 + (q ^ (lane & 7))] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = 4 * i + srow;
-          const int r = row_base + rr, col = 64 * c + 8 * schunk;
-          if (r < tl.rows && col < tl.cols)
-            *reinterpret_cast<uint4*>(tl.out + int64_t(r) * tl.ld + col) = stage[rr * 8 + (schunk ^ (rr & 7))];
+        if (ci < 3) {
+          tmem_wait_regs(n0);
+          tmem_wait_regs(n1);
         }
-        __syncwarp();
       }
       ++j;
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) cluster_sync();   // both CTAs are done with tensor memory
+  else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    if constexpr (CG == 2) tmem_dealloc_pair(tmem, TMEM_COLS);
+    else tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -444,37 +577,100 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2D map over uint8 codes [rows, cols] with row stride ld bytes; box = box_cols x box_rows,
-// 128-byte swizzle (box_cols = 128), zero fill outside the matrix.
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, uint32_t box_rows) {
+// 2D map over a row-major matrix [rows, cols] of `esize`-byte elements with
+// row stride `ld` elements; box = box_cols x box_rows; zero fill outside.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, int esize, int64_t rows, int64_t cols,
+              int64_t ld, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
+  if (!fn || rows < 1 || cols < 1) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * esize)};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceSetup {
+  bool done[2] = {false, false};
+  int num_sms = 0;
+  int max_pairs = 0;
+};
+DeviceSetup g_setup[64];
+
+template <int CG>
+cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_t stream) {
+  using C = Cfg<CG>;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  DeviceSetup& ds = g_setup[dev];
+  auto kernel = grouped_gemm_kernel<CG>;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  if (!ds.done[CG - 1]) {
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    err = cudaDeviceGetAttribute(&ds.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    if (CG == 2) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(2 * (ds.num_sms / 2));
+      q.blockDim = dim3(NUM_THREADS);
+      q.dynamicSmemBytes = C::SMEM_BYTES;
+      q.attrs = attr;
+      q.numAttrs = 1;
+      int clusters = 0;
+      err = cudaOccupancyMaxActiveClusters(&clusters, kernel, &q);
+      if (err != cudaSuccess) return err;
+      ds.max_pairs = clusters > 0 ? clusters : 1;
+    }
+    ds.done[CG - 1] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  if (CG == 2) {
+    cfg.gridDim = dim3(2 * ds.max_pairs);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  } else {
+    cfg.gridDim = dim3(ds.num_sms);
+  }
+  return cudaLaunchKernelEx(&cfg, kernel, maps[0], maps[1], maps[2], maps[3], maps[4], p);
 }
 
 }  // namespace
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** detail) {
-  static int configured_device = -1;
-  static int num_sms = 0;
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
-  if (configured_device != dev) {
-    err = cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (err != cudaSuccess) return err;
-    err = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (err != cudaSuccess) return err;
-    configured_device = dev;
-  }
-  CUtensorMap tmA, tmB;
-  if (!make_map(&tmA, a.a, a.a_rows, a.a_cols, a.lda, BM) || !make_map(&tmB, a.b, a.b_rows, a.b_cols, a.ldb, BN)) {
+  // Tile configuration per pass, from B200 measurements: the forward and
+  // dgrad passes (long K, ragged M) run 1-CTA tiles, whose M granularity of
+  // 128 wastes fewer rows at group tails; wgrad (fixed output rows, ragged
+  // K) runs CTA pairs.  MXF8_GEMM_CTA_PAIR=0/1 forces one configuration.
+  const char* env = std::getenv("MXF8_GEMM_CTA_PAIR");
+  int cg = a.mode == kWgrad ? 2 : 1;
+  if (env && std::strcmp(env, "0") == 0) cg = 1;
+  if (env && std::strcmp(env, "1") == 0) cg = 2;
+  const int64_t out_rows = a.mode == kWgrad ? int64_t(a.E) * a.N : a.M;
+  const int64_t out_cols = a.mode == kFwd ? a.N : a.K;
+  CUtensorMap maps[5];
+  const bool ok =
+      make_map(&maps[0], a.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.a_rows, a.a_cols, a.lda, BK, BM,
+               CU_TENSOR_MAP_SWIZZLE_128B) &&
+      make_map(&maps[1], a.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b_rows, a.b_cols, a.ldb, BK, BN / cg,
+               CU_TENSOR_MAP_SWIZZLE_128B) &&
+      make_map(&maps[2], a.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfa_atoms * 4, 128, 128, 128, 4,
+               CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      make_map(&maps[3], a.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfb_atoms * 4, 128, 128, 128, 4,
+               CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      make_map(&maps[4], a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out_rows, out_cols, out_cols, 64, 32,
+               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) {
     if (detail) *detail = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
@@ -483,14 +679,13 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   p.E = a.E;
   p.M = a.M; p.N = a.N; p.K = a.K;
   p.offs = a.offs;
-  p.sfa = a.sfa; p.sfb = a.sfb;
   p.sfa_pitch = a.sfa_pitch; p.sfb_pitch = a.sfb_pitch;
-  p.sfa_atoms = a.sfa_atoms; p.sfb_atoms = a.sfb_atoms;
   p.out = a.out;
+  p.out_ld = out_cols;
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
-  grouped_gemm_kernel<<<num_sms, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
-  return cudaGetLastError();
+  return cg == 2 ? launch_cg<2>(p, maps, stream) : launch_cg<1>(p, maps, stream);
 }
 
 }  // namespace mxf8
+
