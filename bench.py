@@ -4,8 +4,10 @@
 One step = one pass of the whole path over one synthetic routed batch of the
 DeepSeek-V3-16B-like MoE layer (64 experts, top-6 of 8192 tokens = 49152
 rows; gate/up N = 2816, K = 2048; down N = 2048, K = 1408): for each of the
-two grouped linears, rowwise + colwise MXFP8 quantisation of X, W and dY,
-then the forward, dgrad and wgrad grouped GEMMs.  The metric is algorithmic
+two grouped linears, rowwise + colwise MXFP8 quantisation of X, W and dY
+(by default one fused dual-layout kernel per tensor; --quantiser separate
+runs the rowwise and colwise kernels), then the forward, dgrad and wgrad
+grouped GEMMs.  The metric is algorithmic
 GEMM TFLOP/s (3 passes x 2*M*N*K per linear over real tokens) per step.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
@@ -49,6 +51,8 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quantiser", default="dual", choices=["dual", "separate"],
+                    help="dual: one fused kernel writes both layouts of X, W and dY")
     return ap.parse_args()
 
 
@@ -118,8 +122,9 @@ class ClockSampler:
 class Linear:
     """Device buffers and launches for one grouped linear (all three passes)."""
 
-    def __init__(self, mx, w: wl.Workload, layer: wl.Layer, device):
+    def __init__(self, mx, w: wl.Workload, layer: wl.Layer, device, quantiser="dual"):
         self.mx = mx
+        self.quantiser = quantiser
         self.name = layer.name
         self.M, self.N, self.K, self.E = w.M, layer.N, layer.K, w.E
         self.X, W, self.dY = wl.layer_tensors(w, layer, device=device)
@@ -144,26 +149,46 @@ class Linear:
         return 2 * self.M * self.N * self.K
 
     def quant_bytes(self):
-        """Algorithmic bytes of the six quantisations: 2 B read, 1 + 1/32 B written per element."""
-        el = 2 * (self.M * self.K + self.E * self.N * self.K + self.M * self.N)
-        return el * (2 + 1 + 1 / 32)
+        """Algorithmic bytes of quantising X, W and dY into both layouts: per
+        element 2 B read per pass over the input and 1 + 1/32 B written per
+        layout (dual: one read, separate: two reads)."""
+        el = self.M * self.K + self.E * self.N * self.K + self.M * self.N
+        reads = 1 if self.quantiser == "dual" else 2
+        return el * (2 * reads + 2 * (1 + 1 / 32))
 
     def launches(self):
         """(kind, callable) for one pass of the path; kind is 'quant' or 'gemm:<pass>'."""
         mx = self.mx
+        gemms = {
+            "fwd": lambda: mx.mxfp8_grouped_gemm_fwd(self.xq, self.xs, self.wq, self.ws, self.offs, self.N,
+                                                     out=self.y, work=self.work),
+            "dgrad": lambda: mx.mxfp8_grouped_gemm_dgrad(self.dyq, self.dys, self.wqT, self.wsT, self.offs, self.K,
+                                                         out=self.dx, work=self.work),
+            "wgrad": lambda: mx.mxfp8_grouped_gemm_wgrad(self.dyqT, self.dysT, self.xqT, self.xsT, self.offs, self.M,
+                                                         out=self.dw, work=self.work),
+        }
+        if self.quantiser == "dual":
+            return [
+                ("quant", lambda: mx.mxfp8_quantize_dual(self.X, self.offs, q=self.xq, scales=self.xs, qT=self.xqT,
+                                                         scalesT=self.xsT)),
+                ("quant", lambda: mx.mxfp8_quantize_dual(self.W2, None, q=self.wq, scales=self.ws, qT=self.wqT,
+                                                         scalesT=self.wsT)),
+                ("gemm:fwd", gemms["fwd"]),
+                ("quant", lambda: mx.mxfp8_quantize_dual(self.dY, self.offs, q=self.dyq, scales=self.dys,
+                                                         qT=self.dyqT, scalesT=self.dysT)),
+                ("gemm:dgrad", gemms["dgrad"]),
+                ("gemm:wgrad", gemms["wgrad"]),
+            ]
         return [
             ("quant", lambda: mx.mxfp8_quantize_rowwise(self.X, self.offs, q=self.xq, scales=self.xs)),
             ("quant", lambda: mx.mxfp8_quantize_rowwise(self.W2, None, q=self.wq, scales=self.ws)),
-            ("gemm:fwd", lambda: mx.mxfp8_grouped_gemm_fwd(self.xq, self.xs, self.wq, self.ws, self.offs, self.N,
-                                                           out=self.y, work=self.work)),
+            ("gemm:fwd", gemms["fwd"]),
             ("quant", lambda: mx.mxfp8_quantize_rowwise(self.dY, self.offs, q=self.dyq, scales=self.dys)),
             ("quant", lambda: mx.mxfp8_quantize_colwise(self.W2, None, qT=self.wqT, scales=self.wsT)),
-            ("gemm:dgrad", lambda: mx.mxfp8_grouped_gemm_dgrad(self.dyq, self.dys, self.wqT, self.wsT, self.offs,
-                                                               self.K, out=self.dx, work=self.work)),
+            ("gemm:dgrad", gemms["dgrad"]),
             ("quant", lambda: mx.mxfp8_quantize_colwise(self.dY, self.offs, qT=self.dyqT, scales=self.dysT)),
             ("quant", lambda: mx.mxfp8_quantize_colwise(self.X, self.offs, qT=self.xqT, scales=self.xsT)),
-            ("gemm:wgrad", lambda: mx.mxfp8_grouped_gemm_wgrad(self.dyqT, self.dysT, self.xqT, self.xsT, self.offs,
-                                                               self.M, out=self.dw, work=self.work)),
+            ("gemm:wgrad", gemms["wgrad"]),
         ]
 
 
@@ -174,7 +199,7 @@ def run_ours(args, rank, world, local_rank):
     if not mx.mxfp8_device_supported():
         raise SystemExit("bench: the current device is not sm_100")
     w = wl.WORKLOADS[args.workload]()
-    layers = [Linear(mx, w, L, dev) for L in w.layers]
+    layers = [Linear(mx, w, L, dev, args.quantiser) for L in w.layers]
     calls = [c for L in layers for c in L.launches()]
     step_flops = 3 * sum(L.flops_per_pass() for L in layers)
     quant_bytes = sum(L.quant_bytes() for L in layers)
@@ -244,7 +269,8 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": f"{w.name}-like MoE layer", "experts": w.E, "routed_rows": w.M,
                    "layers": [{"name": L.name, "N": L.N, "K": L.K} for L in w.layers],
                    "routing": "top-6 of 8192 tokens, N(0,1) logits + N(0,0.5) expert bias" if w.name == "ds-v3-16b" else w.name,
-                   "l2": "inputs larger than L2 (step touches > 2 GB)", "parallelism": f"replica x{world}"},
+                   "l2": "inputs larger than L2 (step touches > 2 GB)", "parallelism": f"replica x{world}",
+                   "quantiser": args.quantiser},
         "fraction_of_fp8_peak": round(value / world / fp8_peak, 4),
         "roofline": {"kernel": "grouped_gemm_kernel (fwd+dgrad+wgrad launches)", "bound": "tensor",
                      "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",

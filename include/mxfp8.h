@@ -138,6 +138,18 @@ MXF8_API mxf8_status mxfp8_quantize_colwise(const uint16_t* x, int64_t rows, int
                                    uint8_t* qT, int64_t ldT, uint8_t* scalesT,
                                    int64_t scale_bytes, void* stream);
 
+/* Rowwise and colwise quantisation of the same input in one pass (one read
+ * of x, both outputs).  Outputs, layouts and errors are exactly those of
+ * mxfp8_quantize_rowwise(x, ..., q, scales) followed by
+ * mxfp8_quantize_colwise(x, ..., qT, ldT, scalesT): in training X and dY need
+ * both layouts (forward/dgrad read rowwise, wgrad colwise) and W needs
+ * rowwise (forward) and colwise (dgrad). */
+MXF8_API mxf8_status mxfp8_quantize_dual(const uint16_t* x, int64_t rows, int64_t cols,
+                                         const int32_t* d_offs, int32_t num_groups,
+                                         uint8_t* q, uint8_t* scales, int64_t scale_bytes,
+                                         uint8_t* qT, int64_t ldT, uint8_t* scalesT,
+                                         int64_t scaleT_bytes, void* stream);
+
 /* ---------------------------------------------------------------- grouped GEMMs
  * Shared arguments: E = num_groups (1..MXF8_GEMM_MAX_GROUPS); M = total rows
  * (d_offs[E]); N % 128 == 0; K % 32 == 0; N, K > 0.  `work` is a device

@@ -35,7 +35,7 @@ EXPORTED = ("mxfp8_rowwise_scale_bytes", "mxfp8_colwise_pitch", "mxfp8_colwise_s
             "mxfp8_workspace_bytes", "mxfp8_quantize_rowwise", "mxfp8_quantize_colwise",
             "mxfp8_grouped_gemm_fwd", "mxfp8_grouped_gemm_dgrad", "mxfp8_grouped_gemm_wgrad",
             "mxfp8_get_status", "mxfp8_status_string", "mxfp8_last_cuda_error", "mxfp8_device_supported",
-            "mxfp8_grouped_gemm_fwd_noalloc")
+            "mxfp8_grouped_gemm_fwd_noalloc", "mxfp8_quantize_dual")
 
 
 class MXFP8Error(RuntimeError):
@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.mxfp8_quantize_rowwise.argtypes = [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _i64, _vp]
         L.mxfp8_quantize_colwise.restype = _i32
         L.mxfp8_quantize_colwise.argtypes = [_vp, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _i64, _vp]
+        L.mxfp8_quantize_dual.restype = _i32
+        L.mxfp8_quantize_dual.argtypes = [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _i64, _vp, _i64, _vp, _i64, _vp]
         for n in ("mxfp8_grouped_gemm_fwd", "mxfp8_grouped_gemm_dgrad", "mxfp8_grouped_gemm_wgrad"):
             getattr(L, n).restype = _i32
             getattr(L, n).argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp, _vp, _i64, _vp]
@@ -157,6 +159,22 @@ def mxfp8_quantize_colwise(x: torch.Tensor, offs: torch.Tensor | None = None, qT
     _check(lib().mxfp8_quantize_colwise(_ptr(x), R, C, _ptr(offs), G, _ptr(qT), ld, _ptr(scales), scales.numel(),
                                         _stream(stream)), "mxfp8_quantize_colwise")
     return qT, scales
+
+
+def mxfp8_quantize_dual(x: torch.Tensor, offs: torch.Tensor | None = None, q=None, scales=None, qT=None,
+                        scalesT=None, stream=None):
+    """x: bf16 [rows, cols] -> (q, scales, qT, scalesT): both layouts from one read."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    R, C = x.shape
+    G = _groups(offs)
+    ld = mxfp8_colwise_ld(R, G)
+    q = q if q is not None else torch.empty((R, C), dtype=torch.uint8, device=x.device)
+    scales = scales if scales is not None else _u8(mxfp8_rowwise_scale_bytes(R, C, G), x.device)
+    qT = qT if qT is not None else torch.empty((C, ld), dtype=torch.uint8, device=x.device)
+    scalesT = scalesT if scalesT is not None else _u8(mxfp8_colwise_scale_bytes(R, C, G), x.device)
+    _check(lib().mxfp8_quantize_dual(_ptr(x), R, C, _ptr(offs), G, _ptr(q), _ptr(scales), scales.numel(), _ptr(qT),
+                                     ld, _ptr(scalesT), scalesT.numel(), _stream(stream)), "mxfp8_quantize_dual")
+    return q, scales, qT, scalesT
 
 
 # ------------------------------------------------------------------ grouped GEMMs

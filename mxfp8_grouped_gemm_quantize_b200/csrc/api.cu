@@ -145,6 +145,23 @@ mxf8_status mxfp8_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols
   return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "quantize_colwise launch");
 }
 
+mxf8_status mxfp8_quantize_dual(const uint16_t* x, int64_t rows, int64_t cols, const int32_t* d_offs,
+                                int32_t num_groups, uint8_t* q, uint8_t* scales, int64_t scale_bytes, uint8_t* qT,
+                                int64_t ldT, uint8_t* scalesT, int64_t scaleT_bytes, void* stream) {
+  mxf8_status s = check_quant_args(x, rows, cols, num_groups, q, scales, scale_bytes,
+                                   mxfp8_rowwise_scale_bytes(rows, cols, num_groups));
+  if (s != MXF8_OK) return s;
+  s = check_quant_args(x, rows, cols, num_groups, qT, scalesT, scaleT_bytes,
+                       mxfp8_colwise_scale_bytes(rows, cols, num_groups));
+  if (s != MXF8_OK) return s;
+  if (!d_offs && num_groups != 1) return MXF8_ERR_INVALID_ARG;
+  if (ldT != mxfp8_colwise_ld(rows, num_groups)) return MXF8_ERR_INVALID_ARG;
+  if ((s = check_device()) != MXF8_OK) return s;
+  cudaError_t e = mxf8::launch_quantize_dual(x, rows, cols, d_offs, num_groups, q, scales, qT, ldT, scalesT,
+                                             static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "quantize_dual launch");
+}
+
 mxf8_status mxfp8_grouped_gemm_fwd(const uint8_t* xq, const uint8_t* xs, int64_t xs_bytes, const uint8_t* wq,
                                    const uint8_t* ws, int64_t ws_bytes, const int32_t* d_offs, int32_t E,
                                    int64_t M, int64_t N, int64_t K, uint16_t* y, void* work,

@@ -24,10 +24,11 @@
 // atoms to tensor memory and issues the MMAs; warps 2-5 drain the
 // accumulator: tcgen05.ld -> bf16 -> 128-byte-swizzled shared stage -> TMA
 // bulk-tensor store (plain masked stores only for a group's ragged slice).
-// Two 128x256 fp32 accumulators overlap in 64 columns (0..255 and 192..447);
+// Two 128x256 fp32 accumulators overlap in 64 or 128 columns (0..255 and
+// 192..447, or 128..383 when more pipeline stages need more scale columns);
 // the epilogue drains the shared columns first and releases the accumulator,
-// so the next tile's MMAs overlap the rest of the drain.  Columns 448.. hold
-// one scale-factor set per pipeline stage.
+// so the next tile's MMAs overlap the rest of the drain.  The columns after
+// accumulator 1 hold one scale-factor set per pipeline stage.
 // The tile schedule is built on the device from the group offsets at kernel
 // start (no host synchronisation); tiles are dealt round-robin.  Every wait is
 // bounded: on timeout the kernel records MXF8_ERR_TIMEOUT, drains its
@@ -50,22 +51,30 @@ constexpr int SFA_TILE = 512, SFB_TILE = 1024;
 constexpr int NUM_THREADS = 192;
 constexpr int EPI_STAGE = 32 * 128;        // one epilogue buffer: 32 rows x 64 bf16, 128B-swizzled
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_STRIDE = 192;       // accumulator 1 starts at column 192
-constexpr uint32_t SF_COL = 448;           // stage s: SFA at 448 + 12 s (4 columns), SFB at +4 (8 columns)
-constexpr uint32_t SF_STRIDE = 12;
+constexpr uint32_t SF_STRIDE = 12;        // per stage: SFA 4 columns, then SFB 8 columns
 constexpr int MAXG = MXF8_GEMM_MAX_GROUPS;
-constexpr int PF_DIST = 8;                 // K blocks of L2 prefetch ahead of the TMA loads
+#ifndef MXF8_PAIR_STAGES
+#define MXF8_PAIR_STAGES 5
+#endif
+#ifndef MXF8_PAIR_EPI_BUFS
+#define MXF8_PAIR_EPI_BUFS 2
+#endif
 constexpr int SCHED_INTS = 4 * (MAXG + 1);
 
 constexpr int round_up_c(int a, int b) { return (a + b - 1) / b * b; }
 
 template <int CG>
 struct Cfg {
-  static constexpr int STAGES = CG == 2 ? 5 : 4;
+  static constexpr int STAGES = CG == 2 ? MXF8_PAIR_STAGES : 4;
   static constexpr int B_ROWS = BN / CG;               // B rows staged by each CTA
   static constexpr int A_TILE = BM * BK;               // 16 KB of E4M3 codes
   static constexpr int B_TILE = B_ROWS * BK;
-  static constexpr int EPI_BUFS = CG == 2 ? 2 : 1;
+  static constexpr int EPI_BUFS = CG == 2 ? MXF8_PAIR_EPI_BUFS : 1;
+  // The two 128x256 accumulators overlap in OV 64-column chunks: accumulator 1
+  // starts at column ACC_STRIDE, and the scale sets of all stages follow it.
+  static constexpr int OV = (STAGES * SF_STRIDE <= 64) ? 1 : 2;
+  static constexpr uint32_t ACC_STRIDE = 256 - 64 * OV;
+  static constexpr uint32_t SF_COL = ACC_STRIDE + 256;
   static constexpr uint32_t STAGE_TX = CG * (A_TILE + B_TILE + SFA_TILE + SFB_TILE);
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_TILE;
@@ -78,10 +87,9 @@ struct Cfg {
   static constexpr int SMEM_BYTES = OFF_SCHED + SCHED_INTS * 4 + 1024;   // + slack to align the base
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(OFF_B % 1024 == 0 && B_TILE % 1024 == 0 && OFF_EPI % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-  static_assert(SF_COL + SF_STRIDE * (STAGES - 1) + 12 <= TMEM_COLS, "scale columns");
+  static_assert(SF_COL + SF_STRIDE * STAGES <= TMEM_COLS, "scale columns");
   static_assert((2 * STAGES + 3) * 8 <= 128, "barrier area");
 };
-static_assert(ACC_STRIDE + BN <= SF_COL, "accumulators must not reach the scale columns");
 
 struct Params {
   int mode;
@@ -313,30 +321,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       // ------------------------------------------------------------ producer (every CTA)
       uint32_t it = 0;
       bool failed = false;
-      // L2 prefetch cursor running PF_DIST K blocks ahead of the loads, across
-      // tile boundaries, so first touches of A/B tiles (DRAM misses) overlap
-      // the ring's in-flight loads.
-      int32_t pf_t = unit0, pf_kb = 0;
-      Tile pf_tl;
-      if (pf_t < total) pf_tl = decode_tile<CG>(p, sc, pf_t, rank);
-      auto advance_prefetch = [&]() {
-        while (pf_t < total) {
-          if (pf_kb < pf_tl.kblocks) {
-            tma_prefetch_2d(&tmA, pf_tl.a_x + BK * pf_kb, pf_tl.a_y);
-            tma_prefetch_2d(&tmB, pf_tl.b_x + BK * pf_kb, pf_tl.b_y);
-            ++pf_kb;
-            return;
-          }
-          pf_t += nunits;
-          pf_kb = 0;
-          if (pf_t < total) pf_tl = decode_tile<CG>(p, sc, pf_t, rank);
-        }
-      };
-      for (int i = 0; i < PF_DIST; ++i) advance_prefetch();
       for (int32_t t = unit0; t < total && !failed; t += nunits) {
         const Tile tl = decode_tile<CG>(p, sc, t, rank);
         for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
-          advance_prefetch();
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
           if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, lim)) {
             record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
@@ -393,7 +380,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       for (int32_t t = unit0; t < total && !failed; t += nunits) {
         const Tile tl = decode_tile<CG>(p, sc, t, 0);
         if (tl.kblocks == 0) continue;
-        const uint32_t d_tmem = tmem + (j & 1) * ACC_STRIDE;
+        const uint32_t d_tmem = tmem + (j & 1) * C::ACC_STRIDE;
         if (!mbar_wait(acc_empty, (j & 1) ^ 1, abort_flag, lim)) {
           record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
           failed = true;
@@ -408,7 +395,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             break;
           }
           tc_fence_after();
-          const uint32_t sfa_t = tmem + SF_COL + SF_STRIDE * s, sfb_t = sfa_t + 4;
+          const uint32_t sfa_t = tmem + C::SF_COL + SF_STRIDE * s, sfb_t = sfa_t + 4;
           const uint64_t dsa = desc_sf_32x16(smem_addr(smem + C::OFF_SFA + s * SFA_TILE));
           const uint64_t dsb0 = desc_sf_32x16(smem_addr(smem + C::OFF_SFB + s * SFB_TILE));
           const uint64_t dsb1 = desc_sf_32x16(smem_addr(smem + C::OFF_SFB + s * SFB_TILE + 512));
@@ -477,20 +464,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       }
       tc_fence_after();
       const uint32_t buf = j & 1;
-      const uint32_t tbase = tmem + ((32 * quarter) << 16) + buf * ACC_STRIDE;
-      // Buffer 0 shares its last 64 columns with buffer 1's first 64: drain them first.
-      auto chunk_of = [&](int ci) { return buf == 0 ? (ci + 3) & 3 : ci; };
+      const uint32_t tbase = tmem + ((32 * quarter) << 16) + buf * C::ACC_STRIDE;
+      // Accumulator 0's last OV chunks are accumulator 1's first OV chunks:
+      // drain those first, then release the accumulator to the MMA issuer.
+      auto chunk_of = [&](int ci) { return buf == 0 ? (ci + 4 - C::OV) & 3 : ci; };
+      auto release = [&]() {
+        tc_fence_before();
+        if constexpr (CG == 2) {
+          if (leader) mbar_arrive(acc_empty); else mbar_arrive_cluster(acc_empty, 0);
+        } else {
+          mbar_arrive(acc_empty);
+        }
+      };
       uint32_t ra0[32], ra1[32], rb0[32], rb1[32];
       tmem_ld_32x32b_x32(tbase + 64 * chunk_of(0), ra0);
       tmem_ld_32x32b_x32(tbase + 64 * chunk_of(0) + 32, ra1);
       tmem_wait_regs(ra0);
       tmem_wait_regs(ra1);
-      tc_fence_before();
-      if constexpr (CG == 2) {
-        if (leader) mbar_arrive(acc_empty); else mbar_arrive_cluster(acc_empty, 0);
-      } else {
-        mbar_arrive(acc_empty);
-      }
+      if (C::OV == 1) release();
 #pragma unroll
       for (int ci = 0; ci < 4; ++ci) {
         uint32_t(&c0)[32] = (ci & 1) ? rb0 : ra0;
@@ -540,6 +531,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (ci < 3) {
           tmem_wait_regs(n0);
           tmem_wait_regs(n1);
+          if (ci + 2 == C::OV) release();   // chunk ci + 1 (the last shared one) is now in registers
         }
       }
       ++j;
@@ -648,12 +640,12 @@ cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_
 }  // namespace
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** detail) {
-  // Tile configuration per pass, from B200 measurements: the forward and
-  // dgrad passes (long K, ragged M) run 1-CTA tiles, whose M granularity of
-  // 128 wastes fewer rows at group tails; wgrad (fixed output rows, ragged
-  // K) runs CTA pairs.  MXF8_GEMM_CTA_PAIR=0/1 forces one configuration.
+  // Tile configuration: 1-CTA 128x256 tiles by default -- on B200 they beat
+  // CTA pairs on every pass of the DeepSeek-V3-like layers (pairs also waste
+  // up to 128 rows per group in fwd/dgrad).  MXF8_GEMM_CTA_PAIR=1 selects
+  // pairs, MXF8_GEMM_CTA_PAIR=0 the default.
   const char* env = std::getenv("MXF8_GEMM_CTA_PAIR");
-  int cg = a.mode == kWgrad ? 2 : 1;
+  int cg = 1;
   if (env && std::strcmp(env, "0") == 0) cg = 1;
   if (env && std::strcmp(env, "1") == 0) cg = 2;
   const int64_t out_rows = a.mode == kWgrad ? int64_t(a.E) * a.N : a.M;

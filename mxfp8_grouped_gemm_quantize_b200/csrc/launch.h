@@ -13,6 +13,10 @@ cudaError_t launch_quantize_colwise(const uint16_t* x, int64_t rows, int64_t col
                                     const int32_t* offs, int32_t G, uint8_t* qT, int64_t ldT,
                                     uint8_t* sfT, cudaStream_t stream);
 
+cudaError_t launch_quantize_dual(const uint16_t* x, int64_t rows, int64_t cols, const int32_t* offs,
+                                 int32_t G, uint8_t* q, uint8_t* sf, uint8_t* qT, int64_t ldT, uint8_t* sfT,
+                                 cudaStream_t stream);
+
 enum GemmMode : int { kFwd = 0, kDgrad = 1, kWgrad = 2 };
 
 // One grouped GEMM.  a/b: operand codes (K-major), lda/ldb their row strides

@@ -6,7 +6,8 @@
 // s = floor(log2 amax) - 8 clamped to [-127, 127], and each element is the
 // E4M3 code of x * 2^-s, rounded to nearest even and saturated to +-448.
 //
-// Both kernels are HBM-bound (2 bytes read, 1 + 1/32 written per element).
+// The kernels are HBM-bound (2 bytes read, 1 + 1/32 written per element and
+// layout; the dual kernel writes both layouts from one read, 4 + 1/16 bytes).
 // A CTA owns one 128-row x 128-column tile, i.e. exactly one 512-byte scale
 // atom of the tcgen05 scale-factor layout, so scales leave the CTA as 32
 // coalesced 16-byte stores.  Rows are read with 16-byte loads, block amax is
@@ -213,6 +214,102 @@ __global__ void __launch_bounds__(kThreads) quantize_colwise_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// Dual: one read of the 128x128 bf16 tile produces both layouts.  The load
+// phase uses the rowwise kernel's thread mapping (four consecutive lanes hold
+// one 32-element row block), so rowwise codes and scales are encoded straight
+// from the loaded registers; the tile then goes to shared memory and the
+// colwise pass proceeds exactly as in quantize_colwise_kernel.
+__global__ void __launch_bounds__(kThreads) quantize_dual_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, const int32_t* __restrict__ offs,
+    int32_t G, uint8_t* __restrict__ q, uint8_t* __restrict__ sf, int64_t pitch_r,
+    uint8_t* __restrict__ qT, int64_t ldT, uint8_t* __restrict__ sfT, int64_t pitch_c) {
+  __shared__ __align__(16) uint32_t tile[128 * 64];
+  __shared__ __align__(16) uint8_t atom_r[512];
+  __shared__ __align__(16) uint8_t atom_c[512];
+  BlockRows br;
+  if (!resolve_block(offs, G, rows, &br)) return;
+  const int t = threadIdx.x, ch = t & 15, rsub = t >> 4;
+  const int64_t col0 = static_cast<int64_t>(blockIdx.y) * 128;
+  const bool col_ok = col0 + 8 * ch < cols;
+
+  uint4 v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int rr = rsub + 16 * i;
+    v[i] = make_uint4(0, 0, 0, 0);
+    if (rr < br.nrows && col_ok) v[i] = ld_stream(x + (br.row0 + rr) * cols + col0 + 8 * ch);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int rr = rsub + 16 * i;
+    uint32_t a = amax_bits8(v[i]);
+    a = max(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    a = max(a, __shfl_xor_sync(0xffffffffu, a, 2));
+    const uint32_t sb = scale_byte(a);
+    if (rr < br.nrows && col_ok)
+      *reinterpret_cast<uint2*>(q + (br.row0 + rr) * cols + col0 + 8 * ch) = encode8(v[i], sb);
+    if ((ch & 3) == 0) atom_r[(rr & 31) * 16 + (rr >> 5) * 4 + (ch >> 2)] = static_cast<uint8_t>(sb);
+    reinterpret_cast<uint4*>(tile)[rr * 16 + ch] = v[i];
+  }
+  __syncthreads();
+  if (t < 32) {
+    const int64_t a = static_cast<int64_t>(blockIdx.x) * pitch_r + blockIdx.y;
+    reinterpret_cast<uint4*>(sf + a * 512)[t] = reinterpret_cast<const uint4*>(atom_r)[t];
+  }
+
+  const int blk = t >> 6, p = t & 63;
+  uint32_t w[32];
+  uint32_t mx = 0;
+#pragma unroll
+  for (int r = 0; r < 32; ++r) {
+    w[r] = tile[(32 * blk + r) * 64 + p];
+    mx = __vmaxu2(mx, w[r] & 0x7FFF7FFFu);
+  }
+  const uint32_t sb_lo = scale_byte(mx & 0xFFFFu), sb_hi = scale_byte(mx >> 16);
+  uint32_t olo[8], ohi[8];
+  {
+    const float flo = inv_scale(sb_lo == 0xFFu ? 0u : sb_lo);
+    const float fhi = inv_scale(sb_hi == 0xFFu ? 0u : sb_hi);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t a0 = cvt_e4m3x2(__fmul_rn(bf_lo(w[4 * j]), flo), __fmul_rn(bf_lo(w[4 * j + 1]), flo));
+      const uint32_t a1 = cvt_e4m3x2(__fmul_rn(bf_lo(w[4 * j + 2]), flo), __fmul_rn(bf_lo(w[4 * j + 3]), flo));
+      const uint32_t b0 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * j]), fhi), __fmul_rn(bf_hi(w[4 * j + 1]), fhi));
+      const uint32_t b1 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * j + 2]), fhi), __fmul_rn(bf_hi(w[4 * j + 3]), fhi));
+      olo[j] = sb_lo == 0xFFu ? 0x7F7F7F7Fu : (a0 | (a1 << 16));
+      ohi[j] = sb_hi == 0xFFu ? 0x7F7F7F7Fu : (b0 | (b1 << 16));
+    }
+  }
+  __syncthreads();
+
+  uint4* stage = reinterpret_cast<uint4*>(tile);
+  const int sw = p & 7;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int chunk = (2 * blk + h) ^ sw;
+    stage[(2 * p) * 8 + chunk] = make_uint4(olo[4 * h], olo[4 * h + 1], olo[4 * h + 2], olo[4 * h + 3]);
+    stage[(2 * p + 1) * 8 + chunk] = make_uint4(ohi[4 * h], ohi[4 * h + 1], ohi[4 * h + 2], ohi[4 * h + 3]);
+  }
+  {
+    const int r0 = 2 * p, r1 = 2 * p + 1;
+    atom_c[(r0 & 31) * 16 + (r0 >> 5) * 4 + blk] = static_cast<uint8_t>(sb_lo);
+    atom_c[(r1 & 31) * 16 + (r1 >> 5) * 4 + blk] = static_cast<uint8_t>(sb_hi);
+  }
+  __syncthreads();
+
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int id = t + kThreads * i, c = id >> 3, j = id & 7;
+    if (col0 + c < cols && 16 * j < br.padded)
+      *reinterpret_cast<uint4*>(qT + (col0 + c) * ldT + br.dst0 + 16 * j) = stage[c * 8 + (j ^ ((c >> 1) & 7))];
+  }
+  if (t < 32) {
+    const int64_t a = static_cast<int64_t>(blockIdx.y) * pitch_c + blockIdx.x;
+    reinterpret_cast<uint4*>(sfT + a * 512)[t] = reinterpret_cast<const uint4*>(atom_c)[t];
+  }
+}
+
 int64_t block_bound(int64_t rows, int32_t G) { return rows == 0 ? 0 : (rows + 127) / 128 + G - 1; }
 
 }  // namespace
@@ -234,6 +331,17 @@ cudaError_t launch_quantize_colwise(const uint16_t* x, int64_t rows, int64_t col
   if (nb == 0) return cudaSuccess;
   const dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>((cols + 127) / 128));
   quantize_colwise_kernel<<<grid, kThreads, 0, stream>>>(x, rows, cols, offs, G, qT, ldT, sfT, nb);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_dual(const uint16_t* x, int64_t rows, int64_t cols, const int32_t* offs,
+                                 int32_t G, uint8_t* q, uint8_t* sf, uint8_t* qT, int64_t ldT, uint8_t* sfT,
+                                 cudaStream_t stream) {
+  const int64_t nb = block_bound(rows, G);
+  if (nb == 0) return cudaSuccess;
+  const dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>((cols + 127) / 128));
+  quantize_dual_kernel<<<grid, kThreads, 0, stream>>>(x, rows, cols, offs, G, q, sf, (cols + 127) / 128, qT, ldT,
+                                                       sfT, nb);
   return cudaGetLastError();
 }
 

@@ -19,6 +19,19 @@ pytestmark = pytest.mark.gpu
 POISON = 0x7FC0  # bf16 NaN: any output element the kernel fails to write stays NaN
 
 
+@pytest.fixture(params=["default", "1cta", "pair"])
+def tile_config(request, monkeypatch):
+    """Runs a test under the per-pass default tile configuration, forced
+    1-CTA 128x256 tiles, and forced CTA-pair 256x256 tiles."""
+    if request.param == "1cta":
+        monkeypatch.setenv("MXF8_GEMM_CTA_PAIR", "0")
+    elif request.param == "pair":
+        monkeypatch.setenv("MXF8_GEMM_CTA_PAIR", "1")
+    else:
+        monkeypatch.delenv("MXF8_GEMM_CTA_PAIR", raising=False)
+    return request.param
+
+
 @pytest.fixture(scope="module")
 def mx():
     import mxfp8_grouped_gemm_quantize_b200 as m
@@ -123,7 +136,7 @@ def make_case(mx, counts, N, K, seed=0, w_std=1.0, check_quant=True):
     return Case(mx, X, W, dY, offs, check_quant)
 
 
-def test_tiny_config(mx):
+def test_tiny_config(mx, tile_config):
     w = wl.tiny()
     X, W, dY = wl.layer_tensors(w, w.layers[0])
     run_all_and_compare(Case(mx, X, W, dY, w.offsets))
@@ -134,13 +147,13 @@ def test_tiny_random_counts(mx, seed):
     run_all_and_compare(make_case(mx, wl.tiny_random(seed), 128, 256, seed))
 
 
-def test_ragged_multi_tile(mx):
+def test_ragged_multi_tile(mx, tile_config):
     """Several 128x256 tiles per group, ragged tails, an empty expert, a
     partial output tile (N = 384) and a partial K block (K = 416)."""
     run_all_and_compare(make_case(mx, [0, 1, 129, 300, 77, 255], 384, 416, seed=7))
 
 
-def test_small_integer_operands_exact(mx):
+def test_small_integer_operands_exact(mx, tile_config):
     counts = [0, 7, 21, 36, 200, 1, 130]
     offs = wl.offsets_from_counts(counts)
     M, E, N, K = int(offs[-1]), len(counts), 256, 512
@@ -150,7 +163,7 @@ def test_small_integer_operands_exact(mx):
     run_all_and_compare(Case(mx, X, W, dY, offs), exact=True)
 
 
-def test_distinct_block_scales_pin_the_scale_layout(mx):
+def test_distinct_block_scales_pin_the_scale_layout(mx, tile_config):
     """Every 32-block gets its own power-of-two magnitude, so a scale read
     from the wrong row or block breaks parity."""
     counts = [50, 0, 170, 33]
@@ -172,15 +185,15 @@ def test_distinct_block_scales_pin_the_scale_layout(mx):
 
 @pytest.mark.parametrize("counts,N,K", [([1], 128, 32), ([0, 0, 5], 128, 64), ([300], 128, 160),
                                         ([3, 0, 0, 0], 256, 1024), ([129, 127], 512, 96)])
-def test_edge_shapes(mx, counts, N, K):
+def test_edge_shapes(mx, tile_config, counts, N, K):
     run_all_and_compare(make_case(mx, counts, N, K, seed=sum(counts)))
 
 
-def test_all_rows_in_one_expert(mx):
+def test_all_rows_in_one_expert(mx, tile_config):
     run_all_and_compare(make_case(mx, [0, 0, 400, 0], 256, 256, seed=3))
 
 
-def test_zero_rows(mx):
+def test_zero_rows(mx, tile_config):
     """M = 0: fwd/dgrad have nothing to write; wgrad writes dW = 0."""
     c = make_case(mx, [0, 0], 128, 64, check_quant=False)
     bdw, dw = poisoned((2, 128, 64))

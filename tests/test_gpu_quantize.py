@@ -221,3 +221,66 @@ def test_grouped_full_size_sampled_groups(mx, name):
         for c in range(0, K, 97):
             for j in range((m + 31) // 32):
                 assert gsfT[oracle.sf_offset(c, 4 * int(RB[g]) + j, cpitch)] == osfT[oracle.sf_offset(c, j, sp)]
+
+
+# ------------------------------------------------------------------ dual (rowwise + colwise from one read)
+def check_dual(mx, x: torch.Tensor, offs=None):
+    R, C = x.shape
+    q, sf, qT, sfT = mx.mxfp8_quantize_dual(x.cuda(), _offs_dev(offs))
+    torch.cuda.synchronize()
+    rq, rsf = oracle.quantize_rowwise(x, offs)
+    cq, csf = oracle.quantize_colwise(x, offs)
+    RB, PG = oracle.group_blocks(offs, R)
+    np.testing.assert_array_equal(np_u8(q), rq)
+    n = RB * oracle.rowwise_pitch(C) * 512
+    np.testing.assert_array_equal(np_u8(sf)[:n], rsf[:n])
+    np.testing.assert_array_equal(np_u8(qT)[:, :PG], cq[:, :PG])
+    pitch = oracle.colwise_pitch(R, 1 if offs is None else len(offs) - 1)
+    g = np_u8(sfT)
+    for rb in range((C + 127) // 128):
+        a = rb * pitch
+        np.testing.assert_array_equal(g[a * 512:(a + RB) * 512], csf[a * 512:(a + RB) * 512])
+
+
+@pytest.mark.parametrize("order", ["sorted", "shuffled"])
+def test_dual_every_finite_bf16_pattern(mx, order):
+    check_dual(mx, _all_finite_bf16(order))
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_dual_grouped(mx, seed):
+    counts = np.array([0, 1, 31, 32, 33, 127, 128, 129, 0, 300, 7], dtype=np.int64)
+    counts = np.random.default_rng(seed + 10).permutation(counts)
+    offs = wl.offsets_from_counts(counts)
+    x = wl.with_outliers(wl.normal_bf16((int(offs[-1]), 416), 1.0, seed + 20), 0.01, 1000.0, seed)
+    check_dual(mx, x, offs)
+
+
+def test_dual_tiny_and_edges(mx):
+    w = wl.tiny()
+    X, W, dY = wl.layer_tensors(w, w.layers[0])
+    check_dual(mx, X, w.offsets)
+    check_dual(mx, W.reshape(-1, W.shape[-1]))
+    check_dual(mx, torch.zeros((1, 32), dtype=torch.bfloat16))
+    check_dual(mx, wl.normal_bf16((3, 96), 1.0, 1), [0, 0, 3, 3])
+
+
+def test_dual_matches_separate_at_workload_size(mx):
+    """DeepSeek-V3-16B-like X (49152 x 2048, 64 groups): dual output equals
+    the separate rowwise and colwise kernels' output byte for byte."""
+    w = wl.ds_v3_16b()
+    X, _, _ = wl.layer_tensors(w, w.layers[0], device="cuda")
+    od = torch.from_numpy(w.offsets).cuda()
+    q, sf, qT, sfT = mx.mxfp8_quantize_dual(X, od)
+    q2, sf2 = mx.mxfp8_quantize_rowwise(X, od)
+    qT2, sfT2 = mx.mxfp8_quantize_colwise(X, od)
+    torch.cuda.synchronize()
+    RB, PG = oracle.group_blocks(w.offsets, w.M)
+    assert torch.equal(q, q2)
+    n = RB * oracle.rowwise_pitch(X.shape[1]) * 512
+    assert torch.equal(sf[:n], sf2[:n])
+    assert torch.equal(qT[:, :PG], qT2[:, :PG])
+    pitch = oracle.colwise_pitch(w.M, w.E)
+    for rb in range(X.shape[1] // 128):
+        a = rb * pitch
+        assert torch.equal(sfT[a * 512:(a + RB) * 512], sfT2[a * 512:(a + RB) * 512])
