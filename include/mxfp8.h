@@ -185,6 +185,42 @@ MXF8_API mxf8_status mxfp8_grouped_gemm_wgrad(const uint8_t* dyqT, const uint8_t
                                      int64_t K, uint16_t* dw, void* work, int64_t work_bytes,
                                      void* stream);
 
+/* Fwd and dgrad with a quantising epilogue: the GEMM's output, rounded to
+ * bf16 as in mxfp8_grouped_gemm_fwd/_dgrad, is also written as MXFP8 straight
+ * from the accumulator, so a following MXFP8 GEMM needs no separate
+ * quantisation pass over it.  The copies are exactly (byte for byte) what
+ *   mxfp8_quantize_rowwise(out, rows = M, cols = C, d_offs, E, q, scales) and
+ *   mxfp8_quantize_colwise(out, rows = M, cols = C, d_offs, E, qT, ldT, scalesT)
+ * would write from the bf16 output (C = N for fwd, K for dgrad): the MXFP8
+ * block encoding of opensourcebeat.com, "Enabling up to 41% faster
+ * pre-training: MXFP8 and DeepEP ...", FAQ (OCP MX v1.0), and the layouts at
+ * the top of this header.  The pages do not describe this fusion; it
+ * follows that page's section "Двухсторонняя атака: MXFP8 и DeepEP", which
+ * credits the speed-up to the pipeline as a whole being reworked rather than
+ * to one kernel.  The arithmetic is exactly that of the quantisers.
+ *   out      bf16 [M, C] or NULL (not written)
+ *   q        uint8 [M, C] rowwise codes or NULL; scales (>= scale_bytes =
+ *            mxfp8_rowwise_scale_bytes(M, C, E)) must be given with q
+ *   qT       uint8 [C, ldT] colwise codes or NULL, ldT = mxfp8_colwise_ld(M, E);
+ *            scalesT (>= scaleT_bytes = mxfp8_colwise_scale_bytes(M, C, E))
+ *            must be given with qT
+ * At least one of out, q, qT must be non-NULL.  Other arguments, errors and
+ * the device status are those of mxfp8_grouped_gemm_fwd / _dgrad. */
+MXF8_API mxf8_status mxfp8_grouped_gemm_fwd_quant(const uint8_t* xq, const uint8_t* xs, int64_t xs_bytes,
+                                                  const uint8_t* wq, const uint8_t* ws, int64_t ws_bytes,
+                                                  const int32_t* d_offs, int32_t E, int64_t M, int64_t N,
+                                                  int64_t K, uint16_t* y, uint8_t* q, uint8_t* scales,
+                                                  int64_t scale_bytes, uint8_t* qT, int64_t ldT,
+                                                  uint8_t* scalesT, int64_t scaleT_bytes, void* work,
+                                                  int64_t work_bytes, void* stream);
+MXF8_API mxf8_status mxfp8_grouped_gemm_dgrad_quant(const uint8_t* dyq, const uint8_t* dys, int64_t dys_bytes,
+                                                    const uint8_t* wqT, const uint8_t* wsT, int64_t wsT_bytes,
+                                                    const int32_t* d_offs, int32_t E, int64_t M, int64_t N,
+                                                    int64_t K, uint16_t* dx, uint8_t* q, uint8_t* scales,
+                                                    int64_t scale_bytes, uint8_t* qT, int64_t ldT,
+                                                    uint8_t* scalesT, int64_t scaleT_bytes, void* work,
+                                                    int64_t work_bytes, void* stream);
+
 /* Forward grouped GEMM that allocates nothing and takes no workspace.
  * The paper has no counterpart to this entry point; it exists for callers
  * that cannot call cudaMalloc (for example a plugin inside an engine that owns

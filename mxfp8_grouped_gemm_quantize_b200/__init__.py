@@ -35,7 +35,8 @@ EXPORTED = ("mxfp8_rowwise_scale_bytes", "mxfp8_colwise_pitch", "mxfp8_colwise_s
             "mxfp8_workspace_bytes", "mxfp8_quantize_rowwise", "mxfp8_quantize_colwise",
             "mxfp8_grouped_gemm_fwd", "mxfp8_grouped_gemm_dgrad", "mxfp8_grouped_gemm_wgrad",
             "mxfp8_get_status", "mxfp8_status_string", "mxfp8_last_cuda_error", "mxfp8_device_supported",
-            "mxfp8_grouped_gemm_fwd_noalloc", "mxfp8_quantize_dual")
+            "mxfp8_grouped_gemm_fwd_noalloc", "mxfp8_quantize_dual", "mxfp8_grouped_gemm_fwd_quant",
+            "mxfp8_grouped_gemm_dgrad_quant")
 
 
 class MXFP8Error(RuntimeError):
@@ -73,6 +74,10 @@ def lib() -> ctypes.CDLL:
         for n in ("mxfp8_grouped_gemm_fwd", "mxfp8_grouped_gemm_dgrad", "mxfp8_grouped_gemm_wgrad"):
             getattr(L, n).restype = _i32
             getattr(L, n).argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp, _vp, _i64, _vp]
+        for n in ("mxfp8_grouped_gemm_fwd_quant", "mxfp8_grouped_gemm_dgrad_quant"):
+            getattr(L, n).restype = _i32
+            getattr(L, n).argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i64,
+                                      _vp, _i64, _vp, _i64, _vp, _i64, _vp]
         L.mxfp8_grouped_gemm_fwd_noalloc.restype = _i32
         L.mxfp8_grouped_gemm_fwd_noalloc.argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp,
                                                      ctypes.POINTER(_i32), _vp]
@@ -210,6 +215,51 @@ def mxfp8_grouped_gemm_wgrad(dyqT, dysT, xqT, xsT, offs, M: int, out=None, work=
     E = _groups(offs)
     out = out if out is not None else torch.empty((E, N, K), dtype=torch.bfloat16, device=dyqT.device)
     return _gemm("mxfp8_grouped_gemm_wgrad", dyqT, dysT, xqT, xsT, offs, M, N, K, out, work, stream)
+
+
+def _gemm_quant(fn, a, a_s, b, b_s, offs, M, N, K, C, out, rowwise, colwise, work, stream):
+    E = _groups(offs)
+    dev = a.device
+    q = scales = qT = scalesT = None
+    ld = mxfp8_colwise_ld(M, E)
+    if rowwise is True:
+        rowwise = (torch.empty((M, C), dtype=torch.uint8, device=dev), _u8(mxfp8_rowwise_scale_bytes(M, C, E), dev))
+    if rowwise:
+        q, scales = rowwise
+    if colwise is True:
+        colwise = (torch.empty((C, ld), dtype=torch.uint8, device=dev), _u8(mxfp8_colwise_scale_bytes(M, C, E), dev))
+    if colwise:
+        qT, scalesT = colwise
+    work = work if work is not None else new_workspace(E, M, N, K, dev)
+    _check(getattr(lib(), fn)(_ptr(a), _ptr(a_s), a_s.numel(), _ptr(b), _ptr(b_s), b_s.numel(), _ptr(offs), E, M, N,
+                              K, _ptr(out), _ptr(q), _ptr(scales), scales.numel() if scales is not None else 0,
+                              _ptr(qT), ld, _ptr(scalesT), scalesT.numel() if scalesT is not None else 0,
+                              _ptr(work), work.numel(), _stream(stream)), fn)
+    return out, q, scales, qT, scalesT
+
+
+def mxfp8_grouped_gemm_fwd_quant(xq, xs, wq, ws, offs, N: int, out=True, rowwise=True, colwise=True, work=None,
+                                 stream=None):
+    """Forward GEMM whose epilogue also writes Y as MXFP8, byte for byte what
+    mxfp8_quantize_rowwise / _colwise(Y, offs) give.  out / rowwise / colwise:
+    True = allocate, False/None = skip, or the buffers ((q, scales) and
+    (qT, scalesT) for the quantised copies).  Returns (y, q, scales, qT, scalesT)."""
+    M, K = xq.shape
+    if out is True:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    return _gemm_quant("mxfp8_grouped_gemm_fwd_quant", xq, xs, wq, ws, offs, M, N, K, N, out if isinstance(out, torch.Tensor) else None, rowwise,
+                       colwise, work, stream)
+
+
+def mxfp8_grouped_gemm_dgrad_quant(dyq, dys, wqT, wsT, offs, K: int, out=True, rowwise=True, colwise=True,
+                                   work=None, stream=None):
+    """Dgrad GEMM whose epilogue also writes dX as MXFP8 (see
+    mxfp8_grouped_gemm_fwd_quant).  Returns (dx, q, scales, qT, scalesT)."""
+    M, N = dyq.shape
+    if out is True:
+        out = torch.empty((M, K), dtype=torch.bfloat16, device=dyq.device)
+    return _gemm_quant("mxfp8_grouped_gemm_dgrad_quant", dyq, dys, wqT, wsT, offs, M, N, K, K, out if isinstance(out, torch.Tensor) else None, rowwise,
+                       colwise, work, stream)
 
 
 def mxfp8_grouped_gemm_fwd_noalloc(xq, xs, wq, ws, offs, N: int, out=None, stream=None, want_status=False):

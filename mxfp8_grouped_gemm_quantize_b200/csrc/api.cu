@@ -88,6 +88,27 @@ mxf8_status run_gemm(mxf8::GemmArgs& g, void* work, void* stream) {
   return MXF8_OK;
 }
 
+// Quantising epilogue: checks the output copies and attaches them to g.
+// C = columns of the GEMM output.  `out` may be NULL when a copy is asked for.
+mxf8_status attach_quant_outputs(mxf8::GemmArgs& g, int64_t C, const uint16_t* out, uint8_t* q,
+                                 uint8_t* scales, int64_t scale_bytes, uint8_t* qT, int64_t ldT,
+                                 uint8_t* scalesT, int64_t scaleT_bytes) {
+  if (!out && !q && !qT) return MXF8_ERR_INVALID_ARG;
+  if (q) {
+    if (!scales || scale_bytes < mxfp8_rowwise_scale_bytes(g.M, C, g.E)) return MXF8_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(scales)) return MXF8_ERR_ALIGNMENT;
+  }
+  if (qT) {
+    if (!scalesT || ldT != mxfp8_colwise_ld(g.M, g.E) || scaleT_bytes < mxfp8_colwise_scale_bytes(g.M, C, g.E))
+      return MXF8_ERR_INVALID_ARG;
+    if (!aligned16(qT) || !aligned16(scalesT)) return MXF8_ERR_ALIGNMENT;
+  }
+  g.qr = q; g.sr = q ? scales : nullptr;
+  g.qc = qT; g.sc = qT ? scalesT : nullptr;
+  g.qc_ld = ldT; g.sc_pitch = mxfp8_colwise_pitch(g.M, g.E);
+  return MXF8_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -229,6 +250,60 @@ mxf8_status mxfp8_grouped_gemm_wgrad(const uint8_t* dyqT, const uint8_t* dysT, i
     // M = 0: no scale atoms exist; point at the (unread) code buffers instead.
     g.sfa = dyqT; g.sfb = xqT; g.sfa_atoms = g.sfb_atoms = 1;
   }
+  return run_gemm(g, work, stream);
+}
+
+mxf8_status mxfp8_grouped_gemm_fwd_quant(const uint8_t* xq, const uint8_t* xs, int64_t xs_bytes, const uint8_t* wq,
+                                         const uint8_t* ws, int64_t ws_bytes, const int32_t* d_offs, int32_t E,
+                                         int64_t M, int64_t N, int64_t K, uint16_t* y, uint8_t* q, uint8_t* scales,
+                                         int64_t scale_bytes, uint8_t* qT, int64_t ldT, uint8_t* scalesT,
+                                         int64_t scaleT_bytes, void* work, int64_t work_bytes, void* stream) {
+  // The output pointer check of the plain GEMM applies to whichever output exists.
+  const void* any_out = y ? static_cast<const void*>(y) : (q ? static_cast<const void*>(q) : qT);
+  mxf8_status s = check_gemm_args({xq, xs, xs_bytes, wq, ws, ws_bytes, d_offs, E, M, N, K, any_out, work, work_bytes});
+  if (s != MXF8_OK) return s;
+  if (xs_bytes < mxfp8_rowwise_scale_bytes(M, K, E) || ws_bytes < mxfp8_rowwise_scale_bytes(E * N, K, 1))
+    return MXF8_ERR_INVALID_ARG;
+  mxf8::GemmArgs g{};
+  g.mode = mxf8::kFwd; g.E = E; g.M = M; g.N = N; g.K = K; g.offs = d_offs;
+  if ((s = attach_quant_outputs(g, N, y, q, scales, scale_bytes, qT, ldT, scalesT, scaleT_bytes)) != MXF8_OK)
+    return s;
+  if ((s = check_device()) != MXF8_OK) return s;
+  if (M == 0) return cudaMemsetAsync(work, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) == cudaSuccess
+                         ? MXF8_OK : cuda_fail(cudaGetLastError(), "cudaMemsetAsync(status)");
+  g.a = xq; g.lda = K; g.a_rows = M; g.a_cols = K;
+  g.b = wq; g.ldb = K; g.b_rows = E * N; g.b_cols = K;
+  g.sfa = xs; g.sfa_pitch = cdiv(K, 128); g.sfa_atoms = xs_bytes / 512;
+  g.sfb = ws; g.sfb_pitch = cdiv(K, 128); g.sfb_atoms = ws_bytes / 512;
+  g.out = y;
+  return run_gemm(g, work, stream);
+}
+
+mxf8_status mxfp8_grouped_gemm_dgrad_quant(const uint8_t* dyq, const uint8_t* dys, int64_t dys_bytes,
+                                           const uint8_t* wqT, const uint8_t* wsT, int64_t wsT_bytes,
+                                           const int32_t* d_offs, int32_t E, int64_t M, int64_t N, int64_t K,
+                                           uint16_t* dx, uint8_t* q, uint8_t* scales, int64_t scale_bytes,
+                                           uint8_t* qT, int64_t ldT, uint8_t* scalesT, int64_t scaleT_bytes,
+                                           void* work, int64_t work_bytes, void* stream) {
+  const void* any_out = dx ? static_cast<const void*>(dx) : (q ? static_cast<const void*>(q) : qT);
+  mxf8_status s =
+      check_gemm_args({dyq, dys, dys_bytes, wqT, wsT, wsT_bytes, d_offs, E, M, N, K, any_out, work, work_bytes});
+  if (s != MXF8_OK) return s;
+  if (dys_bytes < mxfp8_rowwise_scale_bytes(M, N, E) || wsT_bytes < mxfp8_colwise_scale_bytes(E * N, K, 1))
+    return MXF8_ERR_INVALID_ARG;
+  mxf8::GemmArgs g{};
+  g.mode = mxf8::kDgrad; g.E = E; g.M = M; g.N = N; g.K = K; g.offs = d_offs;
+  if ((s = attach_quant_outputs(g, K, dx, q, scales, scale_bytes, qT, ldT, scalesT, scaleT_bytes)) != MXF8_OK)
+    return s;
+  if ((s = check_device()) != MXF8_OK) return s;
+  if (M == 0) return cudaMemsetAsync(work, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) == cudaSuccess
+                         ? MXF8_OK : cuda_fail(cudaGetLastError(), "cudaMemsetAsync(status)");
+  const int64_t ldw = mxfp8_colwise_ld(E * N, 1);
+  g.a = dyq; g.lda = N; g.a_rows = M; g.a_cols = N;
+  g.b = wqT; g.ldb = ldw; g.b_rows = K; g.b_cols = ldw;
+  g.sfa = dys; g.sfa_pitch = cdiv(N, 128); g.sfa_atoms = dys_bytes / 512;
+  g.sfb = wsT; g.sfb_pitch = mxfp8_colwise_pitch(E * N, 1); g.sfb_atoms = wsT_bytes / 512;
+  g.out = dx;
   return run_gemm(g, work, stream);
 }
 

@@ -39,6 +39,7 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "codec.cuh"
 #include "launch.h"
 #include "mxfp8.h"
 #include "ptx.cuh"
@@ -53,41 +54,50 @@ constexpr int EPI_STAGE = 32 * 128;        // one epilogue buffer: 32 rows x 64 
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_STRIDE = 12;        // per stage: SFA 4 columns, then SFB 8 columns
 constexpr int MAXG = MXF8_GEMM_MAX_GROUPS;
-#ifndef MXF8_PAIR_STAGES
-#define MXF8_PAIR_STAGES 5
-#endif
-#ifndef MXF8_PAIR_EPI_BUFS
-#define MXF8_PAIR_EPI_BUFS 2
-#endif
 constexpr int SCHED_INTS = 4 * (MAXG + 1);
 
 constexpr int round_up_c(int a, int b) { return (a + b - 1) / b * b; }
 
-template <int CG>
+// Pipeline shape: CG CTAs per MMA, KS 128-wide K blocks per stage.  The ring
+// takes as many stages as shared memory holds: 1 CTA: 4 x 128-deep or
+// 2 x 256-deep; pair: 5 x 128-deep or 3 x 256-deep.  Deeper stages amortise
+// the fixed cost of a stage hand-off (barrier round trip, copy issue) over
+// twice the MMAs.
+template <int CG, int KS_>
 struct Cfg {
-  static constexpr int STAGES = CG == 2 ? MXF8_PAIR_STAGES : 4;
+  static constexpr int KS = KS_;
+  static constexpr int STAGES = CG == 2 ? (KS == 2 ? 3 : 5) : (KS == 2 ? 2 : 4);
+  static constexpr int SLOTS = STAGES * KS;            // 128-wide K-block slots in the ring
   static constexpr int B_ROWS = BN / CG;               // B rows staged by each CTA
   static constexpr int A_TILE = BM * BK;               // 16 KB of E4M3 codes
   static constexpr int B_TILE = B_ROWS * BK;
-  static constexpr int EPI_BUFS = CG == 2 ? MXF8_PAIR_EPI_BUFS : 1;
+  static constexpr int EPI_BUFS = (CG == 2 && KS == 1) ? 2 : 1;
   // The two 128x256 accumulators overlap in OV 64-column chunks: accumulator 1
-  // starts at column ACC_STRIDE, and the scale sets of all stages follow it.
-  static constexpr int OV = (STAGES * SF_STRIDE <= 64) ? 1 : 2;
+  // starts at column ACC_STRIDE, and the scale sets of all slots follow it.
+  static constexpr int OV = (SLOTS * SF_STRIDE <= 64) ? 1 : 2;
   static constexpr uint32_t ACC_STRIDE = 256 - 64 * OV;
   static constexpr uint32_t SF_COL = ACC_STRIDE + 256;
-  static constexpr uint32_t STAGE_TX = CG * (A_TILE + B_TILE + SFA_TILE + SFB_TILE);
+  // Bytes one CTA pair (or CTA) receives for a stage holding `nh` K blocks:
+  // the scale boxes always span all KS atoms.
+  static constexpr uint32_t stage_tx(int nh) {
+    return CG * (nh * (A_TILE + B_TILE) + KS * (SFA_TILE + SFB_TILE));
+  }
+  // Slot q = stage * KS + h.  Scale atoms of one stage are fetched as boxes of
+  // KS consecutive atoms: SFA box at OFF_SFA + stage * KS * 512, the two SFB
+  // boxes (B rows 0-127, 128-255) at OFF_SFB + stage * 2 * KS * 512 (+ KS * 512).
   static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * A_TILE;
-  static constexpr int OFF_SFA = OFF_B + STAGES * B_TILE;
-  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_TILE;
-  static constexpr int OFF_EPI = round_up_c(OFF_SFB + STAGES * SFB_TILE, 1024);
+  static constexpr int OFF_B = OFF_A + SLOTS * A_TILE;
+  static constexpr int OFF_SFA = OFF_B + SLOTS * B_TILE;
+  static constexpr int OFF_SFB = OFF_SFA + SLOTS * SFA_TILE;
+  static constexpr int OFF_EPI = round_up_c(OFF_SFB + SLOTS * SFB_TILE, 1024);
   static constexpr int OFF_BAR = OFF_EPI + 4 * EPI_BUFS * EPI_STAGE;
   static constexpr int OFF_MISC = OFF_BAR + 128;
   static constexpr int OFF_SCHED = OFF_MISC + 64;
   static constexpr int SMEM_BYTES = OFF_SCHED + SCHED_INTS * 4 + 1024;   // + slack to align the base
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(OFF_B % 1024 == 0 && B_TILE % 1024 == 0 && OFF_EPI % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-  static_assert(SF_COL + SF_STRIDE * STAGES <= TMEM_COLS, "scale columns");
+  static_assert(SF_COL + SF_STRIDE * SLOTS <= TMEM_COLS, "scale columns");
+  static_assert(KS >= 1 && KS <= 2 && STAGES >= 2, "pipeline shape");
   static_assert((2 * STAGES + 3) * 8 <= 128, "barrier area");
 };
 
@@ -97,10 +107,18 @@ struct Params {
   int64_t M, N, K;
   const int32_t* offs;
   int64_t sfa_pitch, sfb_pitch;        // atoms per atom row of the A / B scale matrices
-  uint16_t* out;                       // output (fwd [M,N], dgrad [M,K], wgrad [E*N,K])
+  uint16_t* out;                       // output (fwd [M,N], dgrad [M,K], wgrad [E*N,K]); may be
+                                       // null in a quantising epilogue
   int64_t out_ld;                      // output row stride (elements)
   int32_t* status;
   uint64_t timeout_ns;
+  // Quantising epilogue (fwd/dgrad): MXFP8 copies of the bf16 output, in the
+  // quantisers' layouts with the GEMM's groups.  Null pointers skip a layout.
+  uint8_t* qr;                         // rowwise codes [M, out_ld]
+  uint8_t* sr;                         // rowwise scale atoms, pitch ceil(out_ld / 128)
+  uint8_t* qc;                         // colwise codes [out_ld, qc_ld] (transposed)
+  uint8_t* sc;                         // colwise scale atoms, pitch sc_pitch
+  int64_t qc_ld, sc_pitch;
 };
 
 // Per-CTA schedule, built from the offsets by warp 0.
@@ -120,6 +138,9 @@ struct Tile {
   int64_t sfa_atom, sfb_atom0, sfb_atom1;   // scale atoms of the first K block
   int64_t out_row, out_col;             // output element (row, col) of this CTA's tile corner
   int32_t rows, cols;    // valid rows (0..128) and columns (<= 256) of this CTA's tile
+  int32_t q_rb;          // fwd/dgrad: RB_e + row block, the output's rowwise scale atom row
+                         //            and colwise scale atom column
+  int32_t q_p;           // fwd/dgrad: P_e + 128 * row block, the output's colwise code column
 };
 
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
@@ -159,6 +180,7 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int
     tl.b_x = 0;                              tl.b_y = static_cast<int32_t>(e * p.N) + BN * nt + b_half;
     sfa_row = s.rb[e] + mt;                  sfa_col = 0;
     sfb_row = e * (p.N / 128) + 2 * nt;      sfb_col = 0;
+    tl.q_rb = s.rb[e] + mt;                  tl.q_p = s.p[e] + BM * mt;
     tl.out_row = int64_t(row0) + BM * mt;
     tl.rows = static_cast<int32_t>(min64(BM, m - BM * mt));
     out_cols = p.N;
@@ -167,6 +189,7 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int
     tl.b_x = static_cast<int32_t>(e * p.N);  tl.b_y = BN * nt + b_half;
     sfa_row = s.rb[e] + mt;                  sfa_col = 0;
     sfb_row = 2 * nt;                        sfb_col = e * (p.N / 128);
+    tl.q_rb = s.rb[e] + mt;                  tl.q_p = s.p[e] + BM * mt;
     tl.out_row = int64_t(row0) + BM * mt;
     tl.rows = static_cast<int32_t>(min64(BM, m - BM * mt));
     out_cols = p.K;
@@ -175,6 +198,7 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int
     tl.b_x = s.p[e];                         tl.b_y = BN * nt + b_half;
     sfa_row = mt;                            sfa_col = s.rb[e];
     sfb_row = 2 * nt;                        sfb_col = s.rb[e];
+    tl.q_rb = 0;                             tl.q_p = 0;
     tl.out_row = int64_t(e) * p.N + BM * mt;
     tl.rows = static_cast<int32_t>(min64(BM, p.N - int64_t(BM) * mt));
     out_cols = p.K;
@@ -251,12 +275,12 @@ __device__ __forceinline__ void tmem_wait_regs(uint32_t (&r)[32]) {
                : "memory");
 }
 
-template <int CG>
+template <int CG, int KS, bool QE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                     const __grid_constant__ CUtensorMap tmOut, const Params p) {
-  using C = Cfg<CG>;
+  using C = Cfg<CG, KS>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -323,37 +347,49 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       bool failed = false;
       for (int32_t t = unit0; t < total && !failed; t += nunits) {
         const Tile tl = decode_tile<CG>(p, sc, t, rank);
-        for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
+        for (int32_t kb0 = 0; kb0 < tl.kblocks; kb0 += C::KS) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
           if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, lim)) {
             record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
             failed = true;
             break;
           }
+          const int32_t nh = min(C::KS, tl.kblocks - kb0);   // K blocks in this stage
           const uint32_t fb = full_bar(s);
-          const uint32_t sa = smem_addr(smem + C::OFF_A + s * C::A_TILE);
-          const uint32_t sb = smem_addr(smem + C::OFF_B + s * C::B_TILE);
-          const uint32_t ssa = smem_addr(smem + C::OFF_SFA + s * SFA_TILE);
-          const uint32_t ssb = smem_addr(smem + C::OFF_SFB + s * SFB_TILE);
-          // Scale atoms are 4 rows of 128 bytes in the scale maps; atoms past
-          // the buffer read as zero (they only ever feed masked outputs).
-          const int32_t ya = static_cast<int32_t>(4 * (tl.sfa_atom + kb));
-          const int32_t yb0 = static_cast<int32_t>(4 * (tl.sfb_atom0 + kb));
-          const int32_t yb1 = static_cast<int32_t>(4 * (tl.sfb_atom1 + kb));
+          const uint32_t ssa = smem_addr(smem + C::OFF_SFA + s * C::KS * SFA_TILE);
+          const uint32_t ssb = smem_addr(smem + C::OFF_SFB + s * C::KS * SFB_TILE);
+          // Scale atoms are 4 rows of 128 bytes in the scale maps; each box
+          // takes KS consecutive atoms (those past the tile's K blocks are
+          // fetched but unused; atoms past the buffer read as zero).
+          const int32_t ya = static_cast<int32_t>(4 * (tl.sfa_atom + kb0));
+          const int32_t yb0 = static_cast<int32_t>(4 * (tl.sfb_atom0 + kb0));
+          const int32_t yb1 = static_cast<int32_t>(4 * (tl.sfb_atom1 + kb0));
           if constexpr (CG == 2) {
-            if (leader) mbar_arrive_expect_tx(fb, C::STAGE_TX);   // both CTAs' bytes land here
-            tma_load_2d_pair(sa, &tmA, tl.a_x + BK * kb, tl.a_y, fb);
-            tma_load_2d_pair(sb, &tmB, tl.b_x + BK * kb, tl.b_y, fb);
+            if (leader) mbar_arrive_expect_tx(fb, C::stage_tx(nh));   // both CTAs' bytes land here
+          } else {
+            mbar_arrive_expect_tx(fb, C::stage_tx(nh));
+          }
+          for (int32_t h = 0; h < nh; ++h) {
+            const uint32_t q = s * C::KS + h;
+            const uint32_t sa = smem_addr(smem + C::OFF_A + q * C::A_TILE);
+            const uint32_t sb = smem_addr(smem + C::OFF_B + q * C::B_TILE);
+            const int32_t kx = BK * (kb0 + h);
+            if constexpr (CG == 2) {
+              tma_load_2d_pair(sa, &tmA, tl.a_x + kx, tl.a_y, fb);
+              tma_load_2d_pair(sb, &tmB, tl.b_x + kx, tl.b_y, fb);
+            } else {
+              tma_load_2d(sa, &tmA, tl.a_x + kx, tl.a_y, fb);
+              tma_load_2d(sb, &tmB, tl.b_x + kx, tl.b_y, fb);
+            }
+          }
+          if constexpr (CG == 2) {
             tma_load_2d_pair(ssa, &tmSFA, 0, ya, fb);
             tma_load_2d_pair(ssb, &tmSFB, 0, yb0, fb);
-            tma_load_2d_pair(ssb + 512, &tmSFB, 0, yb1, fb);
+            tma_load_2d_pair(ssb + C::KS * 512, &tmSFB, 0, yb1, fb);
           } else {
-            mbar_arrive_expect_tx(fb, C::STAGE_TX);
-            tma_load_2d(sa, &tmA, tl.a_x + BK * kb, tl.a_y, fb);
-            tma_load_2d(sb, &tmB, tl.b_x + BK * kb, tl.b_y, fb);
             tma_load_2d(ssa, &tmSFA, 0, ya, fb);
             tma_load_2d(ssb, &tmSFB, 0, yb0, fb);
-            tma_load_2d(ssb + 512, &tmSFB, 0, yb1, fb);
+            tma_load_2d(ssb + C::KS * 512, &tmSFB, 0, yb1, fb);
           }
           ++it;
         }
@@ -387,7 +423,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           break;
         }
         tc_fence_after();
-        for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
+        for (int32_t kb0 = 0; kb0 < tl.kblocks; kb0 += C::KS) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
           if (!mbar_wait(full_bar(s), ph, abort_flag, lim)) {
             record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
@@ -395,31 +431,38 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             break;
           }
           tc_fence_after();
-          const uint32_t sfa_t = tmem + C::SF_COL + SF_STRIDE * s, sfb_t = sfa_t + 4;
-          const uint64_t dsa = desc_sf_32x16(smem_addr(smem + C::OFF_SFA + s * SFA_TILE));
-          const uint64_t dsb0 = desc_sf_32x16(smem_addr(smem + C::OFF_SFB + s * SFB_TILE));
-          const uint64_t dsb1 = desc_sf_32x16(smem_addr(smem + C::OFF_SFB + s * SFB_TILE + 512));
-          const uint64_t da = desc_kmajor_sw128(smem_addr(smem + C::OFF_A + s * C::A_TILE));
-          const uint64_t db = desc_kmajor_sw128(smem_addr(smem + C::OFF_B + s * C::B_TILE));
-          const int32_t nk = (kb == tl.kblocks - 1) ? tl.ksteps_last : BK / 32;
-          if constexpr (CG == 2) {
-            tc_cp_32x128b_x4_pair(sfa_t, dsa);
-            tc_cp_32x128b_x4_pair(sfb_t, dsb0);
-            tc_cp_32x128b_x4_pair(sfb_t + 4, dsb1);
-          } else {
-            tc_cp_32x128b_x4(sfa_t, dsa);
-            tc_cp_32x128b_x4(sfb_t, dsb0);
-            tc_cp_32x128b_x4(sfb_t + 4, dsb1);
-          }
-          for (int32_t k = 0; k < nk; ++k) {
-            const uint32_t idesc = idesc0 | (uint32_t(k) << 4) | (uint32_t(k) << 29);
-            // +2 per step: the start-address field counts 16-byte units, one step is 32 bytes of K
-            if constexpr (CG == 2)
-              tc_mma_mxf8_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
-                               sfb_t | (uint32_t(k) << 30), (kb | k) != 0);
-            else
-              tc_mma_mxf8(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
-                          sfb_t | (uint32_t(k) << 30), (kb | k) != 0);
+          const int32_t nh = min(C::KS, tl.kblocks - kb0);
+          const uint32_t sfa_s = smem_addr(smem + C::OFF_SFA + s * C::KS * SFA_TILE);
+          const uint32_t sfb_s = smem_addr(smem + C::OFF_SFB + s * C::KS * SFB_TILE);
+          for (int32_t h = 0; h < nh; ++h) {
+            const int32_t kb = kb0 + h;
+            const uint32_t q = s * C::KS + h;
+            const uint32_t sfa_t = tmem + C::SF_COL + SF_STRIDE * q, sfb_t = sfa_t + 4;
+            const uint64_t dsa = desc_sf_32x16(sfa_s + 512 * h);
+            const uint64_t dsb0 = desc_sf_32x16(sfb_s + 512 * h);
+            const uint64_t dsb1 = desc_sf_32x16(sfb_s + 512 * (C::KS + h));
+            const uint64_t da = desc_kmajor_sw128(smem_addr(smem + C::OFF_A + q * C::A_TILE));
+            const uint64_t db = desc_kmajor_sw128(smem_addr(smem + C::OFF_B + q * C::B_TILE));
+            const int32_t nk = (kb == tl.kblocks - 1) ? tl.ksteps_last : BK / 32;
+            if constexpr (CG == 2) {
+              tc_cp_32x128b_x4_pair(sfa_t, dsa);
+              tc_cp_32x128b_x4_pair(sfb_t, dsb0);
+              tc_cp_32x128b_x4_pair(sfb_t + 4, dsb1);
+            } else {
+              tc_cp_32x128b_x4(sfa_t, dsa);
+              tc_cp_32x128b_x4(sfb_t, dsb0);
+              tc_cp_32x128b_x4(sfb_t + 4, dsb1);
+            }
+            for (int32_t k = 0; k < nk; ++k) {
+              const uint32_t idesc = idesc0 | (uint32_t(k) << 4) | (uint32_t(k) << 29);
+              // +2 per step: the start-address field counts 16-byte units, one step is 32 bytes of K
+              if constexpr (CG == 2)
+                tc_mma_mxf8_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
+                                 sfb_t | (uint32_t(k) << 30), (kb | k) != 0);
+              else
+                tc_mma_mxf8(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
+                            sfb_t | (uint32_t(k) << 30), (kb | k) != 0);
+            }
           }
           if constexpr (CG == 2) tc_commit_pair(empty_bar(s), 0x3);
           else tc_commit(empty_bar(s));
@@ -493,6 +536,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           tmem_ld_32x32b_x32(tbase + 64 * chunk_of(ci + 1) + 32, n1);
         }
         const int c = chunk_of(ci);
+        uint32_t rs = 0, cs0 = 0, cs1 = 0;   // quantising epilogue: scale bytes (0 = pad)
         if (vr > 0 && 64 * c < tl.cols) {
           uint32_t pk[32];
 #pragma unroll
@@ -507,26 +551,97 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll
           for (int q = 0; q < 8; ++q)   // 128-byte swizzle: chunk q of row `lane` at q ^ (lane % 8)
             st4[lane * 8 + (q ^ (lane & 7))] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-          if (vr == 32) {
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_2d(&tmOut, static_cast<int32_t>(tl.out_col + 64 * c),
-                           static_cast<int32_t>(tl.out_row + row_base), smem_addr(stg));
-              bulk_commit_group();
-            }
-          } else {
-            __syncwarp();
+          if (!QE || p.out != nullptr) {
+            if (vr == 32) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmOut, static_cast<int32_t>(tl.out_col + 64 * c),
+                             static_cast<int32_t>(tl.out_row + row_base), smem_addr(stg));
+                bulk_commit_group();
+              }
+            } else {
+              __syncwarp();
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int rr = 4 * i + srow, col = 64 * c + 8 * schunk;
-              if (rr < vr && col < tl.cols)
-                *reinterpret_cast<uint4*>(out_tile + int64_t(row_base + rr) * p.out_ld + col) =
-                    st4[rr * 8 + (schunk ^ (rr & 7))];
+              for (int i = 0; i < 8; ++i) {
+                const int rr = 4 * i + srow, col = 64 * c + 8 * schunk;
+                if (rr < vr && col < tl.cols)
+                  *reinterpret_cast<uint4*>(out_tile + int64_t(row_base + rr) * p.out_ld + col) =
+                      st4[rr * 8 + (schunk ^ (rr & 7))];
+              }
+            }
+          }
+          if constexpr (QE) {
+            __syncwarp();
+            if (p.qr != nullptr && lane < vr) {
+              // Rowwise: this lane's row holds the chunk's two 32-blocks.
+              uint8_t* qrow = p.qr + (tl.out_row + row_base + lane) * p.out_ld + tl.out_col + 64 * c;
+#pragma unroll
+              for (int b = 0; b < 2; ++b) {
+                if (64 * c + 32 * b < tl.cols) {
+                  const uint32_t* v = pk + 16 * b;
+                  uint32_t m = 0;
+#pragma unroll
+                  for (int i = 0; i < 16; ++i) m = __vmaxu2(m, v[i] & 0x7FFF7FFFu);
+                  const uint32_t sb = scale_byte(max(m & 0xFFFFu, m >> 16));
+                  uint2 w[4];
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) w[i] = encode8(make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]), sb);
+                  *reinterpret_cast<uint4*>(qrow + 32 * b) = make_uint4(w[0].x, w[0].y, w[1].x, w[1].y);
+                  *reinterpret_cast<uint4*>(qrow + 32 * b + 16) = make_uint4(w[2].x, w[2].y, w[3].x, w[3].y);
+                  rs |= sb << (8 * b);
+                }
+              }
+            }
+            if (p.qc != nullptr && 64 * c + 2 * lane < tl.cols) {
+              // Colwise: this lane takes columns 64c + 2*lane and +1 over the
+              // warp's 32 rows, one group-relative 32-block (rows past the
+              // group are pad: excluded from amax, code 0).
+              const uint32_t* s32 = reinterpret_cast<const uint32_t*>(stg);
+              uint32_t w[32], m = 0;
+#pragma unroll
+              for (int r = 0; r < 32; ++r) {
+                w[r] = r < vr ? s32[r * 32 + (((lane >> 2) ^ (r & 7)) << 2) + (lane & 3)] : 0u;
+                m = __vmaxu2(m, w[r] & 0x7FFF7FFFu);
+              }
+              cs0 = scale_byte(m & 0xFFFFu);
+              cs1 = scale_byte(m >> 16);
+              const float f0 = inv_scale(cs0 == 0xFFu ? 0u : cs0), f1 = inv_scale(cs1 == 0xFFu ? 0u : cs1);
+              uint32_t o0[8], o1[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const uint32_t a0 = cvt_e4m3x2(__fmul_rn(bf_lo(w[4 * j]), f0), __fmul_rn(bf_lo(w[4 * j + 1]), f0));
+                const uint32_t a1 = cvt_e4m3x2(__fmul_rn(bf_lo(w[4 * j + 2]), f0), __fmul_rn(bf_lo(w[4 * j + 3]), f0));
+                const uint32_t b0 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * j]), f1), __fmul_rn(bf_hi(w[4 * j + 1]), f1));
+                const uint32_t b1 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * j + 2]), f1), __fmul_rn(bf_hi(w[4 * j + 3]), f1));
+                o0[j] = cs0 == 0xFFu ? nan_codes4(j, vr) : (a0 | (a1 << 16));
+                o1[j] = cs1 == 0xFFu ? nan_codes4(j, vr) : (b0 | (b1 << 16));
+              }
+              uint8_t* qcol = p.qc + (tl.out_col + 64 * c + 2 * lane) * p.qc_ld + tl.q_p + row_base;
+              reinterpret_cast<uint4*>(qcol)[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+              reinterpret_cast<uint4*>(qcol)[1] = make_uint4(o0[4], o0[5], o0[6], o0[7]);
+              reinterpret_cast<uint4*>(qcol + p.qc_ld)[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+              reinterpret_cast<uint4*>(qcol + p.qc_ld)[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
             }
           }
           __syncwarp();
           ++ec;
+        }
+        if constexpr (QE) {
+          // Scale bytes, zeros included, for every atom this tile covers:
+          // pad rows and blocks inside a written atom are 0x00.
+          if (tl.rows > 0) {
+            const int64_t col = tl.out_col + 64 * c;
+            if (p.sr != nullptr && col / 128 < (p.out_ld + 127) / 128)
+              *reinterpret_cast<uint16_t*>(p.sr + 512 * (int64_t(tl.q_rb) * ((p.out_ld + 127) / 128) + col / 128) +
+                                           lane * 16 + quarter * 4 + 2 * (c & 1)) = static_cast<uint16_t>(rs);
+            const int64_t n = col + 2 * lane;   // colwise: the output columns are the scale rows
+            if (p.sc != nullptr && n / 128 < (p.out_ld + 127) / 128) {
+              uint8_t* a = p.sc + 512 * ((n / 128) * p.sc_pitch + tl.q_rb) + ((n % 128) / 32) * 4 + quarter;
+              a[(n % 32) * 16] = static_cast<uint8_t>(cs0);
+              a[((n + 1) % 32) * 16] = static_cast<uint8_t>(cs1);
+            }
+          }
         }
         if (ci < 3) {
           tmem_wait_regs(n0);
@@ -584,27 +699,27 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, int e
 }
 
 struct DeviceSetup {
-  bool done[2] = {false, false};
+  bool done[2][2][2] = {};    // [CG - 1][KS - 1][QE]
   int num_sms = 0;
-  int max_pairs = 0;
+  int max_pairs[2][2] = {};   // [KS - 1][QE]
 };
 DeviceSetup g_setup[64];
 
-template <int CG>
+template <int CG, int KS, bool QE>
 cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_t stream) {
-  using C = Cfg<CG>;
+  using C = Cfg<CG, KS>;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   DeviceSetup& ds = g_setup[dev];
-  auto kernel = grouped_gemm_kernel<CG>;
+  auto kernel = grouped_gemm_kernel<CG, KS, QE>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  if (!ds.done[CG - 1]) {
+  if (!ds.done[CG - 1][KS - 1][QE]) {
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     err = cudaDeviceGetAttribute(&ds.num_sms, cudaDevAttrMultiProcessorCount, dev);
@@ -619,16 +734,16 @@ cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_
       int clusters = 0;
       err = cudaOccupancyMaxActiveClusters(&clusters, kernel, &q);
       if (err != cudaSuccess) return err;
-      ds.max_pairs = clusters > 0 ? clusters : 1;
+      ds.max_pairs[KS - 1][QE] = clusters > 0 ? clusters : 1;
     }
-    ds.done[CG - 1] = true;
+    ds.done[CG - 1][KS - 1][QE] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
   if (CG == 2) {
-    cfg.gridDim = dim3(2 * ds.max_pairs);
+    cfg.gridDim = dim3(2 * ds.max_pairs[KS - 1][QE]);
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   } else {
@@ -642,12 +757,22 @@ cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** detail) {
   // Tile configuration: 1-CTA 128x256 tiles by default -- on B200 they beat
   // CTA pairs on every pass of the DeepSeek-V3-like layers (pairs also waste
-  // up to 128 rows per group in fwd/dgrad).  MXF8_GEMM_CTA_PAIR=1 selects
-  // pairs, MXF8_GEMM_CTA_PAIR=0 the default.
-  const char* env = std::getenv("MXF8_GEMM_CTA_PAIR");
+  // up to 128 rows per group in fwd/dgrad).  Stage depth: 256-deep stages for
+  // fwd/dgrad, except for a short odd K loop whose last stage would run half
+  // empty; 128-deep stages for wgrad, whose K loops (the groups' token counts)
+  // are short and whose tiles are epilogue-heavy.  MXF8_GEMM_CTA_PAIR=1/0 and
+  // MXF8_GEMM_KS=1/2 override the choices.
   int cg = 1;
-  if (env && std::strcmp(env, "0") == 0) cg = 1;
+  const char* env = std::getenv("MXF8_GEMM_CTA_PAIR");
   if (env && std::strcmp(env, "1") == 0) cg = 2;
+  int ks = 1;
+  if (a.mode != kWgrad) {
+    const int64_t kblocks = ((a.mode == kFwd ? a.K : a.N) + BK - 1) / BK;
+    ks = (kblocks % 2 == 0 || kblocks >= 24) ? 2 : 1;
+  }
+  env = std::getenv("MXF8_GEMM_KS");
+  if (env && std::strcmp(env, "1") == 0) ks = 1;
+  if (env && std::strcmp(env, "2") == 0) ks = 2;
   const int64_t out_rows = a.mode == kWgrad ? int64_t(a.E) * a.N : a.M;
   const int64_t out_cols = a.mode == kFwd ? a.N : a.K;
   CUtensorMap maps[5];
@@ -656,12 +781,17 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
                CU_TENSOR_MAP_SWIZZLE_128B) &&
       make_map(&maps[1], a.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b_rows, a.b_cols, a.ldb, BK, BN / cg,
                CU_TENSOR_MAP_SWIZZLE_128B) &&
-      make_map(&maps[2], a.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfa_atoms * 4, 128, 128, 128, 4,
+      make_map(&maps[2], a.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfa_atoms * 4, 128, 128, 128, 4 * ks,
                CU_TENSOR_MAP_SWIZZLE_NONE) &&
-      make_map(&maps[3], a.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfb_atoms * 4, 128, 128, 128, 4,
+      make_map(&maps[3], a.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfb_atoms * 4, 128, 128, 128, 4 * ks,
                CU_TENSOR_MAP_SWIZZLE_NONE) &&
-      make_map(&maps[4], a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out_rows, out_cols, out_cols, 64, 32,
-               CU_TENSOR_MAP_SWIZZLE_128B);
+      (a.out != nullptr
+           ? make_map(&maps[4], a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out_rows, out_cols, out_cols, 64, 32,
+                      CU_TENSOR_MAP_SWIZZLE_128B)
+           // no bf16 output (quantising epilogue only): a placeholder map over
+           // the status word that the kernel never uses
+           : make_map(&maps[4], a.status, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 1, 64, 64, 64, 32,
+                      CU_TENSOR_MAP_SWIZZLE_128B));
   if (!ok) {
     if (detail) *detail = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
@@ -676,7 +806,15 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   p.out_ld = out_cols;
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
-  return cg == 2 ? launch_cg<2>(p, maps, stream) : launch_cg<1>(p, maps, stream);
+  p.qr = a.qr; p.sr = a.sr; p.qc = a.qc; p.sc = a.sc;
+  p.qc_ld = a.qc_ld; p.sc_pitch = a.sc_pitch;
+  const bool qe = a.qr != nullptr || a.qc != nullptr;
+  if (qe) {
+    if (cg == 2) return ks == 2 ? launch_cg<2, 2, true>(p, maps, stream) : launch_cg<2, 1, true>(p, maps, stream);
+    return ks == 2 ? launch_cg<1, 2, true>(p, maps, stream) : launch_cg<1, 1, true>(p, maps, stream);
+  }
+  if (cg == 2) return ks == 2 ? launch_cg<2, 2, false>(p, maps, stream) : launch_cg<2, 1, false>(p, maps, stream);
+  return ks == 2 ? launch_cg<1, 2, false>(p, maps, stream) : launch_cg<1, 1, false>(p, maps, stream);
 }
 
 }  // namespace mxf8

@@ -31,9 +31,15 @@ struct GemmArgs {
   const uint8_t* b; int64_t ldb, b_rows, b_cols;
   const uint8_t* sfa; int64_t sfa_pitch, sfa_atoms;
   const uint8_t* sfb; int64_t sfb_pitch, sfb_atoms;
-  uint16_t* out;
+  uint16_t* out;                 // bf16 output; may be null when a quantised copy is requested
   int32_t* status;
   uint64_t timeout_ns;
+  // fwd/dgrad only: MXFP8 copies of the output written by the epilogue, in
+  // the quantisers' rowwise (qr, sr) and colwise (qc, sc) layouts over the
+  // GEMM's groups; null = not written.
+  uint8_t* qr = nullptr; uint8_t* sr = nullptr;
+  uint8_t* qc = nullptr; uint8_t* sc = nullptr;
+  int64_t qc_ld = 0, sc_pitch = 0;
 };
 
 // Returns cudaSuccess or the CUDA error; *detail gets a short reason for

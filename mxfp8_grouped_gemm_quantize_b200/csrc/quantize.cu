@@ -15,6 +15,7 @@
 // and codes come from the hardware E4M3x2 conversion.
 #include <cuda_runtime.h>
 
+#include "codec.cuh"
 #include "groups.cuh"
 #include "launch.h"
 #include "ptx.cuh"
@@ -23,41 +24,6 @@ namespace mxf8 {
 namespace {
 
 constexpr int kThreads = 256;
-
-// Scale byte from the largest |x| given as bf16 magnitude bits.  For a normal
-// amax with biased exponent E, floor(log2 amax) = E - 127, so s = E - 135 and
-// the byte is E - 8; E <= 8 (including zero and bf16 subnormals, E = 0)
-// clamps to s = -127, byte 0.  E = 255 (Inf/NaN) gives the NaN scale 0xFF.
-__device__ __forceinline__ uint32_t scale_byte(uint32_t amax_bits) {
-  const uint32_t e = (amax_bits >> 7) & 0xFFu;
-  if (e == 0xFFu) return 0xFFu;
-  return e > 8u ? e - 8u : 0u;
-}
-
-// 2^-s as an fp32 for a finite scale byte b = s + 127 (exponent field
-// 254 - b lies in [8, 254], so the value is a normal number and x * 2^-s is
-// exact whenever it is representable).
-__device__ __forceinline__ float inv_scale(uint32_t b) { return __uint_as_float((254u - b) << 23); }
-
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-__device__ __forceinline__ uint32_t amax_bits8(const uint4& v) {
-  const uint32_t k = 0x7FFF7FFFu;
-  const uint32_t m = __vmaxu2(__vmaxu2(v.x & k, v.y & k), __vmaxu2(v.z & k, v.w & k));
-  return max(m & 0xFFFFu, m >> 16);
-}
-
-// Codes of two bf16 (packed in w) scaled by f: two bytes, low element first.
-__device__ __forceinline__ uint32_t enc2(uint32_t w, float f) {
-  return cvt_e4m3x2(__fmul_rn(bf_lo(w), f), __fmul_rn(bf_hi(w), f));
-}
-
-__device__ __forceinline__ uint2 encode8(const uint4& v, uint32_t sb) {
-  if (sb == 0xFFu) return make_uint2(0x7F7F7F7Fu, 0x7F7F7F7Fu);
-  const float f = inv_scale(sb);
-  return make_uint2(enc2(v.x, f) | (enc2(v.y, f) << 16), enc2(v.z, f) | (enc2(v.w, f) << 16));
-}
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 r;
@@ -171,6 +137,7 @@ __global__ void __launch_bounds__(kThreads) quantize_colwise_kernel(
     mx = __vmaxu2(mx, w[r] & 0x7FFF7FFFu);
   }
   const uint32_t sb_lo = scale_byte(mx & 0xFFFFu), sb_hi = scale_byte(mx >> 16);
+  const int vrows = min(32, max(0, br.nrows - 32 * blk));   // real rows of this 32-block
   uint32_t olo[8], ohi[8];
   {
     const float flo = inv_scale(sb_lo == 0xFFu ? 0u : sb_lo);
@@ -181,8 +148,8 @@ __global__ void __launch_bounds__(kThreads) quantize_colwise_kernel(
       const uint32_t a1 = cvt_e4m3x2(__fmul_rn(bf_lo(w[4 * j + 2]), flo), __fmul_rn(bf_lo(w[4 * j + 3]), flo));
       const uint32_t b0 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * j]), fhi), __fmul_rn(bf_hi(w[4 * j + 1]), fhi));
       const uint32_t b1 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * j + 2]), fhi), __fmul_rn(bf_hi(w[4 * j + 3]), fhi));
-      olo[j] = sb_lo == 0xFFu ? 0x7F7F7F7Fu : (a0 | (a1 << 16));
-      ohi[j] = sb_hi == 0xFFu ? 0x7F7F7F7Fu : (b0 | (b1 << 16));
+      olo[j] = sb_lo == 0xFFu ? nan_codes4(j, vrows) : (a0 | (a1 << 16));
+      ohi[j] = sb_hi == 0xFFu ? nan_codes4(j, vrows) : (b0 | (b1 << 16));
     }
   }
   __syncthreads();   // every thread has read its columns; the tile becomes the code stage
@@ -267,6 +234,7 @@ __global__ void __launch_bounds__(kThreads) quantize_dual_kernel(
     mx = __vmaxu2(mx, w[r] & 0x7FFF7FFFu);
   }
   const uint32_t sb_lo = scale_byte(mx & 0xFFFFu), sb_hi = scale_byte(mx >> 16);
+  const int vrows = min(32, max(0, br.nrows - 32 * blk));   // real rows of this 32-block
   uint32_t olo[8], ohi[8];
   {
     const float flo = inv_scale(sb_lo == 0xFFu ? 0u : sb_lo);
@@ -277,8 +245,8 @@ __global__ void __launch_bounds__(kThreads) quantize_dual_kernel(
       const uint32_t a1 = cvt_e4m3x2(__fmul_rn(bf_lo(w[4 * j + 2]), flo), __fmul_rn(bf_lo(w[4 * j + 3]), flo));
       const uint32_t b0 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * j]), fhi), __fmul_rn(bf_hi(w[4 * j + 1]), fhi));
       const uint32_t b1 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * j + 2]), fhi), __fmul_rn(bf_hi(w[4 * j + 3]), fhi));
-      olo[j] = sb_lo == 0xFFu ? 0x7F7F7F7Fu : (a0 | (a1 << 16));
-      ohi[j] = sb_hi == 0xFFu ? 0x7F7F7F7Fu : (b0 | (b1 << 16));
+      olo[j] = sb_lo == 0xFFu ? nan_codes4(j, vrows) : (a0 | (a1 << 16));
+      ohi[j] = sb_hi == 0xFFu ? nan_codes4(j, vrows) : (b0 | (b1 << 16));
     }
   }
   __syncthreads();

@@ -19,16 +19,18 @@ pytestmark = pytest.mark.gpu
 POISON = 0x7FC0  # bf16 NaN: any output element the kernel fails to write stays NaN
 
 
-@pytest.fixture(params=["default", "1cta", "pair"])
+@pytest.fixture(params=["default", "1cta-ks1", "1cta-ks2", "pair-ks1", "pair-ks2"])
 def tile_config(request, monkeypatch):
-    """Runs a test under the per-pass default tile configuration, forced
-    1-CTA 128x256 tiles, and forced CTA-pair 256x256 tiles."""
-    if request.param == "1cta":
-        monkeypatch.setenv("MXF8_GEMM_CTA_PAIR", "0")
-    elif request.param == "pair":
-        monkeypatch.setenv("MXF8_GEMM_CTA_PAIR", "1")
-    else:
+    """Runs a test under the per-pass default tile configuration and under
+    each forced one: 1-CTA 128x256 or CTA-pair 256x256 tiles, with 128-deep
+    (ks1) or 256-deep (ks2) pipeline stages."""
+    if request.param == "default":
         monkeypatch.delenv("MXF8_GEMM_CTA_PAIR", raising=False)
+        monkeypatch.delenv("MXF8_GEMM_KS", raising=False)
+    else:
+        tiles, ks = request.param.split("-")
+        monkeypatch.setenv("MXF8_GEMM_CTA_PAIR", "1" if tiles == "pair" else "0")
+        monkeypatch.setenv("MXF8_GEMM_KS", ks[-1])
     return request.param
 
 
@@ -184,7 +186,8 @@ def test_distinct_block_scales_pin_the_scale_layout(mx, tile_config):
 
 
 @pytest.mark.parametrize("counts,N,K", [([1], 128, 32), ([0, 0, 5], 128, 64), ([300], 128, 160),
-                                        ([3, 0, 0, 0], 256, 1024), ([129, 127], 512, 96)])
+                                        ([3, 0, 0, 0], 256, 1024), ([129, 127], 512, 96),
+                                        ([40, 0, 260], 384, 544)])
 def test_edge_shapes(mx, tile_config, counts, N, K):
     run_all_and_compare(make_case(mx, counts, N, K, seed=sum(counts)))
 

@@ -284,3 +284,18 @@ def test_dual_matches_separate_at_workload_size(mx):
     for rb in range(X.shape[1] // 128):
         a = rb * pitch
         assert torch.equal(sfT[a * 512:(a + RB) * 512], sfT2[a * 512:(a + RB) * 512])
+
+
+@pytest.mark.parametrize("kind", ["inf", "nan"])
+def test_nonfinite_in_a_short_last_colwise_block(mx, kind):
+    """A non-finite value in a group's short last 32-row block: the block
+    gets the NaN scale and NaN codes on its real rows, while the pad columns
+    up to the group's 32-padded end stay 0x00 (colwise and dual)."""
+    counts = [70, 0, 150, 33]
+    offs = wl.offsets_from_counts(counts)
+    x = wl.normal_bf16((int(offs[-1]), 96), 1.0, 4)
+    bad = float("inf") if kind == "inf" else float("nan")
+    for r, c in ((200, 5), (3, 40), (252, 95)):   # group 2 block 4 (22 rows), a full block, group 3 block 1 (1 row)
+        x[r, c] = bad
+    check_colwise(mx, x, offs)
+    check_dual(mx, x, offs)
