@@ -286,6 +286,7 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(w, budget_s=12.0)
     out["e2e"] = e2e(args, mx, w, layers, dev, world)
+    out["quantising_epilogue"] = quantising_epilogue(mx, layers[0])
     return out
 
 
@@ -332,6 +333,54 @@ def e2e(args, mx, w, layers, dev, world):
     flops = 3 * sum(L.flops_per_pass() for L in layers)
     return {"value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": UNIT, "ms_per_step": round(ms, 3),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": K}
+
+
+def quantising_epilogue(mx, L: Linear, iters=20):
+    """The quantising epilogue (the GEMM writes its output as MXFP8 too)
+    against the GEMM followed by the dual quantiser on its bf16 output, for
+    fwd and dgrad of one linear.  Not part of the step above; reported as
+    its own measurement."""
+    dev = L.y.device
+    M, E = L.M, L.E
+    ld = mx.mxfp8_colwise_ld(M, E)
+    res = {"linear": L.name}
+    for mode, C in (("fwd", L.N), ("dgrad", L.K)):
+        out = L.y if mode == "fwd" else L.dx
+        row = (torch.empty((M, C), dtype=torch.uint8, device=dev),
+               torch.empty(mx.mxfp8_rowwise_scale_bytes(M, C, E), dtype=torch.uint8, device=dev))
+        col = (torch.empty((C, ld), dtype=torch.uint8, device=dev),
+               torch.empty(mx.mxfp8_colwise_scale_bytes(M, C, E), dtype=torch.uint8, device=dev))
+        if mode == "fwd":
+            plain = lambda: mx.mxfp8_grouped_gemm_fwd(L.xq, L.xs, L.wq, L.ws, L.offs, L.N, out=out, work=L.work)  # noqa: E731
+            fused = lambda o: mx.mxfp8_grouped_gemm_fwd_quant(L.xq, L.xs, L.wq, L.ws, L.offs, L.N, out=o,  # noqa: E731
+                                                              rowwise=row, colwise=col, work=L.work)
+        else:
+            plain = lambda: mx.mxfp8_grouped_gemm_dgrad(L.dyq, L.dys, L.wqT, L.wsT, L.offs, L.K, out=out,  # noqa: E731
+                                                        work=L.work)
+            fused = lambda o: mx.mxfp8_grouped_gemm_dgrad_quant(L.dyq, L.dys, L.wqT, L.wsT, L.offs, L.K, out=o,  # noqa: E731
+                                                                rowwise=row, colwise=col, work=L.work)
+        quant = lambda: mx.mxfp8_quantize_dual(out, L.offs, q=row[0], scales=row[1], qT=col[0], scalesT=col[1])  # noqa: E731
+        variants = {"gemm_then_dual_quantiser": lambda: (plain(), quant()),
+                    "quantising_epilogue": lambda: fused(out),
+                    "quantising_epilogue_no_bf16": lambda: fused(None)}
+        r = {}
+        for name, fn in variants.items():
+            for _ in range(3):
+                fn()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record()
+            for _ in range(iters):
+                fn()
+            b.record()
+            torch.cuda.synchronize()
+            r[name + "_ms"] = round(a.elapsed_time(b) / iters, 4)
+        st = mx.mxfp8_get_status(L.work)
+        if st != 0:
+            raise SystemExit(f"bench: device status {st} in the quantising-epilogue measurement")
+        r["tflops"] = round(L.flops_per_pass() / (r["quantising_epilogue_ms"] * 1e-3) / 1e12, 1)
+        res[mode] = r
+    return res
 
 
 # ---------------------------------------------------------------- CPU oracle baseline / reference arm
