@@ -8,8 +8,8 @@ section "Что такое TorchTitan"; aifind.ru, "DeepSeek-V3 ...", section
 "Параметры"), Llama 4 Scout (neurabooks.ru, "New data format speeds up
 Llama 4 Scout training"), and dropless routing where each expert gets its
 real, imbalanced token count (iitak.ru, "NVIDIA ... JAX", dropless paragraph).
-The sizes and distributions are those of the workload table of the task:
-no dataset is involved, so these synthetic draws stand in for real routing.
+The sizes and distributions are the pages' model shapes with synthetic
+routing: no dataset is involved, so these synthetic draws stand in for real routing.
 """
 from __future__ import annotations
 
@@ -110,6 +110,54 @@ def llama4_scout(seed: int = 3) -> Workload:
     counts = _top_k_counts(rng.standard_normal((T, E)), 1)
     return Workload("llama4-scout", counts, [Layer("gate_up", 2 * 8192, 5120), Layer("down", 5120, 8192)],
                     w_std=0.02, seed=seed)
+
+
+@dataclass
+class Routing:
+    """Top-k routing of T tokens: expert ids idx[T, k] (int32, distinct per
+    token) and combine weights w[T, k] (float32, softmax over the chosen
+    logits), plus the token activations' width K."""
+    name: str
+    E: int
+    idx: np.ndarray
+    w: np.ndarray
+    K: int
+
+    @property
+    def T(self) -> int:
+        return int(self.idx.shape[0])
+
+    @property
+    def k(self) -> int:
+        return int(self.idx.shape[1])
+
+
+def _top_k_routing(name, logits: np.ndarray, k: int, K: int) -> Routing:
+    T, E = logits.shape
+    idx = np.argsort(-logits, axis=1, kind="stable")[:, :k]
+    sel = np.take_along_axis(logits, idx, axis=1)
+    w = np.exp(sel - sel.max(axis=1, keepdims=True))
+    w = (w / w.sum(axis=1, keepdims=True)).astype(np.float32)
+    return Routing(name, E, idx.astype(np.int32), w, K)
+
+
+def routing(name: str, seed: int | None = None) -> Routing:
+    """The routing behind a workload's counts: the same draws as the workload
+    generator, kept per token (ds-v3-16b: top-6 of 64 for 8192 tokens, K =
+    2048; llama4-scout: top-1 of 16 for 16384 tokens, K = 5120; tiny: top-2
+    of 5 for 40 tokens, K = 256)."""
+    if name == "ds-v3-16b":
+        rng = np.random.default_rng(1 if seed is None else seed)
+        T, E = 8192, 64
+        logits = rng.standard_normal((T, E)) + rng.normal(0.0, 0.5, size=E)[None, :]
+        return _top_k_routing(name, logits, 6, 2048)
+    if name == "llama4-scout":
+        rng = np.random.default_rng(3 if seed is None else seed)
+        return _top_k_routing(name, rng.standard_normal((16384, 16)), 1, 5120)
+    if name == "tiny":
+        rng = np.random.default_rng(0 if seed is None else seed)
+        return _top_k_routing(name, rng.standard_normal((40, 5)), 2, 256)
+    raise KeyError(name)
 
 
 def quantiser_sweep() -> list[tuple[int, int]]:

@@ -69,6 +69,11 @@ def lib():
             getattr(L, name).argtypes = [_vp, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _i64, _vp]
         L.orc_baseline_quantize_rows.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp]
         L.orc_threads.restype = ctypes.c_int
+        L.orc_moe_plan.argtypes = [_vp, _i64, _i32, _i32, _vp, _vp, _vp]
+        L.orc_moe_combine.argtypes = [_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp]
+        L.orc_bf16_from_double.restype = ctypes.c_uint16
+        L.orc_bf16_from_double.argtypes = [ctypes.c_double]
+        L.orc_bf16_from_double_array.argtypes = [_vp, _i64, _vp]
         _LIB = L
     return _LIB
 
@@ -340,3 +345,37 @@ def baseline_quantize_rows(x_u16, row_lo, row_hi):
 
 
 __all__ = [n for n in dir() if not n.startswith("_") and n not in ("annotations", "ctypes", "np", "os")]
+
+
+# ---------------------------------------------------------------- MoE dispatch plan / combine
+def moe_plan(idx, E: int):
+    """idx: int [T, k] expert ids -> (offs int32 [E+1], perm int32 [T*k], inv int32 [T, k]).
+    Pairs grouped by expert in ascending (token, slot) order."""
+    idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int32))
+    T, k = idx.shape
+    offs = np.zeros(E + 1, dtype=np.int32)
+    perm = np.zeros(T * k, dtype=np.int32)
+    inv = np.zeros((T, k), dtype=np.int32)
+    _check(lib().orc_moe_plan(_p(idx), T, k, E, _p(offs), _p(perm), _p(inv)), "moe_plan")
+    return offs, perm, inv
+
+
+def bf16_from_double(v) -> np.ndarray:
+    """Nearest-even bf16 bits (uint16) of float64 values."""
+    a = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
+    out = np.zeros(a.shape, dtype=np.uint16)
+    lib().orc_bf16_from_double_array(_p(a), a.size, _p(out))
+    return out
+
+
+def moe_combine(yp, inv, w) -> np.ndarray:
+    """yp: bf16 [rows, C]; inv int [T, k]; w float32 [T, k] -> bf16 bits [T, C]:
+    y[t] = sum_j w[t, j] * yp[inv[t, j]], in fp64, rounded once to bf16."""
+    ypu = _u16(yp)
+    rows, C = ypu.shape
+    inv = np.ascontiguousarray(np.asarray(inv, dtype=np.int32))
+    w = np.ascontiguousarray(np.asarray(w, dtype=np.float32))
+    T, k = inv.shape
+    y = np.zeros((T, C), dtype=np.uint16)
+    _check(lib().orc_moe_combine(_p(ypu), rows, C, _p(inv), _p(w), T, k, _p(y)), "moe_combine")
+    return y

@@ -11,8 +11,8 @@
  *   - MXFP8 is a microscaling format in which a block of 32 consecutive
  *     elements shares one exponent (opensourcebeat.com, "Enabling up to 41%
  *     faster pre-training: MXFP8 and DeepEP ...", FAQ "What is MXFP8?").
- *     The block rules are those of the OCP Microscaling (MX) v1.0 format that
- *     the benchmark spec names: E8M0 scale X = 2^(floor(log2(amax)) - emax),
+ *     The block rules are those of the OCP Microscaling (MX) v1.0
+ *     specification: E8M0 scale X = 2^(floor(log2(amax)) - emax),
  *     emax = 8 for E4M3, clamped to the E8M0 range; element = E4M3(v / X)
  *     with round-to-nearest-even and saturation to +-448.
  *   - The grouped GEMM computes every expert on its real token count, with
@@ -613,4 +613,100 @@ int orc_baseline_quantize_rows(const uint16_t* x, int64_t C, int64_t row_lo, int
             orc_quantize_block(x + r * C + 32 * j, 32, 1, q + r * C + 32 * j, 1, s_logical + r * (C / 32) + j);
     }
     return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* MoE token dispatch plan and combine (permute / unpermute)            */
+/* ------------------------------------------------------------------ */
+/* The grouped GEMM consumes each expert's tokens as one contiguous run of
+ * rows, every token with its real count (iitak.ru, "NVIDIA ... JAX",
+ * paragraph on the Transformer Engine grouped GEMM; the all-to-all that
+ * sends tokens to experts and the one that brings results back are on
+ * opensourcebeat.com, section "Двухсторонняя атака: MXFP8 и DeepEP").
+ * Routing gives token t its k experts idx[t*k + j], j = 0..k-1.  The plan
+ * lists the (token, slot) pairs grouped by expert, in ascending (token,
+ * slot) order inside an expert:
+ *   offs[e]      exclusive prefix of the per-expert pair counts, offs[E] = T*k;
+ *   perm[r]      token of permuted row r;
+ *   inv[t*k+j]   permuted row of pair (t, j).
+ * Returns -1 if an expert id is out of range. */
+int orc_moe_plan(const int32_t* idx, int64_t T, int32_t k, int32_t E, int32_t* offs, int32_t* perm,
+                 int32_t* inv)
+{
+    int64_t* fill = (int64_t*)calloc((size_t)E + 1, sizeof(int64_t));
+    int64_t i, t;
+    int32_t e, j;
+    for (i = 0; i < T * k; ++i) {
+        if (idx[i] < 0 || idx[i] >= E) { free(fill); return -1; }
+        fill[idx[i]] += 1;
+    }
+    offs[0] = 0;
+    for (e = 0; e < E; ++e) offs[e + 1] = offs[e] + (int32_t)fill[e];
+    for (e = 0; e < E; ++e) fill[e] = 0;
+    for (t = 0; t < T; ++t) {
+        for (j = 0; j < k; ++j) {
+            int32_t ee = idx[t * k + j];
+            int64_t r = offs[ee] + fill[ee]++;
+            perm[r] = (int32_t)t;
+            inv[t * k + j] = (int32_t)r;
+        }
+    }
+    free(fill);
+    return 0;
+}
+
+/* Nearest-even bf16 bits of a double (8 significant bits, exponent range of
+ * fp32: normals from 2^-126, subnormals in steps of 2^-133, overflow to Inf
+ * at and above 2^128 - 2^119, the midpoint past the largest finite value). */
+uint16_t orc_bf16_from_double(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v), q, m, fl, rem;
+    int e;
+    if (isnan(v)) return (uint16_t)(sign | 0x7FC0u);
+    if (a >= ldexp(1.0, 128) - ldexp(1.0, 119)) return (uint16_t)(sign | 0x7F80u);
+    if (a == 0.0) return sign;
+    frexp(a, &e);                       /* a = f * 2^e, f in [0.5, 1) */
+    e = e - 1;                          /* a in [2^e, 2^(e+1)) */
+    if (e < -126) e = -126;             /* subnormal range: fixed quantum */
+    q = ldexp(1.0, e - 7);              /* spacing of bf16 values there */
+    m = a / q;                          /* exact: q is a power of two */
+    fl = floor(m);
+    rem = m - fl;
+    if (rem > 0.5 || (rem == 0.5 && fmod(fl, 2.0) != 0.0)) fl += 1.0;
+    a = fl * q;                         /* the rounded magnitude, exact */
+    {
+        /* encode: normal if a >= 2^-126, else subnormal */
+        uint32_t bits;
+        float f = (float)a;             /* exact: a has at most 8 significant bits */
+        memcpy(&bits, &f, 4);
+        return (uint16_t)(sign | (uint16_t)(bits >> 16));
+    }
+}
+
+/* Combine: y[t, c] = sum over j of w[t*k+j] * yp[inv[t*k+j], c], summed in
+ * fp64 and rounded once to bf16.  yp: bf16 [rows, C]; y: bf16 [T, C]. */
+int orc_moe_combine(const uint16_t* yp, int64_t rows, int64_t C, const int32_t* inv, const float* w,
+                    int64_t T, int32_t k, uint16_t* y)
+{
+    int64_t t;
+    for (t = 0; t < T * k; ++t)
+        if (inv[t] < 0 || inv[t] >= rows) return -1;
+    for (t = 0; t < T; ++t) {
+        int64_t c;
+        for (c = 0; c < C; ++c) {
+            double acc = 0.0;
+            int32_t j;
+            for (j = 0; j < k; ++j)
+                acc += (double)w[t * k + j] * orc_bf16_to_double(yp[(int64_t)inv[t * k + j] * C + c]);
+            y[t * C + c] = orc_bf16_from_double(acc);
+        }
+    }
+    return 0;
+}
+
+void orc_bf16_from_double_array(const double* v, int64_t n, uint16_t* out)
+{
+    int64_t i;
+    for (i = 0; i < n; ++i) out[i] = orc_bf16_from_double(v[i]);
 }

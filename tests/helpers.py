@@ -2,8 +2,8 @@
 import numpy as np
 import torch
 
-# GEMM tolerance (the task's contract for fp32-accumulated MXFP8 products
-# written as bf16, against the fp64 oracle on identical quantised inputs):
+# GEMM tolerance for fp32-accumulated MXFP8 products written as bf16,
+# against the fp64 oracle on identical quantised inputs:
 FROB_TOL = 5e-3        # ||G - R||_F / ||R||_F
 ELEM_TOL = 2e-2        # |G - R| / |R| where |R| > ELEM_FLOOR * rms(R)
 ELEM_FLOOR = 1e-2

@@ -2,7 +2,7 @@
 
 The rules (32-element blocks sharing one exponent -- opensourcebeat.com,
 "Enabling up to 41% faster pre-training: MXFP8 and DeepEP ...", FAQ; OCP MX
-v1.0 E8M0 scale and E4M3 elements as named by the task) are pinned against:
+v1.0 E8M0 scale and E4M3 elements) are pinned against:
 hand-worked blocks (tests/golden/hand_blocks.txt), two independent library
 codecs (ml_dtypes and torch float8), and properties of the definition.
 """
