@@ -155,16 +155,18 @@ __device__ __forceinline__ int32_t n_tiles(const Params& p) {
   return p.mode == kFwd ? cdiv32(p.N, BN) : cdiv32(p.K, BN);
 }
 
-// Tile t (a pair tile when CG = 2) as seen by CTA `rank` of its pair.
+// Group of tile t: the last group whose first tile is <= t.  A CTA visits
+// its tiles in increasing order, so the search advances from the previous
+// answer `e` (start at 0) instead of bisecting every time.
+__device__ __forceinline__ int32_t advance_group(const Sched& s, int32_t E, int32_t t, int32_t e) {
+  while (e + 1 < E && s.tile0[e + 1] <= t) ++e;
+  return e;
+}
+
+// Tile t (a pair tile when CG = 2) of group e as seen by CTA `rank` of its pair.
 template <int CG>
-__device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int32_t t, uint32_t rank) {
-  int32_t lo = 0, hi = p.E - 1;   // last group whose first tile is <= t
-  while (lo < hi) {
-    const int32_t mid = (lo + hi + 1) >> 1;
-    if (s.tile0[mid] <= t) lo = mid; else hi = mid - 1;
-  }
+__device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int32_t t, int32_t e, uint32_t rank) {
   Tile tl;
-  const int32_t e = lo;
   const int32_t row0 = s.off[e], m = s.off[e + 1] - s.off[e];
   const int32_t munits = group_m_units<CG>(p, m);
   const int32_t local = t - s.tile0[e];
@@ -343,12 +345,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer (every CTA)
-      uint32_t it = 0;
+      uint32_t it = 0, s = 0, ph = 0;
+      int32_t eh = 0;
       bool failed = false;
       for (int32_t t = unit0; t < total && !failed; t += nunits) {
-        const Tile tl = decode_tile<CG>(p, sc, t, rank);
+        eh = advance_group(sc, p.E, t, eh);
+        const Tile tl = decode_tile<CG>(p, sc, t, eh, rank);
         for (int32_t kb0 = 0; kb0 < tl.kblocks; kb0 += C::KS) {
-          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
           if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, lim)) {
             record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
             failed = true;
@@ -392,6 +395,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             tma_load_2d(ssb + C::KS * 512, &tmSFB, 0, yb1, fb);
           }
           ++it;
+          if (++s == STAGES) { s = 0; ph ^= 1; }
         }
       }
       if (failed) {
@@ -411,11 +415,32 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       // M = 128*CG, N = 256; the scale-factor ids (bits 4-5 for B, 29-30 for
       // A) select the byte of the 32-bit scale column used by each K step.
       const uint32_t idesc0 = (1u << 23) | (uint32_t(BN >> 3) << 17) | (uint32_t((BM * CG) >> 4) << 24);
-      uint32_t it = 0, j = 0;
+      // The tensor pipe queues only a few instructions, so scalar work between
+      // MMAs stalls it: everything below is set up once, descriptors of a
+      // slot are the base descriptor plus the slot's offset in 16-byte units
+      // (the 14-bit start field cannot overflow below 256 KB), and the stage
+      // index and phase advance incrementally.
+      const uint64_t da0 = desc_kmajor_sw128(smem_addr(smem + C::OFF_A));
+      const uint64_t db0 = desc_kmajor_sw128(smem_addr(smem + C::OFF_B));
+      const uint64_t dsa0 = desc_sf_32x16(smem_addr(smem + C::OFF_SFA));
+      const uint64_t dsb0 = desc_sf_32x16(smem_addr(smem + C::OFF_SFB));
+      const uint32_t sf_t0 = tmem + C::SF_COL;
+      // fwd/dgrad: every tile has the same K loop; wgrad: the group's rows.
+      const int64_t L_fixed = p.mode == kFwd ? p.K : p.N;
+      const int32_t kb_fixed = static_cast<int32_t>((L_fixed + BK - 1) / BK);
+      const int32_t ks_fixed = static_cast<int32_t>((L_fixed - int64_t(BK) * (kb_fixed - 1) + 31) / 32);
+      uint32_t s = 0, ph = 0, j = 0;
+      int32_t eh = 0;
       bool failed = false;
       for (int32_t t = unit0; t < total && !failed; t += nunits) {
-        const Tile tl = decode_tile<CG>(p, sc, t, 0);
-        if (tl.kblocks == 0) continue;
+        int32_t kblocks = kb_fixed, ksteps_last = ks_fixed;
+        if (p.mode == kWgrad) {
+          eh = advance_group(sc, p.E, t, eh);
+          const int32_t m = sc.off[eh + 1] - sc.off[eh];
+          kblocks = (m + BK - 1) / BK;
+          if (kblocks == 0) continue;
+          ksteps_last = (m - BK * (kblocks - 1) + 31) / 32;
+        }
         const uint32_t d_tmem = tmem + (j & 1) * C::ACC_STRIDE;
         if (!mbar_wait(acc_empty, (j & 1) ^ 1, abort_flag, lim)) {
           record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
@@ -423,50 +448,52 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           break;
         }
         tc_fence_after();
-        for (int32_t kb0 = 0; kb0 < tl.kblocks; kb0 += C::KS) {
-          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+        uint32_t acc = 0;
+        for (int32_t kb0 = 0; kb0 < kblocks; kb0 += C::KS) {
           if (!mbar_wait(full_bar(s), ph, abort_flag, lim)) {
             record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
             failed = true;
             break;
           }
           tc_fence_after();
-          const int32_t nh = min(C::KS, tl.kblocks - kb0);
-          const uint32_t sfa_s = smem_addr(smem + C::OFF_SFA + s * C::KS * SFA_TILE);
-          const uint32_t sfb_s = smem_addr(smem + C::OFF_SFB + s * C::KS * SFB_TILE);
-          for (int32_t h = 0; h < nh; ++h) {
+#pragma unroll
+          for (int h = 0; h < C::KS; ++h) {
             const int32_t kb = kb0 + h;
-            const uint32_t q = s * C::KS + h;
-            const uint32_t sfa_t = tmem + C::SF_COL + SF_STRIDE * q, sfb_t = sfa_t + 4;
-            const uint64_t dsa = desc_sf_32x16(sfa_s + 512 * h);
-            const uint64_t dsb0 = desc_sf_32x16(sfb_s + 512 * h);
-            const uint64_t dsb1 = desc_sf_32x16(sfb_s + 512 * (C::KS + h));
-            const uint64_t da = desc_kmajor_sw128(smem_addr(smem + C::OFF_A + q * C::A_TILE));
-            const uint64_t db = desc_kmajor_sw128(smem_addr(smem + C::OFF_B + q * C::B_TILE));
-            const int32_t nk = (kb == tl.kblocks - 1) ? tl.ksteps_last : BK / 32;
-            if constexpr (CG == 2) {
-              tc_cp_32x128b_x4_pair(sfa_t, dsa);
-              tc_cp_32x128b_x4_pair(sfb_t, dsb0);
-              tc_cp_32x128b_x4_pair(sfb_t + 4, dsb1);
-            } else {
-              tc_cp_32x128b_x4(sfa_t, dsa);
-              tc_cp_32x128b_x4(sfb_t, dsb0);
-              tc_cp_32x128b_x4(sfb_t + 4, dsb1);
-            }
-            for (int32_t k = 0; k < nk; ++k) {
-              const uint32_t idesc = idesc0 | (uint32_t(k) << 4) | (uint32_t(k) << 29);
-              // +2 per step: the start-address field counts 16-byte units, one step is 32 bytes of K
-              if constexpr (CG == 2)
-                tc_mma_mxf8_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
-                                 sfb_t | (uint32_t(k) << 30), (kb | k) != 0);
-              else
-                tc_mma_mxf8(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
-                            sfb_t | (uint32_t(k) << 30), (kb | k) != 0);
+            if (kb < kblocks) {
+              const uint32_t q = s * C::KS + h;
+              const uint32_t sfa_t = sf_t0 + SF_STRIDE * q, sfb_t = sfa_t + 4;
+              const uint64_t dsa = dsa0 + (SFA_TILE >> 4) * q;
+              const uint64_t dsb = dsb0 + (SFB_TILE >> 4) * C::KS * s + (512 >> 4) * h;
+              if constexpr (CG == 2) {
+                tc_cp_32x128b_x4_pair(sfa_t, dsa);
+                tc_cp_32x128b_x4_pair(sfb_t, dsb);
+                tc_cp_32x128b_x4_pair(sfb_t + 4, dsb + (512 >> 4) * C::KS);
+              } else {
+                tc_cp_32x128b_x4(sfa_t, dsa);
+                tc_cp_32x128b_x4(sfb_t, dsb);
+                tc_cp_32x128b_x4(sfb_t + 4, dsb + (512 >> 4) * C::KS);
+              }
+              const uint64_t da = da0 + (C::A_TILE >> 4) * q, db = db0 + (C::B_TILE >> 4) * q;
+              const int32_t nk = (kb == kblocks - 1) ? ksteps_last : BK / 32;
+#pragma unroll
+              for (int k = 0; k < BK / 32; ++k) {
+                if (k < nk) {
+                  // +2 per step: the start-address field counts 16-byte units, one step is 32 bytes of K
+                  const uint32_t idesc = idesc0 | (uint32_t(k) << 4) | (uint32_t(k) << 29);
+                  if constexpr (CG == 2)
+                    tc_mma_mxf8_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
+                                     sfb_t | (uint32_t(k) << 30), acc);
+                  else
+                    tc_mma_mxf8(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
+                                sfb_t | (uint32_t(k) << 30), acc);
+                  acc = 1;
+                }
+              }
             }
           }
           if constexpr (CG == 2) tc_commit_pair(empty_bar(s), 0x3);
           else tc_commit(empty_bar(s));
-          ++it;
+          if (++s == STAGES) { s = 0; ph ^= 1; }
         }
         if (failed) break;
         if constexpr (CG == 2) tc_commit_pair(acc_full, 0x3);
@@ -487,8 +514,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int srow = lane >> 3, schunk = lane & 7;
     const int32_t row_base = 32 * static_cast<int32_t>(quarter);
     uint32_t j = 0, ec = 0;
+    int32_t eh = 0;
     for (int32_t t = unit0; t < total; t += nunits) {
-      const Tile tl = decode_tile<CG>(p, sc, t, rank);
+      eh = advance_group(sc, p.E, t, eh);
+      const Tile tl = decode_tile<CG>(p, sc, t, eh, rank);
       const int32_t vr = max(0, min(32, tl.rows - row_base));       // valid rows of this warp's slice
       uint16_t* out_tile = p.out + tl.out_row * p.out_ld + tl.out_col;
       if (tl.kblocks == 0) {
@@ -756,19 +785,21 @@ cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** detail) {
   // Tile configuration: 1-CTA 128x256 tiles by default -- on B200 they beat
-  // CTA pairs on every pass of the DeepSeek-V3-like layers (pairs also waste
-  // up to 128 rows per group in fwd/dgrad).  Stage depth: 256-deep stages for
-  // fwd/dgrad, except for a short odd K loop whose last stage would run half
-  // empty; 128-deep stages for wgrad, whose K loops (the groups' token counts)
-  // are short and whose tiles are epilogue-heavy.  MXF8_GEMM_CTA_PAIR=1/0 and
+  // CTA pairs on the DeepSeek-V3-like layers (pairs also waste up to 128
+  // rows per group in fwd/dgrad).  Stage depth: 128-deep stages (4-stage
+  // ring) except for long K loops -- fwd/dgrad with at least 64 K blocks,
+  // wgrad with at least 1024 rows per group on average -- where 256-deep
+  // stages (2-stage ring) measured faster.  MXF8_GEMM_CTA_PAIR=1/0 and
   // MXF8_GEMM_KS=1/2 override the choices.
   int cg = 1;
   const char* env = std::getenv("MXF8_GEMM_CTA_PAIR");
   if (env && std::strcmp(env, "1") == 0) cg = 2;
   int ks = 1;
-  if (a.mode != kWgrad) {
+  if (a.mode == kWgrad) {
+    if (a.M >= int64_t(1024) * a.E) ks = 2;
+  } else {
     const int64_t kblocks = ((a.mode == kFwd ? a.K : a.N) + BK - 1) / BK;
-    ks = (kblocks % 2 == 0 || kblocks >= 24) ? 2 : 1;
+    if (kblocks >= 64) ks = 2;
   }
   env = std::getenv("MXF8_GEMM_KS");
   if (env && std::strcmp(env, "1") == 0) ks = 1;
