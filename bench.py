@@ -287,6 +287,7 @@ def run_ours(args, rank, world, local_rank):
         out["cpu_baseline"] = cpu_baseline(w, budget_s=12.0)
     out["e2e"] = e2e(args, mx, w, layers, dev, world)
     out["quantising_epilogue"] = quantising_epilogue(mx, layers[0])
+    out["moe_dispatch"] = moe_dispatch(mx, args, pk["hbm_gbs"])
     return out
 
 
@@ -381,6 +382,49 @@ def quantising_epilogue(mx, L: Linear, iters=20):
         r["tflops"] = round(L.flops_per_pass() / (r["quantising_epilogue_ms"] * 1e-3) / 1e12, 1)
         res[mode] = r
     return res
+
+
+def moe_dispatch(mx, args, hbm_gbs, iters=20):
+    """The steps around the GEMMs on the DeepSeek-V3-16B-like routing (8192
+    tokens, top-6 of 64 experts, hidden 2048): the dispatch plan, the token
+    permute fused with dual MXFP8 quantisation, and the weighted combine of
+    the down projection's outputs.  Timed on their own, not in the step."""
+    r = wl.routing("ds-v3-16b")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    idx = torch.from_numpy(r.idx).to(dev)
+    w = torch.from_numpy(r.w).to(dev)
+    x = wl.normal_bf16((r.T, r.K), 1.0, 101, device=dev)
+    offs, perm, inv, work = mx.mxfp8_moe_plan(idx, r.E)
+    R = perm.numel()
+    q, s, qT, sT = mx.mxfp8_permute_quantize_dual(x, perm, offs)
+    yp = wl.normal_bf16((R, r.K), 1.0, 102, device=dev)
+    y = torch.empty((r.T, r.K), dtype=torch.bfloat16, device=dev)
+
+    def t(fn):
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(iters):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+
+    plan_ms = t(lambda: mx.mxfp8_moe_plan(idx, r.E, work=work))
+    pq_ms = t(lambda: mx.mxfp8_permute_quantize_dual(x, perm, offs, q, s, qT, sT))
+    cb_ms = t(lambda: mx.mxfp8_moe_combine(yp, inv, w, out=y))
+    if mx.mxfp8_get_status(work) != 0:
+        raise SystemExit("bench: dispatch plan reported a bad routing")
+    pq_bytes = R * r.K * (2 + 2 * (1 + 1 / 32))          # gathered bf16 read, both MXFP8 layouts written
+    cb_bytes = R * r.K * 2 + r.T * r.K * 2               # expert outputs read, token outputs written
+    return {"routing": f"{r.T} tokens, top-{r.k} of {r.E}, hidden {r.K}", "plan_ms": round(plan_ms, 4),
+            "permute_quantize_ms": round(pq_ms, 4),
+            "permute_quantize_gbs": round(pq_bytes / (pq_ms * 1e-3) / 1e9, 1),
+            "permute_quantize_frac": round(pq_bytes / (pq_ms * 1e-3) / 1e9 / hbm_gbs, 4),
+            "combine_ms": round(cb_ms, 4), "combine_gbs": round(cb_bytes / (cb_ms * 1e-3) / 1e9, 1),
+            "combine_frac": round(cb_bytes / (cb_ms * 1e-3) / 1e9 / hbm_gbs, 4)}
 
 
 # ---------------------------------------------------------------- CPU oracle baseline / reference arm

@@ -84,7 +84,8 @@ typedef enum {
     MXF8_ERR_UNSUPPORTED = 3,  /* the current device is not sm_100 */
     MXF8_ERR_CUDA = 4,         /* a CUDA call failed; see mxfp8_last_cuda_error() */
     MXF8_ERR_BAD_OFFSETS = 5,  /* device side: d_offs is not a valid prefix of `rows` */
-    MXF8_ERR_TIMEOUT = 6       /* device side: a pipeline wait ran past its limit */
+    MXF8_ERR_TIMEOUT = 6,      /* device side: a pipeline wait ran past its limit */
+    MXF8_ERR_BAD_ROUTING = 7   /* device side: an expert id outside [0, num_experts) */
 } mxf8_status;
 
 /* Largest num_groups (experts) a grouped GEMM accepts. */
@@ -245,6 +246,70 @@ MXF8_API mxf8_status mxfp8_grouped_gemm_fwd_noalloc(const uint8_t* xq, const uin
                                                     const int32_t* d_offs, int32_t E, int64_t M, int64_t N,
                                                     int64_t K, uint16_t* y, int32_t* host_status,
                                                     void* stream);
+
+/* ---------------------------------------------------------------- MoE dispatch / combine */
+/* The steps around the grouped GEMM in a Mixture-of-Experts layer on one
+ * GPU: tokens are permuted so every expert's rows are contiguous (with their
+ * real counts, no capacity padding: iitak.ru, "NVIDIA в 10 раз ускорила
+ * обучение моделей-«смесей экспертов» на JAX", paragraph on the Transformer
+ * Engine grouped GEMM), quantised on the way, and the experts' outputs are
+ * combined back per token with the router weights.  Across GPUs these are
+ * the dispatch and combine all-to-alls (opensourcebeat.com, section
+ * "Двухсторонняя атака: MXFP8 и DeepEP"); the pages give no formulas, so the
+ * plainest reading is used: a stable grouping by expert and a weighted sum. */
+
+/* Largest num_experts the plan accepts. */
+#define MXF8_MOE_MAX_EXPERTS 256
+
+/* Workspace of mxfp8_moe_plan in bytes (status word + per-pair ranks +
+ * per-chunk histograms). */
+MXF8_API int64_t mxfp8_moe_plan_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t num_experts);
+
+/* Dispatch plan of a top-k routing.
+ *   idx     int32 [T, k] expert id of slot j of token t (row-major)
+ *   offs    int32 [E + 1] out: exclusive prefix of the per-expert pair counts
+ *           (offs[E] = T*k when every id is valid) -- the grouped GEMM's d_offs
+ *   perm    int32 [T*k] out: token of permuted row r
+ *   inv     int32 [T, k] out: permuted row of slot (t, j)
+ * Inside an expert the pairs keep ascending (token, slot) order, so the plan
+ * is deterministic.  work/work_bytes >= mxfp8_moe_plan_workspace_bytes; the
+ * device status (mxfp8_get_status(work)) is MXF8_ERR_BAD_ROUTING if an id is
+ * outside [0, E): such slots get inv = -1 and no row.
+ * Errors: INVALID_ARG (null pointers, T < 0, k < 1, E outside [1, 256],
+ * T*k >= 2^31, small workspace), ALIGNMENT (work), UNSUPPORTED, CUDA. */
+MXF8_API mxf8_status mxfp8_moe_plan(const int32_t* idx, int64_t num_tokens, int32_t top_k, int32_t num_experts,
+                                    int32_t* offs, int32_t* perm, int32_t* inv, void* work, int64_t work_bytes,
+                                    void* stream);
+
+/* Token permute fused with dual MXFP8 quantisation: quantises the matrix
+ * Xp[r] = x[perm[r]] (r < rows, grouped by d_offs) into both layouts, byte
+ * for byte what mxfp8_quantize_dual(Xp, rows, cols, d_offs, ...) writes,
+ * without materialising Xp.
+ *   x       bf16 [num_tokens, cols], cols % 32 == 0
+ *   perm    int32 [rows] (from mxfp8_moe_plan; rows = T*k); an entry outside
+ *           [0, num_tokens) quantises a zero row
+ *   d_offs  int32 [num_groups + 1] (from mxfp8_moe_plan)
+ *   q, scales, qT, ldT, scalesT: as mxfp8_quantize_dual with `rows` rows.
+ * Errors as mxfp8_quantize_dual, plus INVALID_ARG for null perm/x. */
+MXF8_API mxf8_status mxfp8_permute_quantize_dual(const uint16_t* x, int64_t num_tokens, int64_t cols,
+                                                 const int32_t* perm, int64_t rows, const int32_t* d_offs,
+                                                 int32_t num_groups, uint8_t* q, uint8_t* scales,
+                                                 int64_t scale_bytes, uint8_t* qT, int64_t ldT, uint8_t* scalesT,
+                                                 int64_t scaleT_bytes, void* stream);
+
+/* Combine: y[t, c] = sum over j < k of w[t, j] * yp[inv[t, j], c].  The
+ * products (fp32 weight x bf16 value) are exact in fp64, the sum runs in
+ * fp64 in slot order and is rounded once to bf16 (nearest even).
+ *   yp      bf16 [rows, cols] expert outputs in permuted order, cols % 8 == 0
+ *   inv     int32 [T, k] (from mxfp8_moe_plan); an entry outside [0, rows)
+ *           contributes nothing
+ *   w       fp32 [T, k] router weights
+ *   y       bf16 [T, cols] out
+ * Errors: INVALID_ARG (null pointers, cols % 8, T < 0, k < 1), ALIGNMENT
+ * (yp, y), UNSUPPORTED, CUDA. */
+MXF8_API mxf8_status mxfp8_moe_combine(const uint16_t* yp, int64_t rows, int64_t cols, const int32_t* inv,
+                                       const float* w, int64_t num_tokens, int32_t top_k, uint16_t* y,
+                                       void* stream);
 
 /* ---------------------------------------------------------------- status */
 

@@ -29,14 +29,15 @@ _vp = ctypes.c_void_p
 MXF8_OK = 0
 MXF8_GEMM_MAX_GROUPS = 256
 STATUS_NAMES = {0: "MXF8_OK", 1: "MXF8_ERR_INVALID_ARG", 2: "MXF8_ERR_ALIGNMENT", 3: "MXF8_ERR_UNSUPPORTED",
-                4: "MXF8_ERR_CUDA", 5: "MXF8_ERR_BAD_OFFSETS", 6: "MXF8_ERR_TIMEOUT"}
+                4: "MXF8_ERR_CUDA", 5: "MXF8_ERR_BAD_OFFSETS", 6: "MXF8_ERR_TIMEOUT", 7: "MXF8_ERR_BAD_ROUTING"}
 
 EXPORTED = ("mxfp8_rowwise_scale_bytes", "mxfp8_colwise_pitch", "mxfp8_colwise_scale_bytes", "mxfp8_colwise_ld",
             "mxfp8_workspace_bytes", "mxfp8_quantize_rowwise", "mxfp8_quantize_colwise",
             "mxfp8_grouped_gemm_fwd", "mxfp8_grouped_gemm_dgrad", "mxfp8_grouped_gemm_wgrad",
             "mxfp8_get_status", "mxfp8_status_string", "mxfp8_last_cuda_error", "mxfp8_device_supported",
             "mxfp8_grouped_gemm_fwd_noalloc", "mxfp8_quantize_dual", "mxfp8_grouped_gemm_fwd_quant",
-            "mxfp8_grouped_gemm_dgrad_quant")
+            "mxfp8_grouped_gemm_dgrad_quant", "mxfp8_moe_plan_workspace_bytes", "mxfp8_moe_plan",
+            "mxfp8_permute_quantize_dual", "mxfp8_moe_combine")
 
 
 class MXFP8Error(RuntimeError):
@@ -78,6 +79,15 @@ def lib() -> ctypes.CDLL:
             getattr(L, n).restype = _i32
             getattr(L, n).argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i64,
                                       _vp, _i64, _vp, _i64, _vp, _i64, _vp]
+        L.mxfp8_moe_plan_workspace_bytes.restype = _i64
+        L.mxfp8_moe_plan_workspace_bytes.argtypes = [_i64, _i32, _i32]
+        L.mxfp8_moe_plan.restype = _i32
+        L.mxfp8_moe_plan.argtypes = [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _i64, _vp]
+        L.mxfp8_permute_quantize_dual.restype = _i32
+        L.mxfp8_permute_quantize_dual.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _i32, _vp, _vp, _i64, _vp, _i64,
+                                                  _vp, _i64, _vp]
+        L.mxfp8_moe_combine.restype = _i32
+        L.mxfp8_moe_combine.argtypes = [_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp]
         L.mxfp8_grouped_gemm_fwd_noalloc.restype = _i32
         L.mxfp8_grouped_gemm_fwd_noalloc.argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp,
                                                      ctypes.POINTER(_i32), _vp]
@@ -285,3 +295,50 @@ def mxfp8_get_status(work: torch.Tensor, stream=None) -> int:
 
 def mxfp8_device_supported() -> bool:
     return bool(lib().mxfp8_device_supported())
+
+
+# ------------------------------------------------------------------ MoE dispatch / combine
+def mxfp8_moe_plan(idx: torch.Tensor, num_experts: int, work=None, stream=None):
+    """idx: int32 [T, k] expert ids -> (offs int32 [E+1], perm int32 [T*k], inv int32 [T, k], work).
+    Pairs grouped by expert in ascending (token, slot) order; mxfp8_get_status(work) reports ids out of range."""
+    assert idx.dtype == torch.int32 and idx.dim() == 2
+    T, k = idx.shape
+    dev = idx.device
+    offs = torch.empty(num_experts + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)[: T * k]
+    inv = torch.empty((T, k), dtype=torch.int32, device=dev)
+    need = lib().mxfp8_moe_plan_workspace_bytes(T, k, num_experts)
+    work = work if work is not None else torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib().mxfp8_moe_plan(_ptr(idx), T, k, num_experts, _ptr(offs), _ptr(perm), _ptr(inv), _ptr(work),
+                                work.numel(), _stream(stream)), "mxfp8_moe_plan")
+    return offs, perm, inv, work
+
+
+def mxfp8_permute_quantize_dual(x: torch.Tensor, perm: torch.Tensor, offs: torch.Tensor, q=None, scales=None, qT=None,
+                                scalesT=None, stream=None):
+    """Quantises Xp = x[perm] (grouped by offs) into both MXFP8 layouts without
+    materialising Xp -> (q, scales, qT, scalesT), as mxfp8_quantize_dual(x[perm], offs)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and perm.dtype == torch.int32
+    T, C = x.shape
+    R = perm.numel()
+    G = _groups(offs)
+    ld = mxfp8_colwise_ld(R, G)
+    q = q if q is not None else torch.empty((R, C), dtype=torch.uint8, device=x.device)
+    scales = scales if scales is not None else _u8(mxfp8_rowwise_scale_bytes(R, C, G), x.device)
+    qT = qT if qT is not None else torch.empty((C, ld), dtype=torch.uint8, device=x.device)
+    scalesT = scalesT if scalesT is not None else _u8(mxfp8_colwise_scale_bytes(R, C, G), x.device)
+    _check(lib().mxfp8_permute_quantize_dual(_ptr(x), T, C, _ptr(perm) if R else None, R, _ptr(offs), G, _ptr(q),
+                                             _ptr(scales), scales.numel(), _ptr(qT), ld, _ptr(scalesT),
+                                             scalesT.numel(), _stream(stream)), "mxfp8_permute_quantize_dual")
+    return q, scales, qT, scalesT
+
+
+def mxfp8_moe_combine(yp: torch.Tensor, inv: torch.Tensor, w: torch.Tensor, out=None, stream=None):
+    """y[t] = sum_j w[t, j] * yp[inv[t, j]] (fp64 sum, one bf16 rounding) -> bf16 [T, cols]."""
+    assert yp.dtype == torch.bfloat16 and inv.dtype == torch.int32 and w.dtype == torch.float32
+    rows, C = yp.shape
+    T, k = inv.shape
+    out = out if out is not None else torch.empty((T, C), dtype=torch.bfloat16, device=yp.device)
+    _check(lib().mxfp8_moe_combine(_ptr(yp) if rows else None, rows, C, _ptr(inv), _ptr(w), T, k, _ptr(out),
+                                   _stream(stream)), "mxfp8_moe_combine")
+    return out

@@ -307,6 +307,66 @@ mxf8_status mxfp8_grouped_gemm_dgrad_quant(const uint8_t* dyq, const uint8_t* dy
   return run_gemm(g, work, stream);
 }
 
+int64_t mxfp8_moe_plan_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t num_experts) {
+  if (num_tokens < 0 || top_k < 1 || num_experts < 1) return 0;
+  const int64_t pairs = num_tokens * top_k;
+  return kWorkspaceBytes + round_up(pairs * 4, 256) +
+         round_up(mxf8::moe_plan_chunks(pairs) * int64_t(num_experts) * 4, 256);
+}
+
+mxf8_status mxfp8_moe_plan(const int32_t* idx, int64_t num_tokens, int32_t top_k, int32_t num_experts,
+                           int32_t* offs, int32_t* perm, int32_t* inv, void* work, int64_t work_bytes,
+                           void* stream) {
+  if (num_tokens < 0 || top_k < 1 || num_experts < 1 || num_experts > MXF8_MOE_MAX_EXPERTS)
+    return MXF8_ERR_INVALID_ARG;
+  const int64_t pairs = num_tokens * top_k;
+  if (pairs >= (int64_t(1) << 31)) return MXF8_ERR_INVALID_ARG;
+  if (!offs || !work || (pairs > 0 && (!idx || !perm || !inv))) return MXF8_ERR_INVALID_ARG;
+  if (work_bytes < mxfp8_moe_plan_workspace_bytes(num_tokens, top_k, num_experts)) return MXF8_ERR_INVALID_ARG;
+  if (!aligned16(work)) return MXF8_ERR_ALIGNMENT;
+  mxf8_status s = check_device();
+  if (s != MXF8_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(work);
+  int32_t* status = reinterpret_cast<int32_t*>(w);
+  int32_t* rank = reinterpret_cast<int32_t*>(w + kWorkspaceBytes);
+  int32_t* hist = reinterpret_cast<int32_t*>(w + kWorkspaceBytes + round_up(pairs * 4, 256));
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  e = mxf8::launch_moe_plan(idx, num_tokens, top_k, num_experts, offs, perm, inv, status, rank, hist, st);
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "moe_plan launch");
+}
+
+mxf8_status mxfp8_permute_quantize_dual(const uint16_t* x, int64_t num_tokens, int64_t cols, const int32_t* perm,
+                                        int64_t rows, const int32_t* d_offs, int32_t num_groups, uint8_t* q,
+                                        uint8_t* scales, int64_t scale_bytes, uint8_t* qT, int64_t ldT,
+                                        uint8_t* scalesT, int64_t scaleT_bytes, void* stream) {
+  if (num_tokens < 0 || (rows > 0 && (!x || !perm)) || !d_offs) return MXF8_ERR_INVALID_ARG;
+  mxf8_status s = check_quant_args(x, rows, cols, num_groups, q, scales, scale_bytes,
+                                   mxfp8_rowwise_scale_bytes(rows, cols, num_groups));
+  if (s != MXF8_OK) return s;
+  s = check_quant_args(x, rows, cols, num_groups, qT, scalesT, scaleT_bytes,
+                       mxfp8_colwise_scale_bytes(rows, cols, num_groups));
+  if (s != MXF8_OK) return s;
+  if (ldT != mxfp8_colwise_ld(rows, num_groups)) return MXF8_ERR_INVALID_ARG;
+  if ((s = check_device()) != MXF8_OK) return s;
+  cudaError_t e = mxf8::launch_permute_quantize_dual(x, num_tokens, cols, perm, rows, d_offs, num_groups, q, scales,
+                                                     qT, ldT, scalesT, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "permute_quantize_dual launch");
+}
+
+mxf8_status mxfp8_moe_combine(const uint16_t* yp, int64_t rows, int64_t cols, const int32_t* inv, const float* w,
+                              int64_t num_tokens, int32_t top_k, uint16_t* y, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 8 != 0 || num_tokens < 0 || top_k < 1) return MXF8_ERR_INVALID_ARG;
+  if (num_tokens > 0 && (!inv || !w || !y || (rows > 0 && !yp))) return MXF8_ERR_INVALID_ARG;
+  if (!aligned16(yp) || !aligned16(y)) return MXF8_ERR_ALIGNMENT;
+  mxf8_status s = check_device();
+  if (s != MXF8_OK) return s;
+  cudaError_t e = mxf8::launch_moe_combine(yp, rows, cols, inv, w, num_tokens, top_k, y,
+                                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "moe_combine launch");
+}
+
 mxf8_status mxfp8_get_status(const void* work, void* stream, int32_t* device_status) {
   if (!work || !device_status) return MXF8_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -326,6 +386,7 @@ const char* mxfp8_status_string(int32_t status) {
     case MXF8_ERR_CUDA: return "CUDA error";
     case MXF8_ERR_BAD_OFFSETS: return "group offsets are not a valid prefix";
     case MXF8_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case MXF8_ERR_BAD_ROUTING: return "an expert id is outside [0, num_experts)";
     default: return "unknown status";
   }
 }

@@ -17,6 +17,21 @@ cudaError_t launch_quantize_dual(const uint16_t* x, int64_t rows, int64_t cols, 
                                  int32_t G, uint8_t* q, uint8_t* sf, uint8_t* qT, int64_t ldT, uint8_t* sfT,
                                  cudaStream_t stream);
 
+// Dual quantisation of x[perm[r]] for r < rows (the MoE token permute);
+// perm entries outside [0, src_rows) read as zero rows.
+cudaError_t launch_permute_quantize_dual(const uint16_t* x, int64_t src_rows, int64_t cols, const int32_t* perm,
+                                         int64_t rows, const int32_t* offs, int32_t G, uint8_t* q, uint8_t* sf,
+                                         uint8_t* qT, int64_t ldT, uint8_t* sfT, cudaStream_t stream);
+
+// MoE dispatch plan: chunks of ranked pairs (workspace sizing) and the launch.
+int64_t moe_plan_chunks(int64_t pairs);
+cudaError_t launch_moe_plan(const int32_t* idx, int64_t T, int32_t k, int32_t E, int32_t* offs, int32_t* perm,
+                            int32_t* inv, int32_t* status, int32_t* rank, int32_t* hist, cudaStream_t stream);
+
+// MoE combine: y[t] = sum_j w[t, j] * yp[inv[t, j]] (cols % 8 == 0).
+cudaError_t launch_moe_combine(const uint16_t* yp, int64_t rows, int64_t cols, const int32_t* inv, const float* w,
+                               int64_t T, int32_t k, uint16_t* y, cudaStream_t stream);
+
 enum GemmMode : int { kFwd = 0, kDgrad = 1, kWgrad = 2 };
 
 // One grouped GEMM.  a/b: operand codes (K-major), lda/ldb their row strides

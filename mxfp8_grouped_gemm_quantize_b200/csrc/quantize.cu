@@ -187,10 +187,15 @@ __global__ void __launch_bounds__(kThreads) quantize_colwise_kernel(
 // one 32-element row block), so rowwise codes and scales are encoded straight
 // from the loaded registers; the tile then goes to shared memory and the
 // colwise pass proceeds exactly as in quantize_colwise_kernel.
+// GATHER: row r of the quantised matrix is row gather[r] of x (a token
+// permute fused with the quantisation); a gather index outside [0, src_rows)
+// reads as a zero row.
+template <bool GATHER>
 __global__ void __launch_bounds__(kThreads) quantize_dual_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, const int32_t* __restrict__ offs,
     int32_t G, uint8_t* __restrict__ q, uint8_t* __restrict__ sf, int64_t pitch_r,
-    uint8_t* __restrict__ qT, int64_t ldT, uint8_t* __restrict__ sfT, int64_t pitch_c) {
+    uint8_t* __restrict__ qT, int64_t ldT, uint8_t* __restrict__ sfT, int64_t pitch_c,
+    const int32_t* __restrict__ gather, int64_t src_rows) {
   __shared__ __align__(16) uint32_t tile[128 * 64];
   __shared__ __align__(16) uint8_t atom_r[512];
   __shared__ __align__(16) uint8_t atom_c[512];
@@ -205,7 +210,11 @@ __global__ void __launch_bounds__(kThreads) quantize_dual_kernel(
   for (int i = 0; i < 8; ++i) {
     const int rr = rsub + 16 * i;
     v[i] = make_uint4(0, 0, 0, 0);
-    if (rr < br.nrows && col_ok) v[i] = ld_stream(x + (br.row0 + rr) * cols + col0 + 8 * ch);
+    if (rr < br.nrows && col_ok) {
+      int64_t src = br.row0 + rr;
+      if constexpr (GATHER) src = __ldg(gather + src);
+      if (!GATHER || (src >= 0 && src < src_rows)) v[i] = ld_stream(x + src * cols + col0 + 8 * ch);
+    }
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -308,8 +317,19 @@ cudaError_t launch_quantize_dual(const uint16_t* x, int64_t rows, int64_t cols, 
   const int64_t nb = block_bound(rows, G);
   if (nb == 0) return cudaSuccess;
   const dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>((cols + 127) / 128));
-  quantize_dual_kernel<<<grid, kThreads, 0, stream>>>(x, rows, cols, offs, G, q, sf, (cols + 127) / 128, qT, ldT,
-                                                       sfT, nb);
+  quantize_dual_kernel<false><<<grid, kThreads, 0, stream>>>(x, rows, cols, offs, G, q, sf, (cols + 127) / 128, qT,
+                                                              ldT, sfT, nb, nullptr, rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_quantize_dual(const uint16_t* x, int64_t src_rows, int64_t cols, const int32_t* perm,
+                                         int64_t rows, const int32_t* offs, int32_t G, uint8_t* q, uint8_t* sf,
+                                         uint8_t* qT, int64_t ldT, uint8_t* sfT, cudaStream_t stream) {
+  const int64_t nb = block_bound(rows, G);
+  if (nb == 0) return cudaSuccess;
+  const dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>((cols + 127) / 128));
+  quantize_dual_kernel<true><<<grid, kThreads, 0, stream>>>(x, rows, cols, offs, G, q, sf, (cols + 127) / 128, qT,
+                                                             ldT, sfT, nb, perm, src_rows);
   return cudaGetLastError();
 }
 
