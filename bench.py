@@ -53,7 +53,41 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quantiser", default="dual", choices=["dual", "separate"],
                     help="dual: one fused kernel writes both layouts of X, W and dY")
+    # profiling aids (the headline line uses the defaults)
+    ap.add_argument("--linears", default="all", help="comma-separated subset of the workload's linears")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the measurements outside the step (e2e, quantising epilogue, MoE dispatch)")
     return ap.parse_args()
+
+
+GEMM_PROFILE = os.path.join(ROOT, "profiles", "grouped_gemm_ds-v3-16b_gate_up.md")
+GEMM_SOURCES = ("grouped_gemm.cu", "ptx.cuh", "codec.cuh", "launch.h")
+
+
+def gemm_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "mxfp8_grouped_gemm_quantize_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def gemm_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary (the mean over
+    the gate/up linear's fwd, dgrad and wgrad launches), or None when the
+    summary is missing or the kernel sources changed since it was taken."""
+    try:
+        kv = {}
+        for line in open(GEMM_PROFILE, encoding="utf-8"):
+            if ":" in line and line.split(":")[0].strip() in ("traffic_bytes_per_launch", "kernel_sources_sha256"):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip().strip("`")
+        if kv.get("kernel_sources_sha256") != gemm_sources_sha256():
+            return None
+        return int(kv["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def peaks():
@@ -199,7 +233,10 @@ def run_ours(args, rank, world, local_rank):
     if not mx.mxfp8_device_supported():
         raise SystemExit("bench: the current device is not sm_100")
     w = wl.WORKLOADS[args.workload]()
-    layers = [Linear(mx, w, L, dev, args.quantiser) for L in w.layers]
+    chosen = w.layers if args.linears == "all" else [L for L in w.layers if L.name in args.linears.split(",")]
+    if not chosen:
+        raise SystemExit(f"bench: no linear named {args.linears!r} in {w.name}")
+    layers = [Linear(mx, w, L, dev, args.quantiser) for L in chosen]
     calls = [c for L in layers for c in L.launches()]
     step_flops = 3 * sum(L.flops_per_pass() for L in layers)
     quant_bytes = sum(L.quant_bytes() for L in layers)
@@ -274,7 +311,10 @@ def run_ours(args, rank, world, local_rank):
         "fraction_of_fp8_peak": round(value / world / fp8_peak, 4),
         "roofline": {"kernel": "grouped_gemm_kernel (fwd+dgrad+wgrad launches)", "bound": "tensor",
                      "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(gemm_tflops / fp8_peak, 4), "traffic": None,
+                     "frac": round(gemm_tflops / fp8_peak, 4), "traffic": gemm_traffic(),
+                     "traffic_source": "mean DRAM read+write bytes per launch over the gate/up linear's fwd, dgrad "
+                                       "and wgrad launches, ncu (profiles/grouped_gemm_ds-v3-16b_gate_up.md); null "
+                                       "if the kernel sources changed since",
                      "peak_source": f"{pk['src']} bf16 burst x {FP8_OVER_BF16} (nominal FP8/BF16)",
                      "launches_timed": gemm_launches},
         "quantiser": {"achieved_gbs": round(quant_gbs, 1), "peak_gbs": pk["hbm_gbs"],
@@ -285,9 +325,12 @@ def run_ours(args, rank, world, local_rank):
     }
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(w, budget_s=12.0)
-    out["e2e"] = e2e(args, mx, w, layers, dev, world)
-    out["quantising_epilogue"] = quantising_epilogue(mx, layers[0])
-    out["moe_dispatch"] = moe_dispatch(mx, args, pk["hbm_gbs"])
+    if args.linears != "all":
+        out["config"]["linears_timed"] = [L.name for L in layers]
+    if not args.no_extras:
+        out["e2e"] = e2e(args, mx, w, layers, dev, world)
+        out["quantising_epilogue"] = quantising_epilogue(mx, layers[0])
+        out["moe_dispatch"] = moe_dispatch(mx, args, pk["hbm_gbs"])
     return out
 
 
