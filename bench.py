@@ -61,7 +61,7 @@ def parse():
 
 
 GEMM_PROFILE = os.path.join(ROOT, "profiles", "grouped_gemm_ds-v3-16b_gate_up.md")
-GEMM_SOURCES = ("grouped_gemm.cu", "ptx.cuh", "codec.cuh", "launch.h")
+GEMM_SOURCES = ("grouped_gemm.cu", "ptx.cuh", "codec.cuh", "launch.h", "tmap.cu")
 
 
 def gemm_sources_sha256() -> str:

@@ -696,37 +696,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 }
 
 // ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-// 2D map over a row-major matrix [rows, cols] of `esize`-byte elements with
-// row stride `ld` elements; box = box_cols x box_rows; zero fill outside.
-bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, int esize, int64_t rows, int64_t cols,
-              int64_t ld, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn || rows < 1 || cols < 1) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * esize)};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 struct DeviceSetup {
   bool done[2][2][2] = {};    // [CG - 1][KS - 1][QE]
   int num_sms = 0;
@@ -808,20 +777,20 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   const int64_t out_cols = a.mode == kFwd ? a.N : a.K;
   CUtensorMap maps[5];
   const bool ok =
-      make_map(&maps[0], a.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.a_rows, a.a_cols, a.lda, BK, BM,
+      make_tensor_map(&maps[0], a.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.a_rows, a.a_cols, a.lda, BK, BM,
                CU_TENSOR_MAP_SWIZZLE_128B) &&
-      make_map(&maps[1], a.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b_rows, a.b_cols, a.ldb, BK, BN / cg,
+      make_tensor_map(&maps[1], a.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b_rows, a.b_cols, a.ldb, BK, BN / cg,
                CU_TENSOR_MAP_SWIZZLE_128B) &&
-      make_map(&maps[2], a.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfa_atoms * 4, 128, 128, 128, 4 * ks,
+      make_tensor_map(&maps[2], a.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfa_atoms * 4, 128, 128, 128, 4 * ks,
                CU_TENSOR_MAP_SWIZZLE_NONE) &&
-      make_map(&maps[3], a.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfb_atoms * 4, 128, 128, 128, 4 * ks,
+      make_tensor_map(&maps[3], a.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfb_atoms * 4, 128, 128, 128, 4 * ks,
                CU_TENSOR_MAP_SWIZZLE_NONE) &&
       (a.out != nullptr
-           ? make_map(&maps[4], a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out_rows, out_cols, out_cols, 64, 32,
+           ? make_tensor_map(&maps[4], a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out_rows, out_cols, out_cols, 64, 32,
                       CU_TENSOR_MAP_SWIZZLE_128B)
            // no bf16 output (quantising epilogue only): a placeholder map over
            // the status word that the kernel never uses
-           : make_map(&maps[4], a.status, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 1, 64, 64, 64, 32,
+           : make_tensor_map(&maps[4], a.status, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 1, 64, 64, 64, 32,
                       CU_TENSOR_MAP_SWIZZLE_128B));
   if (!ok) {
     if (detail) *detail = "cuTensorMapEncodeTiled failed";

@@ -1,9 +1,16 @@
 // launch.h -- internal launchers behind the C ABI (arguments already checked).
 #pragma once
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace mxf8 {
+
+// 2D TMA map over a row-major matrix [rows, cols] of `esize`-byte elements
+// with row stride `ld` elements; box = box_cols x box_rows; zero fill
+// outside the matrix.  False if the driver rejects it.
+bool make_tensor_map(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, int esize, int64_t rows,
+                     int64_t cols, int64_t ld, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
 
 cudaError_t launch_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols,
                                     const int32_t* offs, int32_t G, uint8_t* q, uint8_t* sf,
