@@ -74,6 +74,22 @@ def lib():
         L.orc_bf16_from_double.restype = ctypes.c_uint16
         L.orc_bf16_from_double.argtypes = [ctypes.c_double]
         L.orc_bf16_from_double_array.argtypes = [_vp, _i64, _vp]
+        L.orc_e2m1_decode.restype = ctypes.c_double
+        L.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e2m1_encode.restype = ctypes.c_uint8
+        L.orc_e2m1_encode.argtypes = [ctypes.c_double]
+        L.orc_e2m1_encode_array.argtypes = [_vp, _i64, _vp]
+        L.orc_nvfp4_tensor_scale.restype = ctypes.c_float
+        L.orc_nvfp4_tensor_scale.argtypes = [ctypes.c_float]
+        L.orc_nvfp4_quantize_block.argtypes = [_vp, ctypes.c_int, _i64, ctypes.c_float, _vp, _i64, _vp]
+        L.orc_nvfp4_colwise_pitch.restype = _i64
+        L.orc_nvfp4_colwise_pitch.argtypes = [_i64, _i32]
+        L.orc_nvfp4_colwise_ld.restype = _i64
+        L.orc_nvfp4_colwise_ld.argtypes = [_i64, _i32]
+        for name in ("orc_nvfp4_quantize_rowwise", "orc_nvfp4_quantize_colwise"):
+            getattr(L, name).argtypes = [_vp, _i64, _i64, _vp, _i32, ctypes.c_float, _vp, _vp]
+        for name in ("orc_nvfp4_dequantize_rowwise", "orc_nvfp4_dequantize_colwise"):
+            getattr(L, name).argtypes = [_vp, _vp, _i64, _i64, _vp, _i32, ctypes.c_float, _vp]
         _LIB = L
     return _LIB
 
@@ -379,3 +395,103 @@ def moe_combine(yp, inv, w) -> np.ndarray:
     y = np.zeros((T, C), dtype=np.uint16)
     _check(lib().orc_moe_combine(_p(ypu), rows, C, _p(inv), _p(w), T, k, _p(y)), "moe_combine")
     return y
+
+
+# ---------------------------------------------------------------- NVFP4
+def e2m1_decode(nibbles) -> np.ndarray:
+    n = np.asarray(nibbles, dtype=np.uint8).reshape(-1)
+    return np.array([lib().orc_e2m1_decode(int(b)) for b in n], dtype=np.float64)
+
+
+def e2m1_encode(v) -> np.ndarray:
+    a = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
+    out = np.zeros(a.shape, dtype=np.uint8)
+    lib().orc_e2m1_encode_array(_p(a), a.size, _p(out))
+    return out
+
+
+def nvfp4_tensor_scale(amax: float) -> np.float32:
+    return np.float32(lib().orc_nvfp4_tensor_scale(float(np.float32(amax))))
+
+
+def nvfp4_amax(x) -> np.float32:
+    """Largest |x| of a bf16 tensor, as fp32 (exact)."""
+    xu = _u16(x)
+    return np.float32(np.abs((xu.astype(np.uint32) << 16).view(np.float32)).max()) if xu.size else np.float32(0)
+
+
+def nvfp4_quantize_block(x_u16, S) -> tuple[np.ndarray, int]:
+    xu = np.ascontiguousarray(np.asarray(x_u16, dtype=np.uint16))
+    codes = np.zeros(xu.size, dtype=np.uint8)
+    sb = np.zeros(1, dtype=np.uint8)
+    lib().orc_nvfp4_quantize_block(_p(xu), xu.size, 1, float(S), _p(codes), 1, _p(sb))
+    return codes, int(sb[0])
+
+
+def nvfp4_rowwise_pitch(C: int) -> int:
+    return (C + 63) // 64
+
+
+def nvfp4_colwise_pitch(R: int, G: int) -> int:
+    return lib().orc_nvfp4_colwise_pitch(R, G)
+
+
+def nvfp4_colwise_ld(R: int, G: int) -> int:
+    """Row length of the colwise codes in ELEMENTS (bytes = half)."""
+    return lib().orc_nvfp4_colwise_ld(R, G)
+
+
+def nvfp4_rowwise_scale_bytes(R: int, C: int, G: int) -> int:
+    return _nb128(R, G) * nvfp4_rowwise_pitch(C) * 512
+
+
+def nvfp4_colwise_scale_bytes(R: int, C: int, G: int) -> int:
+    return ((C + 127) // 128) * max(nvfp4_colwise_pitch(R, G), 0) * 512
+
+
+def nvfp4_group_blocks(offs, R):
+    """(RB_G, RB64_G, P_G): 128-row blocks, 64-row blocks and 32-padded rows over all groups."""
+    m = np.diff(np.asarray(offs if offs is not None else [0, R], dtype=np.int64))
+    return int(((m + 127) // 128).sum()), int(((m + 63) // 64).sum()), int(((m + 31) // 32 * 32).sum())
+
+
+def nvfp4_quantize_rowwise(x, S, offs=None):
+    """x: bf16 [R, C] -> (q uint8 [R, C/2] packed, sf uint8 atoms)."""
+    xu = _u16(x)
+    R, C = xu.shape
+    o, G = _offs(offs, R)
+    q = np.zeros((R, C // 2), dtype=np.uint8)
+    sf = np.zeros(max(nvfp4_rowwise_scale_bytes(R, C, G), 512), dtype=np.uint8)
+    _check(lib().orc_nvfp4_quantize_rowwise(_p(xu), R, C, _p(o), G, float(S), _p(q), _p(sf)), "nvfp4_quantize_rowwise")
+    return q, sf
+
+
+def nvfp4_quantize_colwise(x, S, offs=None):
+    """x: bf16 [R, C] -> (qT uint8 [C, ld/2] packed, sfT uint8 atoms)."""
+    xu = _u16(x)
+    R, C = xu.shape
+    o, G = _offs(offs, R)
+    qT = np.zeros((C, nvfp4_colwise_ld(R, G) // 2), dtype=np.uint8)
+    sf = np.zeros(max(nvfp4_colwise_scale_bytes(R, C, G), 512), dtype=np.uint8)
+    _check(lib().orc_nvfp4_quantize_colwise(_p(xu), R, C, _p(o), G, float(S), _p(qT), _p(sf)), "nvfp4_quantize_colwise")
+    return qT, sf
+
+
+def nvfp4_dequantize_rowwise(q, sf, S, offs=None) -> np.ndarray:
+    q = np.ascontiguousarray(q)
+    R, C = q.shape[0], q.shape[1] * 2
+    o, G = _offs(offs, R)
+    out = np.zeros((R, C), dtype=np.float64)
+    _check(lib().orc_nvfp4_dequantize_rowwise(_p(q), _p(np.ascontiguousarray(sf)), R, C, _p(o), G, float(S), _p(out)),
+           "nvfp4_dequantize_rowwise")
+    return out
+
+
+def nvfp4_dequantize_colwise(qT, sf, R: int, S, offs=None) -> np.ndarray:
+    qT = np.ascontiguousarray(qT)
+    C = qT.shape[0]
+    o, G = _offs(offs, R)
+    out = np.zeros((R, C), dtype=np.float64)
+    _check(lib().orc_nvfp4_dequantize_colwise(_p(qT), _p(np.ascontiguousarray(sf)), R, C, _p(o), G, float(S),
+                                              _p(out)), "nvfp4_dequantize_colwise")
+    return out

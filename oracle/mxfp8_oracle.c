@@ -710,3 +710,215 @@ void orc_bf16_from_double_array(const double* v, int64_t n, uint16_t* out)
     int64_t i;
     for (i = 0; i < n; ++i) out[i] = orc_bf16_from_double(v[i]);
 }
+
+/* ------------------------------------------------------------------ */
+/* NVFP4: 4-bit E2M1 elements, 16-element blocks with E4M3 scales and   */
+/* one fp32 scale per tensor                                             */
+/* ------------------------------------------------------------------ */
+/* The pages name NVFP4 only as the format NVIDIA's MoE training adds next
+ * (iitak.ru, "NVIDIA в 10 раз ускорила обучение моделей-«смесей экспертов»
+ * на JAX", closing paragraph).  Its rules here are NVIDIA's public NVFP4
+ * definition, read plainly:
+ *   - E2M1 element: sign, 2 exponent bits (bias 1), 1 mantissa bit; values
+ *     0, 0.5, 1, 1.5, 2, 3, 4, 6; round to nearest even, saturate at 6.
+ *   - tensor scale S = (448 * 6) / amax(tensor) in fp32 (1 when amax = 0);
+ *   - a block of 16 shares the E4M3 scale sf = E4M3(amax_b * S / 6), and an
+ *     element is E2M1((x * S) / sf); the fp32 operations are rounded to
+ *     nearest in exactly this order (the decision that picks each code is
+ *     taken in fp32, as the GPU takes it); sf = 0 gives zero codes.
+ *   - value = code * sf / S. */
+double orc_e2m1_decode(uint8_t nib)
+{
+    int s = (nib >> 3) & 1, e = (nib >> 1) & 3, m = nib & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -v : v;
+}
+
+uint8_t orc_e2m1_encode(double v)
+{
+    uint8_t sign = signbit(v) ? 8 : 0;
+    double a = fabs(v), q, n, fl, rem, k, r;
+    int ex;
+    if (a >= 6.0) return (uint8_t)(sign | 7);          /* saturate (and 6 itself) */
+    if (a < 1.0) q = 0.5;                              /* subnormal spacing, and [0.5, 1) */
+    else { frexp(a, &ex); q = ldexp(1.0, (ex - 1) - 1); }   /* 2^(floor(log2 a) - 1) */
+    n = a / q;
+    fl = floor(n);
+    rem = n - fl;
+    if (rem > 0.5) k = fl + 1.0;
+    else if (rem < 0.5) k = fl;
+    else k = (fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;
+    r = k * q;
+    if (r >= 6.0) return (uint8_t)(sign | 7);
+    if (r == 0.0) return sign;
+    if (r < 1.0) return (uint8_t)(sign | 1);           /* 0.5 */
+    frexp(r, &ex);
+    {
+        int e = ex;                                    /* r in [2^(ex-1), 2^ex): biased exponent ex */
+        int m = (r / ldexp(1.0, ex - 1) > 1.0) ? 1 : 0;
+        return (uint8_t)(sign | (e << 1) | m);
+    }
+}
+
+float orc_nvfp4_tensor_scale(float amax)
+{
+    return amax == 0.0f ? 1.0f : 2688.0f / amax;
+}
+
+/* One block of n <= 16 bf16 elements (stride apart): the E4M3 scale byte and
+ * one E2M1 nibble per element (low 4 bits of codes[i * code_stride]). */
+void orc_nvfp4_quantize_block(const uint16_t* x, int n, int64_t stride, float S, uint8_t* codes,
+                              int64_t code_stride, uint8_t* scale_byte)
+{
+    float amax = 0.0f, t, u, r;
+    int i;
+    uint8_t sf;
+    for (i = 0; i < n; ++i) {
+        float a = fabsf((float)orc_bf16_to_double(x[i * stride]));
+        if (a > amax) amax = a;
+    }
+    t = amax * S;
+    u = t / 6.0f;
+    sf = orc_e4m3_encode((double)u);
+    r = (float)orc_e4m3_decode(sf);
+    *scale_byte = sf;
+    for (i = 0; i < n; ++i) {
+        if (r == 0.0f) {
+            codes[i * code_stride] = 0;
+        } else {
+            float w = ((float)orc_bf16_to_double(x[i * stride]) * S) / r;
+            codes[i * code_stride] = orc_e2m1_encode((double)w);
+        }
+    }
+}
+
+static int64_t nv_pitch_row(int64_t C) { return cdiv(C, 64); }
+
+int64_t orc_nvfp4_colwise_pitch(int64_t R, int32_t G) { return R == 0 ? 0 : cdiv(R, 64) + G - 1; }
+
+int64_t orc_nvfp4_colwise_ld(int64_t R, int32_t G)
+{
+    int64_t ld = rup(rup(R, 32) + 32 * (int64_t)(G - 1), 256);
+    return ld < 256 ? 256 : ld;                         /* elements; bytes = ld / 2 */
+}
+
+/* Rowwise NVFP4 of x [R, C] (C % 64 == 0) with groups offs: packed codes
+ * q [R, C/2] (element c in the low nibble of byte c/2 when c is even),
+ * scales in 512-byte atoms of 128 rows x 4 blocks, rows of group g padded to
+ * a multiple of 128 as for MXFP8, pitch ceil(C/64). */
+int orc_nvfp4_quantize_rowwise(const uint16_t* x, int64_t R, int64_t C, const int32_t* offs, int32_t G,
+                               float S, uint8_t* q, uint8_t* sf)
+{
+    int64_t* RB = (int64_t*)calloc((size_t)G + 1, sizeof(int64_t));
+    int64_t* P = (int64_t*)calloc((size_t)G + 1, sizeof(int64_t));
+    int64_t pitch = nv_pitch_row(C);
+    int32_t g;
+    if (orc_check_offsets(offs, G, R) != 0 || C % 64 != 0) { free(RB); free(P); return -1; }
+    group_prefixes(offs, G, R, RB, P);
+    for (g = 0; g < G; ++g) {
+        int64_t lo = offs[g], hi = offs[g + 1], r;
+        for (r = lo; r < hi; ++r) {
+            int64_t pr = 128 * RB[g] + (r - lo), j;
+            for (j = 0; j < C / 16; ++j) {
+                uint8_t nib[16], sb;
+                int i;
+                orc_nvfp4_quantize_block(x + r * C + 16 * j, 16, 1, S, nib, 1, &sb);
+                for (i = 0; i < 16; i += 2)
+                    q[r * (C / 2) + 8 * j + i / 2] = (uint8_t)(nib[i] | (nib[i + 1] << 4));
+                sf[orc_sf_offset(pr, j, pitch)] = sb;
+            }
+        }
+    }
+    free(RB); free(P);
+    return 0;
+}
+
+/* Colwise NVFP4: blocks of 16 rows restarting at every group offset (a
+ * group's last block may be short), codes transposed and packed along rows:
+ * qT [C, ld/2] bytes, element (offs[g] + t, c) at nibble P_g + t of row c
+ * (P_g = sum over h < g of round_up(m_h, 32); pad nibbles 0).  Scales
+ * S^T[c, 4*RB64_g + t/16], RB64_g = sum over h < g of ceil(m_h/64), pitch
+ * orc_nvfp4_colwise_pitch(R, G). */
+int orc_nvfp4_quantize_colwise(const uint16_t* x, int64_t R, int64_t C, const int32_t* offs, int32_t G,
+                               float S, uint8_t* qT, uint8_t* sfT)
+{
+    int64_t ld = orc_nvfp4_colwise_ld(R, G), pitch = orc_nvfp4_colwise_pitch(R, G);
+    int64_t p0 = 0, rb64 = 0;
+    int32_t g;
+    if (orc_check_offsets(offs, G, R) != 0 || C % 64 != 0) return -1;
+    for (g = 0; g < G; ++g) {
+        int64_t lo = offs[g], m = offs[g + 1] - offs[g], c;
+        for (c = 0; c < C; ++c) {
+            int64_t b;
+            for (b = 0; b < cdiv(m, 16); ++b) {
+                int64_t n = m - 16 * b < 16 ? m - 16 * b : 16, i;
+                uint8_t nib[16], sb;
+                orc_nvfp4_quantize_block(x + (lo + 16 * b) * C + c, (int)n, C, S, nib, 1, &sb);
+                for (i = 0; i < n; ++i) {
+                    int64_t col = p0 + 16 * b + i;
+                    uint8_t* dst = qT + c * (ld / 2) + col / 2;
+                    *dst = (uint8_t)((col & 1) ? ((*dst & 0x0F) | (nib[i] << 4)) : ((*dst & 0xF0) | nib[i]));
+                }
+                sfT[orc_sf_offset(c, 4 * rb64 + b, pitch)] = sb;
+            }
+        }
+        p0 += rup(m, 32);
+        rb64 += cdiv(m, 64);
+    }
+    return 0;
+}
+
+/* Dequantisation back to fp64 (value = code * sf / S), same layouts. */
+int orc_nvfp4_dequantize_rowwise(const uint8_t* q, const uint8_t* sf, int64_t R, int64_t C, const int32_t* offs,
+                                 int32_t G, float S, double* out)
+{
+    int64_t* RB = (int64_t*)calloc((size_t)G + 1, sizeof(int64_t));
+    int64_t* P = (int64_t*)calloc((size_t)G + 1, sizeof(int64_t));
+    int64_t pitch = nv_pitch_row(C);
+    int32_t g;
+    if (orc_check_offsets(offs, G, R) != 0) { free(RB); free(P); return -1; }
+    group_prefixes(offs, G, R, RB, P);
+    for (g = 0; g < G; ++g) {
+        int64_t r;
+        for (r = offs[g]; r < offs[g + 1]; ++r) {
+            int64_t pr = 128 * RB[g] + (r - offs[g]), c;
+            for (c = 0; c < C; ++c) {
+                uint8_t byte = q[r * (C / 2) + c / 2];
+                uint8_t nib = (c & 1) ? (byte >> 4) : (byte & 0xF);
+                double s = orc_e4m3_decode(sf[orc_sf_offset(pr, c / 16, pitch)]);
+                out[r * C + c] = orc_e2m1_decode(nib) * s / (double)S;
+            }
+        }
+    }
+    free(RB); free(P);
+    return 0;
+}
+
+int orc_nvfp4_dequantize_colwise(const uint8_t* qT, const uint8_t* sfT, int64_t R, int64_t C,
+                                 const int32_t* offs, int32_t G, float S, double* out)
+{
+    int64_t ld = orc_nvfp4_colwise_ld(R, G), pitch = orc_nvfp4_colwise_pitch(R, G);
+    int64_t p0 = 0, rb64 = 0;
+    int32_t g;
+    if (orc_check_offsets(offs, G, R) != 0) return -1;
+    for (g = 0; g < G; ++g) {
+        int64_t lo = offs[g], m = offs[g + 1] - offs[g], t, c;
+        for (t = 0; t < m; ++t)
+            for (c = 0; c < C; ++c) {
+                int64_t col = p0 + t;
+                uint8_t byte = qT[c * (ld / 2) + col / 2];
+                uint8_t nib = (col & 1) ? (byte >> 4) : (byte & 0xF);
+                double s = orc_e4m3_decode(sfT[orc_sf_offset(c, 4 * rb64 + t / 16, pitch)]);
+                out[(lo + t) * C + c] = orc_e2m1_decode(nib) * s / (double)S;
+            }
+        p0 += rup(m, 32);
+        rb64 += cdiv(m, 64);
+    }
+    return 0;
+}
+
+void orc_e2m1_encode_array(const double* v, int64_t n, uint8_t* out)
+{
+    int64_t i;
+    for (i = 0; i < n; ++i) out[i] = orc_e2m1_encode(v[i]);
+}
