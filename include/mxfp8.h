@@ -311,6 +311,50 @@ MXF8_API mxf8_status mxfp8_moe_combine(const uint16_t* yp, int64_t rows, int64_t
                                        const float* w, int64_t num_tokens, int32_t top_k, uint16_t* y,
                                        void* stream);
 
+/* ---------------------------------------------------------------- NVFP4 */
+/* NVFP4 quantisation: 4-bit E2M1 elements in blocks of 16 that share an E4M3
+ * scale, plus one fp32 scale per tensor.  The pages name NVFP4 only as the
+ * format NVIDIA's MoE training adds next (iitak.ru, "NVIDIA в 10 раз
+ * ускорила обучение моделей-«смесей экспертов» на JAX", closing paragraph);
+ * the rules are NVIDIA's public NVFP4 definition, read plainly, with every
+ * fp32 operation rounded to nearest in this order:
+ *   S  = 2688 / amax(tensor)         (2688 = 448 * 6; S = 1 when amax = 0)
+ *   sf = E4M3((amax_block * S) / 6)  (nearest even, saturating at 448)
+ *   q  = E2M1((x * S) / sf)          (nearest even, saturating at +-6; 0 when sf = 0)
+ *   x ~ q * sf / S
+ * Non-finite inputs are outside the contract.
+ * Layouts (as MXFP8, with 16-element blocks and packed codes):
+ *   codes hold two elements per byte, element 2i in the low nibble of byte i;
+ *   a 512-byte scale atom covers 128 rows x 4 blocks = 64 elements, byte
+ *   (row%32)*16 + ((row%128)/32)*4 + blk%4;
+ *   rowwise: q [rows, cols/2]; scale rows of group g start at a multiple of
+ *     128 (as MXFP8); pitch ceil(cols/64) atoms;
+ *   colwise: qT [cols, ldT/2] bytes, ldT = mxfp8_nvfp4_colwise_ld(rows, G)
+ *     elements; element (d_offs[g] + t, c) at nibble P_g + t of row c,
+ *     P_g = sum over h < g of round_up(m_h, 32), pad nibbles 0; blocks of 16
+ *     rows restart at every group offset; scales S^T[c, 4*Q_g + t/16] with
+ *     Q_g = sum over h < g of ceil(m_h/64), pitch mxfp8_nvfp4_colwise_pitch. */
+MXF8_API int64_t mxfp8_nvfp4_rowwise_scale_bytes(int64_t rows, int64_t cols, int32_t num_groups);
+MXF8_API int64_t mxfp8_nvfp4_colwise_pitch(int64_t rows, int32_t num_groups);
+MXF8_API int64_t mxfp8_nvfp4_colwise_scale_bytes(int64_t rows, int64_t cols, int32_t num_groups);
+MXF8_API int64_t mxfp8_nvfp4_colwise_ld(int64_t rows, int32_t num_groups);
+
+/* amax (device fp32, out) = largest |x| over n bf16 elements (x 16-byte
+ * aligned; n = 0 gives 0).  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, CUDA. */
+MXF8_API mxf8_status mxfp8_nvfp4_amax(const uint16_t* x, int64_t n, float* amax, void* stream);
+
+/* Rowwise / colwise NVFP4 of x [rows, cols] (cols % 64 == 0) with groups
+ * d_offs, the tensor scale taken from the device amax written by
+ * mxfp8_nvfp4_amax.  Buffer sizes from the functions above; errors as the
+ * MXFP8 quantisers. */
+MXF8_API mxf8_status mxfp8_nvfp4_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols,
+                                                  const int32_t* d_offs, int32_t num_groups, const float* amax,
+                                                  uint8_t* q, uint8_t* scales, int64_t scale_bytes, void* stream);
+MXF8_API mxf8_status mxfp8_nvfp4_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols,
+                                                  const int32_t* d_offs, int32_t num_groups, const float* amax,
+                                                  uint8_t* qT, int64_t ldT, uint8_t* scalesT, int64_t scale_bytes,
+                                                  void* stream);
+
 /* ---------------------------------------------------------------- status */
 
 /* Synchronises `stream`, then stores the device status of the last GEMM that

@@ -37,7 +37,9 @@ EXPORTED = ("mxfp8_rowwise_scale_bytes", "mxfp8_colwise_pitch", "mxfp8_colwise_s
             "mxfp8_get_status", "mxfp8_status_string", "mxfp8_last_cuda_error", "mxfp8_device_supported",
             "mxfp8_grouped_gemm_fwd_noalloc", "mxfp8_quantize_dual", "mxfp8_grouped_gemm_fwd_quant",
             "mxfp8_grouped_gemm_dgrad_quant", "mxfp8_moe_plan_workspace_bytes", "mxfp8_moe_plan",
-            "mxfp8_permute_quantize_dual", "mxfp8_moe_combine")
+            "mxfp8_permute_quantize_dual", "mxfp8_moe_combine", "mxfp8_nvfp4_rowwise_scale_bytes",
+            "mxfp8_nvfp4_colwise_pitch", "mxfp8_nvfp4_colwise_scale_bytes", "mxfp8_nvfp4_colwise_ld",
+            "mxfp8_nvfp4_amax", "mxfp8_nvfp4_quantize_rowwise", "mxfp8_nvfp4_quantize_colwise")
 
 
 class MXFP8Error(RuntimeError):
@@ -88,6 +90,18 @@ def lib() -> ctypes.CDLL:
                                                   _vp, _i64, _vp]
         L.mxfp8_moe_combine.restype = _i32
         L.mxfp8_moe_combine.argtypes = [_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp]
+        for n in ("mxfp8_nvfp4_rowwise_scale_bytes", "mxfp8_nvfp4_colwise_scale_bytes"):
+            getattr(L, n).restype = _i64
+            getattr(L, n).argtypes = [_i64, _i64, _i32]
+        for n in ("mxfp8_nvfp4_colwise_pitch", "mxfp8_nvfp4_colwise_ld"):
+            getattr(L, n).restype = _i64
+            getattr(L, n).argtypes = [_i64, _i32]
+        L.mxfp8_nvfp4_amax.restype = _i32
+        L.mxfp8_nvfp4_amax.argtypes = [_vp, _i64, _vp, _vp]
+        L.mxfp8_nvfp4_quantize_rowwise.restype = _i32
+        L.mxfp8_nvfp4_quantize_rowwise.argtypes = [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _i64, _vp]
+        L.mxfp8_nvfp4_quantize_colwise.restype = _i32
+        L.mxfp8_nvfp4_quantize_colwise.argtypes = [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _i64, _vp, _i64, _vp]
         L.mxfp8_grouped_gemm_fwd_noalloc.restype = _i32
         L.mxfp8_grouped_gemm_fwd_noalloc.argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp,
                                                      ctypes.POINTER(_i32), _vp]
@@ -342,3 +356,36 @@ def mxfp8_moe_combine(yp: torch.Tensor, inv: torch.Tensor, w: torch.Tensor, out=
     _check(lib().mxfp8_moe_combine(_ptr(yp) if rows else None, rows, C, _ptr(inv), _ptr(w), T, k, _ptr(out),
                                    _stream(stream)), "mxfp8_moe_combine")
     return out
+
+
+# ------------------------------------------------------------------ NVFP4
+def mxfp8_nvfp4_amax(x: torch.Tensor, amax=None, stream=None) -> torch.Tensor:
+    """Largest |x| of a bf16 tensor -> fp32 device scalar (shape [1])."""
+    assert x.dtype == torch.bfloat16
+    amax = amax if amax is not None else torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(lib().mxfp8_nvfp4_amax(_ptr(x) if x.numel() else None, x.numel(), _ptr(amax), _stream(stream)),
+           "mxfp8_nvfp4_amax")
+    return amax
+
+
+def mxfp8_nvfp4_quantize_rowwise(x, amax, offs=None, q=None, scales=None, stream=None):
+    """x: bf16 [rows, cols] -> (q uint8 [rows, cols/2], scales); amax from mxfp8_nvfp4_amax."""
+    R, C = x.shape
+    G = _groups(offs)
+    q = q if q is not None else torch.empty((R, C // 2), dtype=torch.uint8, device=x.device)
+    scales = scales if scales is not None else _u8(lib().mxfp8_nvfp4_rowwise_scale_bytes(R, C, G), x.device)
+    _check(lib().mxfp8_nvfp4_quantize_rowwise(_ptr(x), R, C, _ptr(offs), G, _ptr(amax), _ptr(q), _ptr(scales),
+                                              scales.numel(), _stream(stream)), "mxfp8_nvfp4_quantize_rowwise")
+    return q, scales
+
+
+def mxfp8_nvfp4_quantize_colwise(x, amax, offs=None, qT=None, scales=None, stream=None):
+    """x: bf16 [rows, cols] -> (qT uint8 [cols, ld/2], scales); ld = mxfp8_nvfp4_colwise_ld(rows, G) elements."""
+    R, C = x.shape
+    G = _groups(offs)
+    ld = lib().mxfp8_nvfp4_colwise_ld(R, G)
+    qT = qT if qT is not None else torch.empty((C, ld // 2), dtype=torch.uint8, device=x.device)
+    scales = scales if scales is not None else _u8(lib().mxfp8_nvfp4_colwise_scale_bytes(R, C, G), x.device)
+    _check(lib().mxfp8_nvfp4_quantize_colwise(_ptr(x), R, C, _ptr(offs), G, _ptr(amax), _ptr(qT), ld, _ptr(scales),
+                                              scales.numel(), _stream(stream)), "mxfp8_nvfp4_quantize_colwise")
+    return qT, scales

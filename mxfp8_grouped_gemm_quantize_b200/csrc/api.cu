@@ -367,6 +367,63 @@ mxf8_status mxfp8_moe_combine(const uint16_t* yp, int64_t rows, int64_t cols, co
   return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "moe_combine launch");
 }
 
+int64_t mxfp8_nvfp4_rowwise_scale_bytes(int64_t rows, int64_t cols, int32_t num_groups) {
+  if (rows < 0 || cols <= 0 || num_groups < 1) return 0;
+  return blocks128_bound(rows, num_groups) * cdiv(cols, 64) * 512;
+}
+
+int64_t mxfp8_nvfp4_colwise_pitch(int64_t rows, int32_t num_groups) {
+  if (rows <= 0 || num_groups < 1) return 0;
+  return cdiv(rows, 64) + num_groups - 1;
+}
+
+int64_t mxfp8_nvfp4_colwise_scale_bytes(int64_t rows, int64_t cols, int32_t num_groups) {
+  if (rows < 0 || cols <= 0 || num_groups < 1) return 0;
+  return cdiv(cols, 128) * mxfp8_nvfp4_colwise_pitch(rows, num_groups) * 512;
+}
+
+int64_t mxfp8_nvfp4_colwise_ld(int64_t rows, int32_t num_groups) {
+  if (rows < 0 || num_groups < 1) return 0;
+  const int64_t ld = round_up(round_up(rows, 32) + 32 * int64_t(num_groups - 1), 256);
+  return ld < 256 ? 256 : ld;
+}
+
+mxf8_status mxfp8_nvfp4_amax(const uint16_t* x, int64_t n, float* amax, void* stream) {
+  if (n < 0 || !amax || (n > 0 && !x)) return MXF8_ERR_INVALID_ARG;
+  if (!aligned16(x)) return MXF8_ERR_ALIGNMENT;
+  mxf8_status s = check_device();
+  if (s != MXF8_OK) return s;
+  cudaError_t e = mxf8::launch_nvfp4_amax(x, n, amax, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "nvfp4_amax launch");
+}
+
+mxf8_status mxfp8_nvfp4_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols, const int32_t* d_offs,
+                                         int32_t num_groups, const float* amax, uint8_t* q, uint8_t* scales,
+                                         int64_t scale_bytes, void* stream) {
+  if (!amax || cols % 64 != 0) return MXF8_ERR_INVALID_ARG;
+  mxf8_status s = check_quant_args(x, rows, cols, num_groups, q, scales, scale_bytes,
+                                   mxfp8_nvfp4_rowwise_scale_bytes(rows, cols, num_groups));
+  if (s != MXF8_OK) return s;
+  if ((s = check_device()) != MXF8_OK) return s;
+  cudaError_t e = mxf8::launch_nvfp4_rowwise(x, rows, cols, d_offs, num_groups, amax, q, scales,
+                                             static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "nvfp4_rowwise launch");
+}
+
+mxf8_status mxfp8_nvfp4_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols, const int32_t* d_offs,
+                                         int32_t num_groups, const float* amax, uint8_t* qT, int64_t ldT,
+                                         uint8_t* scalesT, int64_t scale_bytes, void* stream) {
+  if (!amax || cols % 64 != 0) return MXF8_ERR_INVALID_ARG;
+  mxf8_status s = check_quant_args(x, rows, cols, num_groups, qT, scalesT, scale_bytes,
+                                   mxfp8_nvfp4_colwise_scale_bytes(rows, cols, num_groups));
+  if (s != MXF8_OK) return s;
+  if (ldT != mxfp8_nvfp4_colwise_ld(rows, num_groups)) return MXF8_ERR_INVALID_ARG;
+  if ((s = check_device()) != MXF8_OK) return s;
+  cudaError_t e = mxf8::launch_nvfp4_colwise(x, rows, cols, d_offs, num_groups, amax, qT, ldT, scalesT,
+                                             static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "nvfp4_colwise launch");
+}
+
 mxf8_status mxfp8_get_status(const void* work, void* stream, int32_t* device_status) {
   if (!work || !device_status) return MXF8_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

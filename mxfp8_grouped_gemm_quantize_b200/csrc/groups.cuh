@@ -6,6 +6,7 @@
 // (m_g = offs'[g+1] - offs'[g]):
 //   RB_g = sum over h < g of ceil(m_h / 128)   (128-row blocks; scale atoms)
 //   P_g  = sum over h < g of round_up(m_h, 32) (32-padded rows; colwise codes)
+//   Q_g  = sum over h < g of ceil(m_h / 64)    (64-row blocks; NVFP4 colwise scale atoms)
 #pragma once
 #include <cstdint>
 
@@ -17,6 +18,7 @@ struct GroupBlock {
   int64_t m;       // rows in the group
   int64_t rb;      // RB_g
   int64_t p;       // P_g
+  int64_t q;       // Q_g
 };
 
 __device__ __forceinline__ int64_t clamp_off(const int32_t* offs, int32_t h, int64_t rows) {
@@ -30,7 +32,7 @@ __device__ __forceinline__ GroupBlock warp_find_block(const int32_t* offs, int32
                                                       int64_t pb) {
   const int lane = threadIdx.x & 31;
   int64_t o_prev = clamp_off(offs, 0, rows);
-  int64_t carry_rb = 0, carry_p = 0;
+  int64_t carry_rb = 0, carry_p = 0, carry_q = 0;
   for (int32_t base = 0; base < G; base += 32) {
     const int32_t h = base + lane;
     int64_t v = (h < G) ? clamp_off(offs, h + 1, rows) : 0;
@@ -43,15 +45,16 @@ __device__ __forceinline__ GroupBlock warp_find_block(const int32_t* offs, int32
     int64_t lo = __shfl_up_sync(0xffffffffu, hi, 1);
     if (lane == 0) lo = o_prev;                           // offs'[h]
     const int64_t m = (h < G) ? hi - lo : 0;
-    const int64_t nb = (m + 127) / 128, np = (m + 31) / 32 * 32;
-    int64_t snb = nb, snp = np;
+    const int64_t nb = (m + 127) / 128, np = (m + 31) / 32 * 32, nq = (m + 63) / 64;
+    int64_t snb = nb, snp = np, snq = nq;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
       int64_t a = __shfl_up_sync(0xffffffffu, snb, d);
       int64_t b = __shfl_up_sync(0xffffffffu, snp, d);
-      if (lane >= d) { snb += a; snp += b; }
+      int64_t c = __shfl_up_sync(0xffffffffu, snq, d);
+      if (lane >= d) { snb += a; snp += b; snq += c; }
     }
-    const int64_t rb0 = carry_rb + snb - nb, p0 = carry_p + snp - np;
+    const int64_t rb0 = carry_rb + snb - nb, p0 = carry_p + snp - np, q0 = carry_q + snq - nq;
     const bool found = (h < G) && nb > 0 && pb >= rb0 && pb < rb0 + nb;
     const uint32_t ball = __ballot_sync(0xffffffffu, found);
     if (ball) {
@@ -62,14 +65,16 @@ __device__ __forceinline__ GroupBlock warp_find_block(const int32_t* offs, int32
       r.m = __shfl_sync(0xffffffffu, m, src);
       r.rb = __shfl_sync(0xffffffffu, rb0, src);
       r.p = __shfl_sync(0xffffffffu, p0, src);
+      r.q = __shfl_sync(0xffffffffu, q0, src);
       return r;
     }
     carry_rb = __shfl_sync(0xffffffffu, carry_rb + snb, 31);
     carry_p = __shfl_sync(0xffffffffu, carry_p + snp, 31);
+    carry_q = __shfl_sync(0xffffffffu, carry_q + snq, 31);
     o_prev = __shfl_sync(0xffffffffu, hi, 31);
   }
   GroupBlock none;
-  none.g = -1; none.lo = 0; none.m = 0; none.rb = 0; none.p = 0;
+  none.g = -1; none.lo = 0; none.m = 0; none.rb = 0; none.p = 0; none.q = 0;
   return none;
 }
 

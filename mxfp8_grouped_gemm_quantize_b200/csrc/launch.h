@@ -39,6 +39,13 @@ cudaError_t launch_moe_plan(const int32_t* idx, int64_t T, int32_t k, int32_t E,
 cudaError_t launch_moe_combine(const uint16_t* yp, int64_t rows, int64_t cols, const int32_t* inv, const float* w,
                                int64_t T, int32_t k, uint16_t* y, cudaStream_t stream);
 
+// NVFP4: tensor amax (fp32, device), rowwise and colwise quantisation.
+cudaError_t launch_nvfp4_amax(const uint16_t* x, int64_t n, float* amax, cudaStream_t stream);
+cudaError_t launch_nvfp4_rowwise(const uint16_t* x, int64_t rows, int64_t cols, const int32_t* offs, int32_t G,
+                                 const float* amax, uint8_t* q, uint8_t* sf, cudaStream_t stream);
+cudaError_t launch_nvfp4_colwise(const uint16_t* x, int64_t rows, int64_t cols, const int32_t* offs, int32_t G,
+                                 const float* amax, uint8_t* qT, int64_t ldT, uint8_t* sfT, cudaStream_t stream);
+
 enum GemmMode : int { kFwd = 0, kDgrad = 1, kWgrad = 2 };
 
 // One grouped GEMM.  a/b: operand codes (K-major), lda/ldb their row strides
