@@ -355,6 +355,33 @@ MXF8_API mxf8_status mxfp8_nvfp4_quantize_colwise(const uint16_t* x, int64_t row
                                                   uint8_t* qT, int64_t ldT, uint8_t* scalesT, int64_t scale_bytes,
                                                   void* stream);
 
+/* NVFP4 grouped GEMMs: the MXFP8 fwd / dgrad / wgrad with NVFP4 operands
+ * (E2M1 x E2M1 block-scaled MMA, kind::mxf4nvf4, 16-element E4M3 scales
+ * applied in hardware, fp32 accumulation), the output multiplied by
+ * 1 / (S_a * S_b) (S = 2688 / amax of each operand's tensor, as the
+ * quantisers use) and written as bf16.  Operands are the NVFP4 quantisers'
+ * outputs in the same roles as for MXFP8:
+ *   fwd:   rowwise(X, d_offs), rowwise(W as [E*N, K], one group)
+ *   dgrad: rowwise(dY, d_offs), colwise(W as [E*N, K], one group)
+ *   wgrad: colwise(dY, d_offs), colwise(X, d_offs)
+ * with the amax (device fp32) each was quantised with.  K % 64 == 0 and the
+ * MXFP8 GEMMs' other rules apply; errors and device status as for MXFP8. */
+MXF8_API mxf8_status mxfp8_nvfp4_grouped_gemm_fwd(const uint8_t* xq, const uint8_t* xs, int64_t xs_bytes,
+                                                  const float* x_amax, const uint8_t* wq, const uint8_t* ws,
+                                                  int64_t ws_bytes, const float* w_amax, const int32_t* d_offs,
+                                                  int32_t E, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                                  void* work, int64_t work_bytes, void* stream);
+MXF8_API mxf8_status mxfp8_nvfp4_grouped_gemm_dgrad(const uint8_t* dyq, const uint8_t* dys, int64_t dys_bytes,
+                                                    const float* dy_amax, const uint8_t* wqT, const uint8_t* wsT,
+                                                    int64_t wsT_bytes, const float* w_amax, const int32_t* d_offs,
+                                                    int32_t E, int64_t M, int64_t N, int64_t K, uint16_t* dx,
+                                                    void* work, int64_t work_bytes, void* stream);
+MXF8_API mxf8_status mxfp8_nvfp4_grouped_gemm_wgrad(const uint8_t* dyqT, const uint8_t* dysT, int64_t dysT_bytes,
+                                                    const float* dy_amax, const uint8_t* xqT, const uint8_t* xsT,
+                                                    int64_t xsT_bytes, const float* x_amax, const int32_t* d_offs,
+                                                    int32_t E, int64_t M, int64_t N, int64_t K, uint16_t* dw,
+                                                    void* work, int64_t work_bytes, void* stream);
+
 /* ---------------------------------------------------------------- status */
 
 /* Synchronises `stream`, then stores the device status of the last GEMM that

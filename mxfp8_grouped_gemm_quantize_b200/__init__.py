@@ -39,7 +39,8 @@ EXPORTED = ("mxfp8_rowwise_scale_bytes", "mxfp8_colwise_pitch", "mxfp8_colwise_s
             "mxfp8_grouped_gemm_dgrad_quant", "mxfp8_moe_plan_workspace_bytes", "mxfp8_moe_plan",
             "mxfp8_permute_quantize_dual", "mxfp8_moe_combine", "mxfp8_nvfp4_rowwise_scale_bytes",
             "mxfp8_nvfp4_colwise_pitch", "mxfp8_nvfp4_colwise_scale_bytes", "mxfp8_nvfp4_colwise_ld",
-            "mxfp8_nvfp4_amax", "mxfp8_nvfp4_quantize_rowwise", "mxfp8_nvfp4_quantize_colwise")
+            "mxfp8_nvfp4_amax", "mxfp8_nvfp4_quantize_rowwise", "mxfp8_nvfp4_quantize_colwise",
+            "mxfp8_nvfp4_grouped_gemm_fwd", "mxfp8_nvfp4_grouped_gemm_dgrad", "mxfp8_nvfp4_grouped_gemm_wgrad")
 
 
 class MXFP8Error(RuntimeError):
@@ -102,6 +103,10 @@ def lib() -> ctypes.CDLL:
         L.mxfp8_nvfp4_quantize_rowwise.argtypes = [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _i64, _vp]
         L.mxfp8_nvfp4_quantize_colwise.restype = _i32
         L.mxfp8_nvfp4_quantize_colwise.argtypes = [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _i64, _vp, _i64, _vp]
+        for n in ("mxfp8_nvfp4_grouped_gemm_fwd", "mxfp8_nvfp4_grouped_gemm_dgrad", "mxfp8_nvfp4_grouped_gemm_wgrad"):
+            getattr(L, n).restype = _i32
+            getattr(L, n).argtypes = [_vp, _vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i32, _i64, _i64, _i64, _vp,
+                                      _vp, _i64, _vp]
         L.mxfp8_grouped_gemm_fwd_noalloc.restype = _i32
         L.mxfp8_grouped_gemm_fwd_noalloc.argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp,
                                                      ctypes.POINTER(_i32), _vp]
@@ -389,3 +394,39 @@ def mxfp8_nvfp4_quantize_colwise(x, amax, offs=None, qT=None, scales=None, strea
     _check(lib().mxfp8_nvfp4_quantize_colwise(_ptr(x), R, C, _ptr(offs), G, _ptr(amax), _ptr(qT), ld, _ptr(scales),
                                               scales.numel(), _stream(stream)), "mxfp8_nvfp4_quantize_colwise")
     return qT, scales
+
+
+def _nvfp4_gemm(fn, a, a_s, a_amax, b, b_s, b_amax, offs, M, N, K, out, work, stream):
+    E = _groups(offs)
+    work = work if work is not None else new_workspace(E, M, N, K, out.device)
+    _check(getattr(lib(), fn)(_ptr(a), _ptr(a_s), a_s.numel(), _ptr(a_amax), _ptr(b), _ptr(b_s), b_s.numel(),
+                              _ptr(b_amax), _ptr(offs), E, M, N, K, _ptr(out), _ptr(work), work.numel(),
+                              _stream(stream)), fn)
+    return out
+
+
+def mxfp8_nvfp4_grouped_gemm_fwd(xq, xs, x_amax, wq, ws, w_amax, offs, N: int, out=None, work=None, stream=None):
+    """Y[M, N] from NVFP4 rowwise(X, offs) [M, K/2] and rowwise(W as [E*N, K]) with their amaxes."""
+    M, K = xq.shape[0], xq.shape[1] * 2
+    out = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    return _nvfp4_gemm("mxfp8_nvfp4_grouped_gemm_fwd", xq, xs, x_amax, wq, ws, w_amax, offs, M, N, K, out, work,
+                       stream)
+
+
+def mxfp8_nvfp4_grouped_gemm_dgrad(dyq, dys, dy_amax, wqT, wsT, w_amax, offs, K: int, out=None, work=None,
+                                   stream=None):
+    """dX[M, K] from NVFP4 rowwise(dY, offs) and colwise(W as [E*N, K])."""
+    M, N = dyq.shape[0], dyq.shape[1] * 2
+    out = out if out is not None else torch.empty((M, K), dtype=torch.bfloat16, device=dyq.device)
+    return _nvfp4_gemm("mxfp8_nvfp4_grouped_gemm_dgrad", dyq, dys, dy_amax, wqT, wsT, w_amax, offs, M, N, K, out,
+                       work, stream)
+
+
+def mxfp8_nvfp4_grouped_gemm_wgrad(dyqT, dysT, dy_amax, xqT, xsT, x_amax, offs, M: int, out=None, work=None,
+                                   stream=None):
+    """dW[E, N, K] from NVFP4 colwise(dY, offs) and colwise(X, offs)."""
+    N, K = dyqT.shape[0], xqT.shape[0]
+    E = _groups(offs)
+    out = out if out is not None else torch.empty((E, N, K), dtype=torch.bfloat16, device=dyqT.device)
+    return _nvfp4_gemm("mxfp8_nvfp4_grouped_gemm_wgrad", dyqT, dysT, dy_amax, xqT, xsT, x_amax, offs, M, N, K, out,
+                       work, stream)

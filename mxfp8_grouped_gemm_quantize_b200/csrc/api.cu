@@ -424,6 +424,85 @@ mxf8_status mxfp8_nvfp4_quantize_colwise(const uint16_t* x, int64_t rows, int64_
   return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "nvfp4_colwise launch");
 }
 
+mxf8_status mxfp8_nvfp4_grouped_gemm_fwd(const uint8_t* xq, const uint8_t* xs, int64_t xs_bytes, const float* x_amax,
+                                         const uint8_t* wq, const uint8_t* ws, int64_t ws_bytes, const float* w_amax,
+                                         const int32_t* d_offs, int32_t E, int64_t M, int64_t N, int64_t K,
+                                         uint16_t* y, void* work, int64_t work_bytes, void* stream) {
+  mxf8_status s = check_gemm_args({xq, xs, xs_bytes, wq, ws, ws_bytes, d_offs, E, M, N, K, y, work, work_bytes});
+  if (s != MXF8_OK) return s;
+  if (!x_amax || !w_amax || K % 64 != 0) return MXF8_ERR_INVALID_ARG;
+  if (xs_bytes < mxfp8_nvfp4_rowwise_scale_bytes(M, K, E) || ws_bytes < mxfp8_nvfp4_rowwise_scale_bytes(E * N, K, 1))
+    return MXF8_ERR_INVALID_ARG;
+  if ((s = check_device()) != MXF8_OK) return s;
+  if (M == 0) return cudaMemsetAsync(work, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) == cudaSuccess
+                         ? MXF8_OK : cuda_fail(cudaGetLastError(), "cudaMemsetAsync(status)");
+  mxf8::GemmArgs g{};
+  g.mode = mxf8::kFwd; g.E = E; g.M = M; g.N = N; g.K = K; g.offs = d_offs;
+  g.fp4 = true; g.amax_a = x_amax; g.amax_b = w_amax;
+  g.a = xq; g.lda = K / 2; g.a_rows = M; g.a_cols = K / 2;
+  g.b = wq; g.ldb = K / 2; g.b_rows = E * N; g.b_cols = K / 2;
+  g.sfa = xs; g.sfa_pitch = cdiv(K, 64); g.sfa_atoms = xs_bytes / 512;
+  g.sfb = ws; g.sfb_pitch = cdiv(K, 64); g.sfb_atoms = ws_bytes / 512;
+  g.out = y;
+  return run_gemm(g, work, stream);
+}
+
+mxf8_status mxfp8_nvfp4_grouped_gemm_dgrad(const uint8_t* dyq, const uint8_t* dys, int64_t dys_bytes,
+                                           const float* dy_amax, const uint8_t* wqT, const uint8_t* wsT,
+                                           int64_t wsT_bytes, const float* w_amax, const int32_t* d_offs, int32_t E,
+                                           int64_t M, int64_t N, int64_t K, uint16_t* dx, void* work,
+                                           int64_t work_bytes, void* stream) {
+  mxf8_status s =
+      check_gemm_args({dyq, dys, dys_bytes, wqT, wsT, wsT_bytes, d_offs, E, M, N, K, dx, work, work_bytes});
+  if (s != MXF8_OK) return s;
+  if (!dy_amax || !w_amax || K % 64 != 0) return MXF8_ERR_INVALID_ARG;
+  if (dys_bytes < mxfp8_nvfp4_rowwise_scale_bytes(M, N, E) ||
+      wsT_bytes < mxfp8_nvfp4_colwise_scale_bytes(E * N, K, 1))
+    return MXF8_ERR_INVALID_ARG;
+  if ((s = check_device()) != MXF8_OK) return s;
+  if (M == 0) return cudaMemsetAsync(work, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) == cudaSuccess
+                         ? MXF8_OK : cuda_fail(cudaGetLastError(), "cudaMemsetAsync(status)");
+  const int64_t ldw = mxfp8_nvfp4_colwise_ld(E * N, 1) / 2;   // bytes
+  mxf8::GemmArgs g{};
+  g.mode = mxf8::kDgrad; g.E = E; g.M = M; g.N = N; g.K = K; g.offs = d_offs;
+  g.fp4 = true; g.amax_a = dy_amax; g.amax_b = w_amax;
+  g.a = dyq; g.lda = N / 2; g.a_rows = M; g.a_cols = N / 2;
+  g.b = wqT; g.ldb = ldw; g.b_rows = K; g.b_cols = ldw;
+  g.sfa = dys; g.sfa_pitch = cdiv(N, 64); g.sfa_atoms = dys_bytes / 512;
+  g.sfb = wsT; g.sfb_pitch = mxfp8_nvfp4_colwise_pitch(E * N, 1); g.sfb_atoms = wsT_bytes / 512;
+  g.out = dx;
+  return run_gemm(g, work, stream);
+}
+
+mxf8_status mxfp8_nvfp4_grouped_gemm_wgrad(const uint8_t* dyqT, const uint8_t* dysT, int64_t dysT_bytes,
+                                           const float* dy_amax, const uint8_t* xqT, const uint8_t* xsT,
+                                           int64_t xsT_bytes, const float* x_amax, const int32_t* d_offs, int32_t E,
+                                           int64_t M, int64_t N, int64_t K, uint16_t* dw, void* work,
+                                           int64_t work_bytes, void* stream) {
+  mxf8_status s =
+      check_gemm_args({dyqT, dysT, dysT_bytes, xqT, xsT, xsT_bytes, d_offs, E, M, N, K, dw, work, work_bytes});
+  if (s != MXF8_OK) return s;
+  if (!dy_amax || !x_amax || K % 64 != 0) return MXF8_ERR_INVALID_ARG;
+  if (dysT_bytes < mxfp8_nvfp4_colwise_scale_bytes(M, N, E) || xsT_bytes < mxfp8_nvfp4_colwise_scale_bytes(M, K, E))
+    return MXF8_ERR_INVALID_ARG;
+  if ((s = check_device()) != MXF8_OK) return s;
+  const int64_t ldt = mxfp8_nvfp4_colwise_ld(M, E) / 2;   // bytes
+  mxf8::GemmArgs g{};
+  g.mode = mxf8::kWgrad; g.E = E; g.M = M; g.N = N; g.K = K; g.offs = d_offs;
+  g.fp4 = true; g.amax_a = dy_amax; g.amax_b = x_amax;
+  g.a = dyqT; g.lda = ldt; g.a_rows = N; g.a_cols = ldt;
+  g.b = xqT; g.ldb = ldt; g.b_rows = K; g.b_cols = ldt;
+  const int64_t pitch = mxfp8_nvfp4_colwise_pitch(M, E);
+  g.sfa = dysT; g.sfa_pitch = pitch; g.sfa_atoms = dysT_bytes / 512;
+  g.sfb = xsT; g.sfb_pitch = pitch; g.sfb_atoms = xsT_bytes / 512;
+  g.out = dw;
+  if (g.sfa_atoms < 1 || g.sfb_atoms < 1) {
+    // M = 0: no scale atoms exist; point at the (unread) code buffers instead.
+    g.sfa = dyqT; g.sfb = xqT; g.sfa_atoms = g.sfb_atoms = 1;
+  }
+  return run_gemm(g, work, stream);
+}
+
 mxf8_status mxfp8_get_status(const void* work, void* stream, int32_t* device_status) {
   if (!work || !device_status) return MXF8_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -54,7 +54,7 @@ constexpr int EPI_STAGE = 32 * 128;        // one epilogue buffer: 32 rows x 64 
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_STRIDE = 12;        // per stage: SFA 4 columns, then SFB 8 columns
 constexpr int MAXG = MXF8_GEMM_MAX_GROUPS;
-constexpr int SCHED_INTS = 4 * (MAXG + 1);
+constexpr int SCHED_INTS = 5 * (MAXG + 1);
 
 constexpr int round_up_c(int a, int b) { return (a + b - 1) / b * b; }
 
@@ -63,10 +63,16 @@ constexpr int round_up_c(int a, int b) { return (a + b - 1) / b * b; }
 // 2 x 256-deep; pair: 5 x 128-deep or 3 x 256-deep.  Deeper stages amortise
 // the fixed cost of a stage hand-off (barrier round trip, copy issue) over
 // twice the MMAs.
-template <int CG, int KS_>
+// FP4 (NVFP4 operands): a 128-byte K block holds 256 elements = four MMAs of
+// K = 64, each with its own scale atom (16-element blocks), so a stage
+// carries four times the scale bytes, the ring is one stage shorter, and the
+// scale sets alternate between two tensor-memory sets of 48 columns.
+template <int CG, int KS_, bool FP4 = false>
 struct Cfg {
   static constexpr int KS = KS_;
-  static constexpr int STAGES = CG == 2 ? (KS == 2 ? 3 : 5) : (KS == 2 ? 2 : 4);
+  static constexpr int STAGES = FP4 ? 3 : (CG == 2 ? (KS == 2 ? 3 : 5) : (KS == 2 ? 2 : 4));
+  static constexpr int APK = FP4 ? 4 : 1;              // scale atoms per K block and 128 rows
+  static constexpr int SFA_T = SFA_TILE * APK, SFB_T = SFB_TILE * APK;
   static constexpr int SLOTS = STAGES * KS;            // 128-wide K-block slots in the ring
   static constexpr int B_ROWS = BN / CG;               // B rows staged by each CTA
   static constexpr int A_TILE = BM * BK;               // 16 KB of E4M3 codes
@@ -74,13 +80,15 @@ struct Cfg {
   static constexpr int EPI_BUFS = (CG == 2 && KS == 1) ? 2 : 1;
   // The two 128x256 accumulators overlap in OV 64-column chunks: accumulator 1
   // starts at column ACC_STRIDE, and the scale sets of all slots follow it.
-  static constexpr int OV = (SLOTS * SF_STRIDE <= 64) ? 1 : 2;
+  static constexpr int SF_SETS = FP4 ? 2 : SLOTS;      // scale sets in tensor memory
+  static constexpr int SF_SET_COLS = SF_STRIDE * APK;  // columns of one set
+  static constexpr int OV = (SF_SETS * SF_SET_COLS <= 64) ? 1 : 2;
   static constexpr uint32_t ACC_STRIDE = 256 - 64 * OV;
   static constexpr uint32_t SF_COL = ACC_STRIDE + 256;
   // Bytes one CTA pair (or CTA) receives for a stage holding `nh` K blocks:
   // the scale boxes always span all KS atoms.
   static constexpr uint32_t stage_tx(int nh) {
-    return CG * (nh * (A_TILE + B_TILE) + KS * (SFA_TILE + SFB_TILE));
+    return CG * (nh * (A_TILE + B_TILE) + KS * (SFA_T + SFB_T));
   }
   // Slot q = stage * KS + h.  Scale atoms of one stage are fetched as boxes of
   // KS consecutive atoms: SFA box at OFF_SFA + stage * KS * 512, the two SFB
@@ -88,15 +96,15 @@ struct Cfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + SLOTS * A_TILE;
   static constexpr int OFF_SFA = OFF_B + SLOTS * B_TILE;
-  static constexpr int OFF_SFB = OFF_SFA + SLOTS * SFA_TILE;
-  static constexpr int OFF_EPI = round_up_c(OFF_SFB + SLOTS * SFB_TILE, 1024);
+  static constexpr int OFF_SFB = OFF_SFA + SLOTS * SFA_T;
+  static constexpr int OFF_EPI = round_up_c(OFF_SFB + SLOTS * SFB_T, 1024);
   static constexpr int OFF_BAR = OFF_EPI + 4 * EPI_BUFS * EPI_STAGE;
   static constexpr int OFF_MISC = OFF_BAR + 128;
   static constexpr int OFF_SCHED = OFF_MISC + 64;
   static constexpr int SMEM_BYTES = OFF_SCHED + SCHED_INTS * 4 + 1024;   // + slack to align the base
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(OFF_B % 1024 == 0 && B_TILE % 1024 == 0 && OFF_EPI % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-  static_assert(SF_COL + SF_STRIDE * SLOTS <= TMEM_COLS, "scale columns");
+  static_assert(SF_COL + SF_SET_COLS * SF_SETS <= TMEM_COLS, "scale columns");
   static_assert(KS >= 1 && KS <= 2 && STAGES >= 2, "pipeline shape");
   static_assert((2 * STAGES + 3) * 8 <= 128, "barrier area");
 };
@@ -119,6 +127,10 @@ struct Params {
   uint8_t* qc;                         // colwise codes [out_ld, qc_ld] (transposed)
   uint8_t* sc;                         // colwise scale atoms, pitch sc_pitch
   int64_t qc_ld, sc_pitch;
+  // NVFP4 operands: device amax of each operand's tensor (tensor scale
+  // S = 2688 / amax); the output is the accumulator times 1 / (S_a * S_b).
+  const float* amax_a;
+  const float* amax_b;
 };
 
 // Per-CTA schedule, built from the offsets by warp 0.
@@ -128,6 +140,7 @@ struct Sched {
   int32_t* rb;      // [E]   RB_e: 128-row blocks before group e (rowwise scale rows,
                     //       colwise scale block-columns / 4)
   int32_t* p;       // [E]   P_e: 32-padded rows before group e (colwise code column)
+  int32_t* q;       // [E]   Q_e: 64-row blocks before group e (NVFP4 colwise scale atoms)
 };
 
 // One CTA's share of a tile.
@@ -164,8 +177,12 @@ __device__ __forceinline__ int32_t advance_group(const Sched& s, int32_t E, int3
 }
 
 // Tile t (a pair tile when CG = 2) of group e as seen by CTA `rank` of its pair.
-template <int CG>
+template <int CG, bool FP4 = false>
 __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int32_t t, int32_t e, uint32_t rank) {
+  // K blocks are 128 bytes of codes: 128 E4M3 or 256 E2M1 elements; MMA steps
+  // take 32 (E4M3) or 64 (E2M1) elements.  TMA x coordinates count bytes.
+  constexpr int KE = FP4 ? 256 : 128, KSTEP = FP4 ? 64 : 32, EB = FP4 ? 2 : 1;   // EB: elements per byte
+  constexpr int RPA = FP4 ? 64 : 128;   // colwise rows per scale atom column
   Tile tl;
   const int32_t row0 = s.off[e], m = s.off[e + 1] - s.off[e];
   const int32_t munits = group_m_units<CG>(p, m);
@@ -174,8 +191,8 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int
   const int32_t nt = local / munits;
   const int32_t b_half = (CG == 2) ? BN / 2 * static_cast<int32_t>(rank) : 0;
   const int64_t L = p.mode == kFwd ? p.K : (p.mode == kDgrad ? p.N : m);
-  tl.kblocks = static_cast<int32_t>((L + BK - 1) / BK);
-  tl.ksteps_last = tl.kblocks > 0 ? static_cast<int32_t>((L - int64_t(BK) * (tl.kblocks - 1) + 31) / 32) : 0;
+  tl.kblocks = static_cast<int32_t>((L + KE - 1) / KE);
+  tl.ksteps_last = tl.kblocks > 0 ? static_cast<int32_t>((L - int64_t(KE) * (tl.kblocks - 1) + KSTEP - 1) / KSTEP) : 0;
   int64_t sfa_row, sfa_col, sfb_row, sfb_col, out_cols;
   if (p.mode == kFwd) {
     tl.a_x = 0;                              tl.a_y = row0 + BM * mt;
@@ -188,18 +205,18 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int
     out_cols = p.N;
   } else if (p.mode == kDgrad) {
     tl.a_x = 0;                              tl.a_y = row0 + BM * mt;
-    tl.b_x = static_cast<int32_t>(e * p.N);  tl.b_y = BN * nt + b_half;
+    tl.b_x = static_cast<int32_t>(e * p.N / EB); tl.b_y = BN * nt + b_half;
     sfa_row = s.rb[e] + mt;                  sfa_col = 0;
-    sfb_row = 2 * nt;                        sfb_col = e * (p.N / 128);
+    sfb_row = 2 * nt;                        sfb_col = e * (p.N / RPA);
     tl.q_rb = s.rb[e] + mt;                  tl.q_p = s.p[e] + BM * mt;
     tl.out_row = int64_t(row0) + BM * mt;
     tl.rows = static_cast<int32_t>(min64(BM, m - BM * mt));
     out_cols = p.K;
   } else {
-    tl.a_x = s.p[e];                         tl.a_y = BM * mt;
-    tl.b_x = s.p[e];                         tl.b_y = BN * nt + b_half;
-    sfa_row = mt;                            sfa_col = s.rb[e];
-    sfb_row = 2 * nt;                        sfb_col = s.rb[e];
+    tl.a_x = s.p[e] / EB;                    tl.a_y = BM * mt;
+    tl.b_x = s.p[e] / EB;                    tl.b_y = BN * nt + b_half;
+    sfa_row = mt;                            sfa_col = FP4 ? s.q[e] : s.rb[e];
+    sfb_row = 2 * nt;                        sfb_col = FP4 ? s.q[e] : s.rb[e];
     tl.q_rb = 0;                             tl.q_p = 0;
     tl.out_row = int64_t(e) * p.N + BM * mt;
     tl.rows = static_cast<int32_t>(min64(BM, p.N - int64_t(BM) * mt));
@@ -225,7 +242,7 @@ template <int CG>
 __device__ int32_t build_schedule(const Params& p, const Sched& s) {
   const int lane = threadIdx.x & 31;
   const int32_t ntl = n_tiles(p);
-  int32_t carry_t = 0, carry_rb = 0, carry_p = 0;
+  int32_t carry_t = 0, carry_rb = 0, carry_p = 0, carry_q = 0;
   bool bad = false;
   for (int32_t base = 0; base < p.E; base += 32) {
     const int32_t h = base + lane;
@@ -237,25 +254,28 @@ __device__ int32_t build_schedule(const Params& p, const Sched& s) {
     bad |= __any_sync(0xffffffffu, lbad);
     const int32_t m = (h < p.E && !lbad) ? b - a : 0;
     const int32_t tiles = (h < p.E) ? group_m_units<CG>(p, m) * ntl : 0;
-    const int32_t nb = (m + BM - 1) / BM, np = (m + 31) / 32 * 32;
-    int32_t st = tiles, sr = nb, sp = np;
+    const int32_t nb = (m + BM - 1) / BM, np = (m + 31) / 32 * 32, nq = (m + 63) / 64;
+    int32_t st = tiles, sr = nb, sp = np, sq = nq;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
       const int32_t x = __shfl_up_sync(0xffffffffu, st, d);
       const int32_t y = __shfl_up_sync(0xffffffffu, sr, d);
       const int32_t z = __shfl_up_sync(0xffffffffu, sp, d);
-      if (lane >= d) { st += x; sr += y; sp += z; }
+      const int32_t w = __shfl_up_sync(0xffffffffu, sq, d);
+      if (lane >= d) { st += x; sr += y; sp += z; sq += w; }
     }
     if (h < p.E) {
       s.tile0[h] = carry_t + st - tiles;
       s.rb[h] = carry_rb + sr - nb;
       s.p[h] = carry_p + sp - np;
+      s.q[h] = carry_q + sq - nq;
       s.off[h] = a;
       if (h == p.E - 1) { s.off[p.E] = b; s.tile0[p.E] = carry_t + st; }
     }
     carry_t = __shfl_sync(0xffffffffu, carry_t + st, 31);
     carry_rb = __shfl_sync(0xffffffffu, carry_rb + sr, 31);
     carry_p = __shfl_sync(0xffffffffu, carry_p + sp, 31);
+    carry_q = __shfl_sync(0xffffffffu, carry_q + sq, 31);
   }
   if (bad) {
     if (lane == 0 && blockIdx.x == 0) atomicCAS(p.status, 0, static_cast<int32_t>(MXF8_ERR_BAD_OFFSETS));
@@ -277,12 +297,12 @@ __device__ __forceinline__ void tmem_wait_regs(uint32_t (&r)[32]) {
                : "memory");
 }
 
-template <int CG, int KS, bool QE>
+template <int CG, int KS, bool QE, bool FP4>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                     const __grid_constant__ CUtensorMap tmOut, const Params p) {
-  using C = Cfg<CG, KS>;
+  using C = Cfg<CG, KS, FP4>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -306,6 +326,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   sc.off = sched + (MAXG + 1);
   sc.rb = sched + 2 * (MAXG + 1);
   sc.p = sched + 3 * (MAXG + 1);
+  sc.q = sched + 4 * (MAXG + 1);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -350,7 +371,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       bool failed = false;
       for (int32_t t = unit0; t < total && !failed; t += nunits) {
         eh = advance_group(sc, p.E, t, eh);
-        const Tile tl = decode_tile<CG>(p, sc, t, eh, rank);
+        const Tile tl = decode_tile<CG, FP4>(p, sc, t, eh, rank);
         for (int32_t kb0 = 0; kb0 < tl.kblocks; kb0 += C::KS) {
           if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, lim)) {
             record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
@@ -359,14 +380,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           }
           const int32_t nh = min(C::KS, tl.kblocks - kb0);   // K blocks in this stage
           const uint32_t fb = full_bar(s);
-          const uint32_t ssa = smem_addr(smem + C::OFF_SFA + s * C::KS * SFA_TILE);
-          const uint32_t ssb = smem_addr(smem + C::OFF_SFB + s * C::KS * SFB_TILE);
+          const uint32_t ssa = smem_addr(smem + C::OFF_SFA + s * C::KS * C::SFA_T);
+          const uint32_t ssb = smem_addr(smem + C::OFF_SFB + s * C::KS * C::SFB_T);
           // Scale atoms are 4 rows of 128 bytes in the scale maps; each box
-          // takes KS consecutive atoms (those past the tile's K blocks are
-          // fetched but unused; atoms past the buffer read as zero).
-          const int32_t ya = static_cast<int32_t>(4 * (tl.sfa_atom + kb0));
-          const int32_t yb0 = static_cast<int32_t>(4 * (tl.sfb_atom0 + kb0));
-          const int32_t yb1 = static_cast<int32_t>(4 * (tl.sfb_atom1 + kb0));
+          // takes the KS * APK consecutive atoms of the stage (those past the
+          // tile's K blocks are fetched but unused; atoms past the buffer read
+          // as zero).
+          const int32_t ya = static_cast<int32_t>(4 * (tl.sfa_atom + C::APK * kb0));
+          const int32_t yb0 = static_cast<int32_t>(4 * (tl.sfb_atom0 + C::APK * kb0));
+          const int32_t yb1 = static_cast<int32_t>(4 * (tl.sfb_atom1 + C::APK * kb0));
           if constexpr (CG == 2) {
             if (leader) mbar_arrive_expect_tx(fb, C::stage_tx(nh));   // both CTAs' bytes land here
           } else {
@@ -388,11 +410,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           if constexpr (CG == 2) {
             tma_load_2d_pair(ssa, &tmSFA, 0, ya, fb);
             tma_load_2d_pair(ssb, &tmSFB, 0, yb0, fb);
-            tma_load_2d_pair(ssb + C::KS * 512, &tmSFB, 0, yb1, fb);
+            tma_load_2d_pair(ssb + C::KS * C::APK * 512, &tmSFB, 0, yb1, fb);
           } else {
             tma_load_2d(ssa, &tmSFA, 0, ya, fb);
             tma_load_2d(ssb, &tmSFB, 0, yb0, fb);
-            tma_load_2d(ssb + C::KS * 512, &tmSFB, 0, yb1, fb);
+            tma_load_2d(ssb + C::KS * C::APK * 512, &tmSFB, 0, yb1, fb);
           }
           ++it;
           if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -414,7 +436,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       // Instruction descriptor: E4M3 x E4M3, E8M0 scales, K-major A and B,
       // M = 128*CG, N = 256; the scale-factor ids (bits 4-5 for B, 29-30 for
       // A) select the byte of the 32-bit scale column used by each K step.
-      const uint32_t idesc0 = (1u << 23) | (uint32_t(BN >> 3) << 17) | (uint32_t((BM * CG) >> 4) << 24);
+      // FP4: E2M1 x E2M1 (format 1 in both fields), E4M3 scales (bit 23 clear),
+      // K = 64 per MMA, the whole 32-bit scale column (4 blocks of 16) per MMA.
+      const uint32_t idesc0 = FP4 ? ((1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t((BM * CG) >> 4) << 24))
+                                  : ((1u << 23) | (uint32_t(BN >> 3) << 17) | (uint32_t((BM * CG) >> 4) << 24));
+      constexpr int KE = FP4 ? 256 : 128, KSTEP = FP4 ? 64 : 32;   // elements per K block / per MMA
+      uint32_t kbc = 0;                                             // K blocks issued (FP4 scale set parity)
       // The tensor pipe queues only a few instructions, so scalar work between
       // MMAs stalls it: everything below is set up once, descriptors of a
       // slot are the base descriptor plus the slot's offset in 16-byte units
@@ -427,8 +454,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const uint32_t sf_t0 = tmem + C::SF_COL;
       // fwd/dgrad: every tile has the same K loop; wgrad: the group's rows.
       const int64_t L_fixed = p.mode == kFwd ? p.K : p.N;
-      const int32_t kb_fixed = static_cast<int32_t>((L_fixed + BK - 1) / BK);
-      const int32_t ks_fixed = static_cast<int32_t>((L_fixed - int64_t(BK) * (kb_fixed - 1) + 31) / 32);
+      const int32_t kb_fixed = static_cast<int32_t>((L_fixed + KE - 1) / KE);
+      const int32_t ks_fixed = static_cast<int32_t>((L_fixed - int64_t(KE) * (kb_fixed - 1) + KSTEP - 1) / KSTEP);
       uint32_t s = 0, ph = 0, j = 0;
       int32_t eh = 0;
       bool failed = false;
@@ -437,9 +464,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (p.mode == kWgrad) {
           eh = advance_group(sc, p.E, t, eh);
           const int32_t m = sc.off[eh + 1] - sc.off[eh];
-          kblocks = (m + BK - 1) / BK;
+          kblocks = (m + KE - 1) / KE;
           if (kblocks == 0) continue;
-          ksteps_last = (m - BK * (kblocks - 1) + 31) / 32;
+          ksteps_last = (m - KE * (kblocks - 1) + KSTEP - 1) / KSTEP;
         }
         const uint32_t d_tmem = tmem + (j & 1) * C::ACC_STRIDE;
         if (!mbar_wait(acc_empty, (j & 1) ^ 1, abort_flag, lim)) {
@@ -461,32 +488,58 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const int32_t kb = kb0 + h;
             if (kb < kblocks) {
               const uint32_t q = s * C::KS + h;
-              const uint32_t sfa_t = sf_t0 + SF_STRIDE * q, sfb_t = sfa_t + 4;
-              const uint64_t dsa = dsa0 + (SFA_TILE >> 4) * q;
-              const uint64_t dsb = dsb0 + (SFB_TILE >> 4) * C::KS * s + (512 >> 4) * h;
-              if constexpr (CG == 2) {
-                tc_cp_32x128b_x4_pair(sfa_t, dsa);
-                tc_cp_32x128b_x4_pair(sfb_t, dsb);
-                tc_cp_32x128b_x4_pair(sfb_t + 4, dsb + (512 >> 4) * C::KS);
-              } else {
-                tc_cp_32x128b_x4(sfa_t, dsa);
-                tc_cp_32x128b_x4(sfb_t, dsb);
-                tc_cp_32x128b_x4(sfb_t + 4, dsb + (512 >> 4) * C::KS);
-              }
               const uint64_t da = da0 + (C::A_TILE >> 4) * q, db = db0 + (C::B_TILE >> 4) * q;
-              const int32_t nk = (kb == kblocks - 1) ? ksteps_last : BK / 32;
+              const int32_t nk = (kb == kblocks - 1) ? ksteps_last : 4;
+              if constexpr (FP4) {
+                // four MMAs of K = 64, each with its own atoms: SFA atom i of the
+                // stage's SFA box, SFB atoms i of its two SFB boxes
+                const uint32_t set0 = sf_t0 + C::SF_SET_COLS * (kbc & 1);
+                const uint64_t dsa = dsa0 + (C::SFA_T >> 4) * q;
+                const uint64_t dsb = dsb0 + (C::SFB_T >> 4) * C::KS * s + (C::APK * 512 >> 4) * h;
 #pragma unroll
-              for (int k = 0; k < BK / 32; ++k) {
-                if (k < nk) {
-                  // +2 per step: the start-address field counts 16-byte units, one step is 32 bytes of K
-                  const uint32_t idesc = idesc0 | (uint32_t(k) << 4) | (uint32_t(k) << 29);
-                  if constexpr (CG == 2)
-                    tc_mma_mxf8_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
-                                     sfb_t | (uint32_t(k) << 30), acc);
-                  else
-                    tc_mma_mxf8(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
-                                sfb_t | (uint32_t(k) << 30), acc);
-                  acc = 1;
+                for (int i = 0; i < 4; ++i) {
+                  if (i < nk) {
+                    const uint32_t sfa_t = set0 + SF_STRIDE * i, sfb_t = sfa_t + 4;
+                    tc_cp_32x128b_x4(sfa_t, dsa + (512 >> 4) * i);
+                    tc_cp_32x128b_x4(sfb_t, dsb + (512 >> 4) * i);
+                    tc_cp_32x128b_x4(sfb_t + 4, dsb + (512 >> 4) * (C::KS * C::APK + i));
+                  }
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  if (i < nk) {
+                    const uint32_t sfa_t = set0 + SF_STRIDE * i, sfb_t = sfa_t + 4;
+                    tc_mma_nvf4(d_tmem, da + 2 * i, db + 2 * i, idesc0, sfa_t, sfb_t, acc);
+                    acc = 1;
+                  }
+                }
+                ++kbc;
+              } else {
+                const uint32_t sfa_t = sf_t0 + SF_STRIDE * q, sfb_t = sfa_t + 4;
+                const uint64_t dsa = dsa0 + (SFA_TILE >> 4) * q;
+                const uint64_t dsb = dsb0 + (SFB_TILE >> 4) * C::KS * s + (512 >> 4) * h;
+                if constexpr (CG == 2) {
+                  tc_cp_32x128b_x4_pair(sfa_t, dsa);
+                  tc_cp_32x128b_x4_pair(sfb_t, dsb);
+                  tc_cp_32x128b_x4_pair(sfb_t + 4, dsb + (512 >> 4) * C::KS);
+                } else {
+                  tc_cp_32x128b_x4(sfa_t, dsa);
+                  tc_cp_32x128b_x4(sfb_t, dsb);
+                  tc_cp_32x128b_x4(sfb_t + 4, dsb + (512 >> 4) * C::KS);
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  if (k < nk) {
+                    // +2 per step: the start-address field counts 16-byte units, one step is 32 bytes of K
+                    const uint32_t idesc = idesc0 | (uint32_t(k) << 4) | (uint32_t(k) << 29);
+                    if constexpr (CG == 2)
+                      tc_mma_mxf8_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
+                                       sfb_t | (uint32_t(k) << 30), acc);
+                    else
+                      tc_mma_mxf8(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
+                                  sfb_t | (uint32_t(k) << 30), acc);
+                    acc = 1;
+                  }
                 }
               }
             }
@@ -515,9 +568,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int32_t row_base = 32 * static_cast<int32_t>(quarter);
     uint32_t j = 0, ec = 0;
     int32_t eh = 0;
+    float oscale = 1.0f;   // FP4: 1 / (S_a * S_b), S = 2688 / amax (1 when amax = 0)
+    if constexpr (FP4) {
+      const float aa = __ldg(p.amax_a), ab = __ldg(p.amax_b);
+      const float sa = aa == 0.0f ? 1.0f : __fdiv_rn(2688.0f, aa), sb = ab == 0.0f ? 1.0f : __fdiv_rn(2688.0f, ab);
+      oscale = __frcp_rn(__fmul_rn(sa, sb));
+    }
     for (int32_t t = unit0; t < total; t += nunits) {
       eh = advance_group(sc, p.E, t, eh);
-      const Tile tl = decode_tile<CG>(p, sc, t, eh, rank);
+      const Tile tl = decode_tile<CG, FP4>(p, sc, t, eh, rank);
       const int32_t vr = max(0, min(32, tl.rows - row_base));       // valid rows of this warp's slice
       uint16_t* out_tile = p.out + tl.out_row * p.out_ld + tl.out_col;
       if (tl.kblocks == 0) {
@@ -570,8 +629,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           uint32_t pk[32];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            pk[i] = cvt_bf16x2(__uint_as_float(c0[2 * i]), __uint_as_float(c0[2 * i + 1]));
-            pk[16 + i] = cvt_bf16x2(__uint_as_float(c1[2 * i]), __uint_as_float(c1[2 * i + 1]));
+            if constexpr (FP4) {
+              pk[i] = cvt_bf16x2(__fmul_rn(__uint_as_float(c0[2 * i]), oscale),
+                                 __fmul_rn(__uint_as_float(c0[2 * i + 1]), oscale));
+              pk[16 + i] = cvt_bf16x2(__fmul_rn(__uint_as_float(c1[2 * i]), oscale),
+                                      __fmul_rn(__uint_as_float(c1[2 * i + 1]), oscale));
+            } else {
+              pk[i] = cvt_bf16x2(__uint_as_float(c0[2 * i]), __uint_as_float(c0[2 * i + 1]));
+              pk[16 + i] = cvt_bf16x2(__uint_as_float(c1[2 * i]), __uint_as_float(c1[2 * i + 1]));
+            }
           }
           uint8_t* stg = stage_base + (ec % C::EPI_BUFS) * EPI_STAGE;
           uint4* st4 = reinterpret_cast<uint4*>(stg);
@@ -697,27 +763,27 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
 // ---------------------------------------------------------------- host side
 struct DeviceSetup {
-  bool done[2][2][2] = {};    // [CG - 1][KS - 1][QE]
+  bool done[2][2][2][2] = {};    // [CG - 1][KS - 1][QE][FP4]
   int num_sms = 0;
-  int max_pairs[2][2] = {};   // [KS - 1][QE]
+  int max_pairs[2][2][2] = {};   // [KS - 1][QE][FP4]
 };
 DeviceSetup g_setup[64];
 
-template <int CG, int KS, bool QE>
+template <int CG, int KS, bool QE, bool FP4 = false>
 cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_t stream) {
-  using C = Cfg<CG, KS>;
+  using C = Cfg<CG, KS, FP4>;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   DeviceSetup& ds = g_setup[dev];
-  auto kernel = grouped_gemm_kernel<CG, KS, QE>;
+  auto kernel = grouped_gemm_kernel<CG, KS, QE, FP4>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  if (!ds.done[CG - 1][KS - 1][QE]) {
+  if (!ds.done[CG - 1][KS - 1][QE][FP4]) {
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     err = cudaDeviceGetAttribute(&ds.num_sms, cudaDevAttrMultiProcessorCount, dev);
@@ -732,16 +798,16 @@ cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_
       int clusters = 0;
       err = cudaOccupancyMaxActiveClusters(&clusters, kernel, &q);
       if (err != cudaSuccess) return err;
-      ds.max_pairs[KS - 1][QE] = clusters > 0 ? clusters : 1;
+      ds.max_pairs[KS - 1][QE][FP4] = clusters > 0 ? clusters : 1;
     }
-    ds.done[CG - 1][KS - 1][QE] = true;
+    ds.done[CG - 1][KS - 1][QE][FP4] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
   if (CG == 2) {
-    cfg.gridDim = dim3(2 * ds.max_pairs[KS - 1][QE]);
+    cfg.gridDim = dim3(2 * ds.max_pairs[KS - 1][QE][FP4]);
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   } else {
@@ -773,6 +839,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   env = std::getenv("MXF8_GEMM_KS");
   if (env && std::strcmp(env, "1") == 0) ks = 1;
   if (env && std::strcmp(env, "2") == 0) ks = 2;
+  if (a.fp4) { cg = 1; ks = 1; }   // NVFP4: one configuration (1-CTA, 3 x 128-byte stages)
+  const uint32_t sf_box_rows = 4 * ks * (a.fp4 ? 4 : 1);
   const int64_t out_rows = a.mode == kWgrad ? int64_t(a.E) * a.N : a.M;
   const int64_t out_cols = a.mode == kFwd ? a.N : a.K;
   CUtensorMap maps[5];
@@ -781,9 +849,9 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
                CU_TENSOR_MAP_SWIZZLE_128B) &&
       make_tensor_map(&maps[1], a.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b_rows, a.b_cols, a.ldb, BK, BN / cg,
                CU_TENSOR_MAP_SWIZZLE_128B) &&
-      make_tensor_map(&maps[2], a.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfa_atoms * 4, 128, 128, 128, 4 * ks,
+      make_tensor_map(&maps[2], a.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfa_atoms * 4, 128, 128, 128, sf_box_rows,
                CU_TENSOR_MAP_SWIZZLE_NONE) &&
-      make_tensor_map(&maps[3], a.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfb_atoms * 4, 128, 128, 128, 4 * ks,
+      make_tensor_map(&maps[3], a.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfb_atoms * 4, 128, 128, 128, sf_box_rows,
                CU_TENSOR_MAP_SWIZZLE_NONE) &&
       (a.out != nullptr
            ? make_tensor_map(&maps[4], a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out_rows, out_cols, out_cols, 64, 32,
@@ -808,6 +876,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   p.timeout_ns = a.timeout_ns;
   p.qr = a.qr; p.sr = a.sr; p.qc = a.qc; p.sc = a.sc;
   p.qc_ld = a.qc_ld; p.sc_pitch = a.sc_pitch;
+  p.amax_a = a.amax_a; p.amax_b = a.amax_b;
+  if (a.fp4) return launch_cg<1, 1, false, true>(p, maps, stream);
   const bool qe = a.qr != nullptr || a.qc != nullptr;
   if (qe) {
     if (cg == 2) return ks == 2 ? launch_cg<2, 2, true>(p, maps, stream) : launch_cg<2, 1, true>(p, maps, stream);

@@ -69,6 +69,11 @@ struct GemmArgs {
   uint8_t* qr = nullptr; uint8_t* sr = nullptr;
   uint8_t* qc = nullptr; uint8_t* sc = nullptr;
   int64_t qc_ld = 0, sc_pitch = 0;
+  // NVFP4 operands (codes packed two per byte, 16-element E4M3 scales):
+  // device amax of each operand tensor; lda/ldb/a_cols/b_cols are in bytes.
+  bool fp4 = false;
+  const float* amax_a = nullptr;
+  const float* amax_b = nullptr;
 };
 
 // Returns cudaSuccess or the CUDA error; *detail gets a short reason for

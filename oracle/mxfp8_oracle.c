@@ -816,7 +816,8 @@ int orc_nvfp4_quantize_rowwise(const uint16_t* x, int64_t R, int64_t C, const in
     if (orc_check_offsets(offs, G, R) != 0 || C % 64 != 0) { free(RB); free(P); return -1; }
     group_prefixes(offs, G, R, RB, P);
     for (g = 0; g < G; ++g) {
-        int64_t lo = offs[g], hi = offs[g + 1], r;
+        int64_t lo, hi, r;
+        group_bounds(offs, G, R, g, &lo, &hi);
         for (r = lo; r < hi; ++r) {
             int64_t pr = 128 * RB[g] + (r - lo), j;
             for (j = 0; j < C / 16; ++j) {
@@ -847,7 +848,9 @@ int orc_nvfp4_quantize_colwise(const uint16_t* x, int64_t R, int64_t C, const in
     int32_t g;
     if (orc_check_offsets(offs, G, R) != 0 || C % 64 != 0) return -1;
     for (g = 0; g < G; ++g) {
-        int64_t lo = offs[g], m = offs[g + 1] - offs[g], c;
+        int64_t lo, hi, m, c;
+        group_bounds(offs, G, R, g, &lo, &hi);
+        m = hi - lo;
         for (c = 0; c < C; ++c) {
             int64_t b;
             for (b = 0; b < cdiv(m, 16); ++b) {
@@ -879,9 +882,10 @@ int orc_nvfp4_dequantize_rowwise(const uint8_t* q, const uint8_t* sf, int64_t R,
     if (orc_check_offsets(offs, G, R) != 0) { free(RB); free(P); return -1; }
     group_prefixes(offs, G, R, RB, P);
     for (g = 0; g < G; ++g) {
-        int64_t r;
-        for (r = offs[g]; r < offs[g + 1]; ++r) {
-            int64_t pr = 128 * RB[g] + (r - offs[g]), c;
+        int64_t r, lo, hi;
+        group_bounds(offs, G, R, g, &lo, &hi);
+        for (r = lo; r < hi; ++r) {
+            int64_t pr = 128 * RB[g] + (r - lo), c;
             for (c = 0; c < C; ++c) {
                 uint8_t byte = q[r * (C / 2) + c / 2];
                 uint8_t nib = (c & 1) ? (byte >> 4) : (byte & 0xF);
@@ -902,7 +906,9 @@ int orc_nvfp4_dequantize_colwise(const uint8_t* qT, const uint8_t* sfT, int64_t 
     int32_t g;
     if (orc_check_offsets(offs, G, R) != 0) return -1;
     for (g = 0; g < G; ++g) {
-        int64_t lo = offs[g], m = offs[g + 1] - offs[g], t, c;
+        int64_t lo, hi, m, t, c;
+        group_bounds(offs, G, R, g, &lo, &hi);
+        m = hi - lo;
         for (t = 0; t < m; ++t)
             for (c = 0; c < C; ++c) {
                 int64_t col = p0 + t;

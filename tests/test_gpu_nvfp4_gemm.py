@@ -1,0 +1,144 @@
+"""GPU parity of the NVFP4 grouped GEMMs (fwd, dgrad, wgrad) against the fp64
+oracle on identical quantised inputs: the oracle dequantises the GPU's own
+NVFP4 bytes (code * E4M3 scale / tensor scale) and forms the per-expert
+products in fp64; the GPU accumulates in fp32.  Same tolerance as the MXFP8
+GEMMs (tests/helpers.py)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mxfp8_grouped_gemm_quantize_b200 import workloads as wl
+from tests.helpers import assert_gemm_close, f64, np_u8
+
+pytestmark = pytest.mark.gpu
+
+POISON = 0x7FC0
+
+
+@pytest.fixture(scope="module")
+def mx():
+    import mxfp8_grouped_gemm_quantize_b200 as m
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    assert m.mxfp8_device_supported(), "GPU tests need an sm_100 device"
+    return m
+
+
+class Fp4Case:
+    def __init__(self, mx, X, W, dY, offs):
+        self.mx, self.offs = mx, np.asarray(offs, dtype=np.int32)
+        self.E, self.N, self.K = W.shape
+        self.M = X.shape[0]
+        self.od = torch.from_numpy(self.offs).cuda()
+        Xd, Wd, dYd = X.cuda(), W.reshape(self.E * self.N, self.K).cuda(), dY.cuda()
+        self.ax, self.aw, self.ady = mx.mxfp8_nvfp4_amax(Xd), mx.mxfp8_nvfp4_amax(Wd), mx.mxfp8_nvfp4_amax(dYd)
+        self.xq, self.xs = mx.mxfp8_nvfp4_quantize_rowwise(Xd, self.ax, self.od)
+        self.wq, self.ws = mx.mxfp8_nvfp4_quantize_rowwise(Wd, self.aw)
+        self.dyq, self.dys = mx.mxfp8_nvfp4_quantize_rowwise(dYd, self.ady, self.od)
+        self.wqT, self.wsT = mx.mxfp8_nvfp4_quantize_colwise(Wd, self.aw)
+        self.dyqT, self.dysT = mx.mxfp8_nvfp4_quantize_colwise(dYd, self.ady, self.od)
+        self.xqT, self.xsT = mx.mxfp8_nvfp4_quantize_colwise(Xd, self.ax, self.od)
+        torch.cuda.synchronize()
+        S = lambda a: oracle.nvfp4_tensor_scale(np.float32(a.item()))  # noqa: E731
+        self.Sx, self.Sw, self.Sdy = S(self.ax), S(self.aw), S(self.ady)
+
+    def refs(self):
+        o, E, N, K, M = self.offs, self.E, self.N, self.K, self.M
+        Xd = oracle.nvfp4_dequantize_rowwise(np_u8(self.xq), np_u8(self.xs), self.Sx, o)
+        Wd = oracle.nvfp4_dequantize_rowwise(np_u8(self.wq), np_u8(self.ws), self.Sw).reshape(E, N, K)
+        dYd = oracle.nvfp4_dequantize_rowwise(np_u8(self.dyq), np_u8(self.dys), self.Sdy, o)
+        WdT = oracle.nvfp4_dequantize_colwise(np_u8(self.wqT), np_u8(self.wsT), E * N, self.Sw).reshape(E, N, K)
+        dYc = oracle.nvfp4_dequantize_colwise(np_u8(self.dyqT), np_u8(self.dysT), M, self.Sdy, o)
+        Xc = oracle.nvfp4_dequantize_colwise(np_u8(self.xqT), np_u8(self.xsT), M, self.Sx, o)
+        return (oracle.gemm_fwd(Xd, Wd, o), oracle.gemm_dgrad(dYd, WdT, o), oracle.gemm_wgrad(dYc, Xc, o))
+
+    def run(self):
+        mx = self.mx
+        y = mx.mxfp8_nvfp4_grouped_gemm_fwd(self.xq, self.xs, self.ax, self.wq, self.ws, self.aw, self.od, self.N)
+        dx = mx.mxfp8_nvfp4_grouped_gemm_dgrad(self.dyq, self.dys, self.ady, self.wqT, self.wsT, self.aw, self.od,
+                                               self.K)
+        dw = mx.mxfp8_nvfp4_grouped_gemm_wgrad(self.dyqT, self.dysT, self.ady, self.xqT, self.xsT, self.ax, self.od,
+                                               self.M)
+        torch.cuda.synchronize()
+        return y, dx, dw
+
+
+def check(mx, counts, N, K, seed=0):
+    offs = wl.offsets_from_counts(counts)
+    M, E = int(offs[-1]), len(counts)
+    c = Fp4Case(mx, wl.normal_bf16((M, K), 1.0, seed + 1), wl.normal_bf16((E, N, K), 1.0, seed + 2),
+                wl.normal_bf16((M, N), 1.0, seed + 3), offs)
+    y, dx, dw = c.run()
+    ry, rdx, rdw = c.refs()
+    assert_gemm_close(f64(y), ry, "nvfp4 fwd")
+    assert_gemm_close(f64(dx), rdx, "nvfp4 dgrad")
+    gdw = f64(dw)
+    for e in range(E):
+        if counts[e] == 0:
+            assert np.all(gdw[e] == 0.0)
+        else:
+            assert_gemm_close(gdw[e], rdw[e], f"nvfp4 wgrad expert {e}")
+
+
+def test_tiny(mx):
+    check(mx, [0, 7, 21, 36], 128, 256)
+
+
+def test_ragged_multi_tile(mx):
+    """Several tiles per group, ragged tails, an empty expert, a partial output
+    tile (N = 384) and a partial K block (K = 448: one full 256-element block
+    and one of three MMAs)."""
+    check(mx, [0, 1, 129, 300, 77, 255], 384, 448, seed=7)
+
+
+@pytest.mark.parametrize("counts,N,K", [([1], 128, 64), ([0, 0, 5], 128, 128), ([300], 256, 320),
+                                        ([129, 127], 512, 192), ([70, 0, 33, 200], 256, 1024)])
+def test_edge_shapes(mx, counts, N, K):
+    check(mx, counts, N, K, seed=sum(counts))
+
+
+def test_full_size_sampled_ds_v3_16b(mx):
+    """The DeepSeek-V3-16B-like gate/up linear at full size: outputs sampled
+    against the oracle's dot products of the dequantised operands."""
+    w = wl.WORKLOADS["ds-v3-16b"]()
+    L = w.layers[0]
+    X, W, dY = wl.layer_tensors(w, L)
+    c = Fp4Case(mx, X, W, dY, w.offsets)
+    y, dx, dw = c.run()
+    rng = np.random.default_rng(3)
+    o = c.offs
+    r = rng.integers(0, c.M, 128)
+    cn = rng.integers(0, c.N, 128)
+    ck = rng.integers(0, c.K, 128)
+    xq, xs = np_u8(c.xq), np_u8(c.xs)
+    wq, ws = np_u8(c.wq), np_u8(c.ws)
+    # dequantise only the rows needed (one expert's W rows per sample)
+    gy = f64(y)
+    group = np.searchsorted(o, r, side="right") - 1
+    ref = np.zeros(r.size)
+    xd_rows = {}
+    for i, (ri, ni, gi) in enumerate(zip(r, cn, group)):
+        if ri not in xd_rows:
+            xd_rows[ri] = oracle.nvfp4_dequantize_rowwise(xq[ri:ri + 1], _row_scales(xs, ri, o, c.K), c.Sx)[0]
+        wrow = int(gi) * c.N + int(ni)
+        wd = oracle.nvfp4_dequantize_rowwise(wq[wrow:wrow + 1], _row_scales(ws, wrow, None, c.K), c.Sw)[0]
+        ref[i] = float(np.dot(xd_rows[ri], wd))
+    assert_gemm_close(gy[r, cn], ref, "nvfp4 fwd (sampled)")
+    assert np.all(np.isfinite(f64(dx)[r[:16]])) and np.all(np.isfinite(f64(dw)[:, cn[:8], :][:, :, ck[:8]]))
+
+
+def _row_scales(sf, row, offs, C):
+    """The scale atom bytes of one row, re-packed as a single-row buffer in the
+    same layout (row 0 of a one-group matrix)."""
+    pitch = (C + 63) // 64
+    if offs is None:
+        pr = row
+    else:
+        m = np.diff(offs)
+        g = int(np.searchsorted(offs, row, side="right") - 1)
+        pr = int(((m[:g] + 127) // 128).sum()) * 128 + (row - int(offs[g]))
+    out = np.zeros(pitch * 512, dtype=np.uint8)
+    for j in range(C // 16):
+        src = ((pr // 128) * pitch + j // 4) * 512 + (pr % 32) * 16 + ((pr % 128) // 32) * 4 + j % 4
+        out[(j // 4) * 512 + j % 4] = sf[src]
+    return out

@@ -178,3 +178,19 @@ def test_dequantisation_error_bounds():
     qT, sfT = oracle.nvfp4_quantize_colwise(x, S, offs)
     dT = oracle.nvfp4_dequantize_colwise(qT, sfT, 133, S, offs)
     assert np.abs(dT - xf).max() <= np.abs(xf).max() * 0.3
+
+
+def test_ungrouped_equals_one_group():
+    """No offsets means one group over all rows (quantise and dequantise, both layouts)."""
+    x = wl.normal_bf16((100, 128), 1.0, 9)
+    S = oracle.nvfp4_tensor_scale(oracle.nvfp4_amax(x))
+    one = np.array([0, 100], dtype=np.int32)
+    for fn in (oracle.nvfp4_quantize_rowwise, oracle.nvfp4_quantize_colwise):
+        a, b = fn(x, S), fn(x, S, one)
+        np.testing.assert_array_equal(a[0], b[0])
+        np.testing.assert_array_equal(a[1], b[1])
+    q, sf = oracle.nvfp4_quantize_rowwise(x, S)
+    np.testing.assert_array_equal(oracle.nvfp4_dequantize_rowwise(q, sf, S), oracle.nvfp4_dequantize_rowwise(q, sf, S, one))
+    qT, sfT = oracle.nvfp4_quantize_colwise(x, S)
+    np.testing.assert_array_equal(oracle.nvfp4_dequantize_colwise(qT, sfT, 100, S),
+                                  oracle.nvfp4_dequantize_colwise(qT, sfT, 100, S, one))
