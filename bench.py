@@ -331,6 +331,7 @@ def run_ours(args, rank, world, local_rank):
         out["e2e"] = e2e(args, mx, w, layers, dev, world)
         out["quantising_epilogue"] = quantising_epilogue(mx, layers[0])
         out["moe_dispatch"] = moe_dispatch(mx, args, pk["hbm_gbs"])
+        out["nvfp4"] = nvfp4_measure(mx, layers[0], fp8_peak, pk["hbm_gbs"])
     return out
 
 
@@ -468,6 +469,61 @@ def moe_dispatch(mx, args, hbm_gbs, iters=20):
             "permute_quantize_frac": round(pq_bytes / (pq_ms * 1e-3) / 1e9 / hbm_gbs, 4),
             "combine_ms": round(cb_ms, 4), "combine_gbs": round(cb_bytes / (cb_ms * 1e-3) / 1e9, 1),
             "combine_frac": round(cb_bytes / (cb_ms * 1e-3) / 1e9 / hbm_gbs, 4)}
+
+
+def nvfp4_measure(mx, L: Linear, fp8_peak, hbm_gbs, iters=20):
+    """The NVFP4 variant of one linear (same shapes and routing): tensor amax,
+    the rowwise / colwise quantisers of X, W and dY, and the three grouped
+    GEMMs on E2M1 x E2M1 block-scaled MMAs.  Timed on its own; the FP4 dense
+    peak is twice the FP8 one (nominal ratio 9 / 4.5 PFLOP/s)."""
+    X, W2, dY, od = L.X, L.W2, L.dY, L.offs
+
+    def t(fn):
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(iters):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+
+    ax, aw, ady = mx.mxfp8_nvfp4_amax(X), mx.mxfp8_nvfp4_amax(W2), mx.mxfp8_nvfp4_amax(dY)
+    xq, xs = mx.mxfp8_nvfp4_quantize_rowwise(X, ax, od)
+    wq, ws = mx.mxfp8_nvfp4_quantize_rowwise(W2, aw)
+    dyq, dys = mx.mxfp8_nvfp4_quantize_rowwise(dY, ady, od)
+    wqT, wsT = mx.mxfp8_nvfp4_quantize_colwise(W2, aw)
+    dyqT, dysT = mx.mxfp8_nvfp4_quantize_colwise(dY, ady, od)
+    xqT, xsT = mx.mxfp8_nvfp4_quantize_colwise(X, ax, od)
+    quant = [lambda: mx.mxfp8_nvfp4_amax(X, ax), lambda: mx.mxfp8_nvfp4_amax(W2, aw),
+             lambda: mx.mxfp8_nvfp4_amax(dY, ady),
+             lambda: mx.mxfp8_nvfp4_quantize_rowwise(X, ax, od, xq, xs),
+             lambda: mx.mxfp8_nvfp4_quantize_rowwise(W2, aw, None, wq, ws),
+             lambda: mx.mxfp8_nvfp4_quantize_rowwise(dY, ady, od, dyq, dys),
+             lambda: mx.mxfp8_nvfp4_quantize_colwise(W2, aw, None, wqT, wsT),
+             lambda: mx.mxfp8_nvfp4_quantize_colwise(dY, ady, od, dyqT, dysT),
+             lambda: mx.mxfp8_nvfp4_quantize_colwise(X, ax, od, xqT, xsT)]
+    q_ms = t(lambda: [f() for f in quant])
+    el = L.X.numel() + L.W2.numel() + L.dY.numel()
+    q_bytes = el * 2 + 2 * el * (2 + 0.5 + 1 / 16)        # amax reads, then two quantisations each
+    fl = L.flops_per_pass()
+    r = {"linear": L.name, "peak_tflops": round(2 * fp8_peak, 1)}
+    for name, fn in (("fwd", lambda: mx.mxfp8_nvfp4_grouped_gemm_fwd(xq, xs, ax, wq, ws, aw, od, L.N, out=L.y,
+                                                                       work=L.work)),
+                     ("dgrad", lambda: mx.mxfp8_nvfp4_grouped_gemm_dgrad(dyq, dys, ady, wqT, wsT, aw, od, L.K,
+                                                                         out=L.dx, work=L.work)),
+                     ("wgrad", lambda: mx.mxfp8_nvfp4_grouped_gemm_wgrad(dyqT, dysT, ady, xqT, xsT, ax, od, L.M,
+                                                                         out=L.dw, work=L.work))):
+        ms = t(fn)
+        r[name] = {"ms": round(ms, 4), "tflops": round(fl / (ms * 1e-3) / 1e12, 1),
+                   "frac": round(fl / (ms * 1e-3) / 1e12 / (2 * fp8_peak), 4)}
+    if mx.mxfp8_get_status(L.work) != 0:
+        raise SystemExit("bench: NVFP4 GEMM reported a device error")
+    r["quantisers"] = {"ms": round(q_ms, 4), "gbs": round(q_bytes / (q_ms * 1e-3) / 1e9, 1),
+                       "frac": round(q_bytes / (q_ms * 1e-3) / 1e9 / hbm_gbs, 4)}
+    return r
 
 
 # ---------------------------------------------------------------- CPU oracle baseline / reference arm
