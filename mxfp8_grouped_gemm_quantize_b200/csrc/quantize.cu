@@ -182,109 +182,325 @@ __global__ void __launch_bounds__(kThreads) quantize_colwise_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Dual: one read of the 128x128 bf16 tile produces both layouts.  The load
-// phase uses the rowwise kernel's thread mapping (four consecutive lanes hold
-// one 32-element row block), so rowwise codes and scales are encoded straight
-// from the loaded registers; the tile then goes to shared memory and the
-// colwise pass proceeds exactly as in quantize_colwise_kernel.
+// Dual: one read of each 128x128 bf16 tile produces both layouts.
+//
+// Persistent CTAs walk a contiguous range of tiles (row block pb, column tile
+// ct), row block by row block, so the group lookup runs once per row block,
+// not per tile.  Tiles stream into shared memory with cp.async (no
+// registers held) through a two-buffer ring: tile k+1 is in flight while
+// tile k is encoded.  Per tile:
+//   rowwise: thread (rsub = t/16, ch = t%16) reads 8 columns of rows
+//            rsub + 16 i; four consecutive lanes form a 32-element block;
+//   colwise: thread (blk = t/64, p = t%64) reduces columns 2p, 2p+1 over rows
+//            32 blk..+31, and the transposed codes leave through a swizzled
+//            stage that reuses the tile's buffer.
+// Block amax is a bf16 max of magnitudes (NaN-propagating, so any Inf/NaN
+// gives exponent field 255 and the NaN scale), and x * 2^-s is a bf16x2
+// multiply: 2^-s is a power of two and |x| * 2^-s < 512, so the product is
+// exact unless it falls below 2^-126, where it is far under E4M3's smallest
+// subnormal and encodes as a signed zero either way.
 // GATHER: row r of the quantised matrix is row gather[r] of x (a token
 // permute fused with the quantisation); a gather index outside [0, src_rows)
 // reads as a zero row.
+constexpr int kDualTile = 128 * 128 * 2;
+constexpr int kDualSmem = 2 * kDualTile + 2 * 512 + 3 * 32 + 16;
+
+__device__ __forceinline__ uint32_t bmax_abs2(uint32_t a, uint32_t b) {
+  uint32_t r;   // per half: max(|a|, |b|), NaN if either is NaN; the sign bits are not meaningful
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Scale byte from a bf16 amax bit pattern (sign ignored): exponent field e,
+// s = e - 135 clamped below at -127 (byte e - 8, at least 0); 255 for Inf/NaN.
+__device__ __forceinline__ uint32_t scale_byte_bf(uint32_t amax_bits) {
+  const uint32_t e = (amax_bits >> 7) & 0xFFu;
+  return e == 0xFFu ? 0xFFu : max(e, 8u) - 8u;
+}
+
+// E4M3 codes of two scaled bf16 pairs a, b: bytes lo(a), hi(a), lo(b), hi(b).
+__device__ __forceinline__ uint32_t e4m3_pairs(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("{\n\t.reg .b32 l0, h0, l1, h1;\n\t.reg .b16 c0, c1;\n\t"
+      "shl.b32 l0, %1, 16;\n\tand.b32 h0, %1, 0xFFFF0000;\n\t"
+      "shl.b32 l1, %2, 16;\n\tand.b32 h1, %2, 0xFFFF0000;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 c0, h0, l0;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 c1, h1, l1;\n\t"
+      "mov.b32 %0, {c0, c1};\n\t}"
+      : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Colwise codes of four scaled bf16 pairs (rows r..r+3 of two columns):
+// lo = bytes lo(a), lo(b), lo(c), lo(d); hi = the high halves.
+__device__ __forceinline__ void e4m3_cols(uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t& lo,
+                                          uint32_t& hi) {
+  asm("{\n\t.reg .b32 a0, a1, a2, a3, b0, b1, b2, b3;\n\t.reg .b16 c0, c1, c2, c3;\n\t"
+      "shl.b32 a0, %2, 16;\n\tshl.b32 a1, %3, 16;\n\tshl.b32 a2, %4, 16;\n\tshl.b32 a3, %5, 16;\n\t"
+      "and.b32 b0, %2, 0xFFFF0000;\n\tand.b32 b1, %3, 0xFFFF0000;\n\t"
+      "and.b32 b2, %4, 0xFFFF0000;\n\tand.b32 b3, %5, 0xFFFF0000;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 c0, a1, a0;\n\tcvt.rn.satfinite.e4m3x2.f32 c1, a3, a2;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 c2, b1, b0;\n\tcvt.rn.satfinite.e4m3x2.f32 c3, b3, b2;\n\t"
+      "mov.b32 %0, {c0, c1};\n\tmov.b32 %1, {c2, c3};\n\t}"
+      : "=r"(lo), "=r"(hi) : "r"(a), "r"(b), "r"(c), "r"(d));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(g), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Real 128-row blocks over all groups (the offsets clamped and made
+// non-decreasing as in warp_find_block).  Warp-cooperative.
+__device__ __forceinline__ int64_t warp_count_blocks(const int32_t* offs, int32_t G, int64_t rows) {
+  const int lane = threadIdx.x & 31;
+  int64_t o_prev = clamp_off(offs, 0, rows), total = 0;
+  for (int32_t base = 0; base < G; base += 32) {
+    const int32_t h = base + lane;
+    int64_t v = (h < G) ? clamp_off(offs, h + 1, rows) : 0;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int64_t u = __shfl_up_sync(0xffffffffu, v, d);
+      if (lane >= d) v = v > u ? v : u;
+    }
+    const int64_t hi = v > o_prev ? v : o_prev;
+    int64_t lo = __shfl_up_sync(0xffffffffu, hi, 1);
+    if (lane == 0) lo = o_prev;
+    int64_t nb = (h < G) ? (hi - lo + 127) / 128 : 0;
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) nb += __shfl_xor_sync(0xffffffffu, nb, d);
+    total += nb;
+    o_prev = __shfl_sync(0xffffffffu, hi, 31);
+  }
+  return total;
+}
+
+struct DualItem {
+  int64_t row0;     // first row of the block (in the quantised matrix)
+  int64_t dst0;     // colwise: first code column
+  int64_t pb;       // padded 128-row block index
+  int32_t nrows;    // real rows (<= 128)
+  int32_t padded;   // colwise: code columns written (multiple of 32, <= 128)
+};
+
+// Warp 0: the row block of padded block index pb (pb < the real block count).
+__device__ __forceinline__ DualItem dual_resolve(const int32_t* offs, int32_t G, int64_t rows, int64_t pb) {
+  const GroupBlock gb = warp_find_block(offs, G, rows, pb);
+  DualItem it;
+  const int64_t local = pb - gb.rb;
+  const int64_t left = gb.m - 128 * local, pad_left = (gb.m + 31) / 32 * 32 - 128 * local;
+  it.row0 = gb.lo + 128 * local;
+  it.dst0 = gb.p + 128 * local;
+  it.pb = pb;
+  it.nrows = static_cast<int32_t>(left < 128 ? left : 128);
+  it.padded = static_cast<int32_t>(pad_left < 128 ? pad_left : 128);
+  if (gb.g < 0) { it.nrows = 0; it.padded = 0; }
+  return it;
+}
+
 template <bool GATHER>
-__global__ void __launch_bounds__(kThreads) quantize_dual_kernel(
+__global__ void __launch_bounds__(kThreads, 3) quantize_dual_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, const int32_t* __restrict__ offs,
     int32_t G, uint8_t* __restrict__ q, uint8_t* __restrict__ sf, int64_t pitch_r,
     uint8_t* __restrict__ qT, int64_t ldT, uint8_t* __restrict__ sfT, int64_t pitch_c,
     const int32_t* __restrict__ gather, int64_t src_rows) {
-  __shared__ __align__(16) uint32_t tile[128 * 64];
-  __shared__ __align__(16) uint8_t atom_r[512];
-  __shared__ __align__(16) uint8_t atom_c[512];
-  BlockRows br;
-  if (!resolve_block(offs, G, rows, &br)) return;
-  const int t = threadIdx.x, ch = t & 15, rsub = t >> 4;
-  const int64_t col0 = static_cast<int64_t>(blockIdx.y) * 128;
-  const bool col_ok = col0 + 8 * ch < cols;
+  extern __shared__ __align__(16) uint8_t dsm[];
+  uint8_t* bufs = dsm;                                           // two 32 KB tiles: [row][64 words]
+  uint8_t* atom_r = dsm + 2 * kDualTile;
+  uint8_t* atom_c = atom_r + 512;
+  DualItem* slot = reinterpret_cast<DualItem*>(atom_c + 512);    // item k's block in slot k % 3
+  int64_t* s_total = reinterpret_cast<int64_t*>(slot + 3);
+  const int t = threadIdx.x, warp = t >> 5, ch = t & 15, rsub = t >> 4;
+  const int32_t nct = static_cast<int32_t>((cols + 127) / 128);
 
-  uint4 v[8];
+  // Tiles (pb, ct) in row-block order, split evenly over the CTAs.
+  if (warp == 0) {
+    const int64_t nbt = warp_count_blocks(offs, G, rows);
+    if (t == 0) *s_total = nbt;
+  }
+  __syncthreads();
+  const int64_t total = *s_total * nct;
+  const int64_t w0 = total * blockIdx.x / gridDim.x, w1 = total * (blockIdx.x + 1) / gridDim.x;
+  if (w0 >= w1) return;
+
+  // warp 0 keeps the last block it resolved
+  DualItem cached;
+  cached.pb = -1;
+  auto resolve_into = [&](int64_t w, int k) {
+    const int64_t pb = w / nct;
+    if (pb != cached.pb) cached = dual_resolve(offs, G, rows, pb);
+    if (t == 0) slot[k % 3] = cached;
+  };
+  if (warp == 0) {
+    resolve_into(w0, 0);
+    if (w0 + 1 < w1) resolve_into(w0 + 1, 1);
+  }
+  __syncthreads();
+
+  // copy issue: thread (rsub, ch) fetches rows rsub + 16 i, 16 bytes at column 8 ch
+  int64_t g_pb = -1;           // GATHER: block whose source rows are cached below
+  int32_t g_src[8];
+  auto issue = [&](const DualItem& it, int64_t w, int b) {
+    const int64_t c = (w % nct) * 128 + 8 * ch;
+    const bool col_ok = c < cols;
+    const uint32_t sbase = smem_addr(bufs + b * kDualTile);
+    if constexpr (GATHER) {
+      if (it.pb != g_pb) {
+        g_pb = it.pb;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int rr = rsub + 16 * i;
-    v[i] = make_uint4(0, 0, 0, 0);
-    if (rr < br.nrows && col_ok) {
-      int64_t src = br.row0 + rr;
-      if constexpr (GATHER) src = __ldg(gather + src);
-      if (!GATHER || (src >= 0 && src < src_rows)) v[i] = ld_stream(x + src * cols + col0 + 8 * ch);
+        for (int i = 0; i < 8; ++i) {
+          const int rr = rsub + 16 * i;
+          int32_t src = -1;
+          if (rr < it.nrows) {
+            src = __ldg(gather + it.row0 + rr);
+            if (src >= src_rows) src = -1;
+          }
+          g_src[i] = src;
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int rr = rsub + 16 * i;
+      int64_t src = it.row0 + rr;
+      bool ok = rr < it.nrows && col_ok;
+      if constexpr (GATHER) {
+        src = g_src[i];
+        ok = ok && src >= 0;
+      }
+      const uint16_t* gp = ok ? x + src * cols + c : x;
+      cp_async16(sbase + (rr * 16 + ch) * 16, gp, ok ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+
+  {
+    const DualItem it0 = slot[0];
+    issue(it0, w0, 0);
+  }
+
+  for (int64_t w = w0; w < w1; ++w) {
+    const int k = static_cast<int>(w - w0), b = k & 1;
+    cp_async_wait_all();
+    __syncthreads();   // tile k landed for every thread; buffer b^1 and the atoms are free
+    const DualItem it = slot[k % 3];
+    if (w + 1 < w1) {
+      const DualItem nx = slot[(k + 1) % 3];
+      issue(nx, w + 1, b ^ 1);
+    }
+    if (warp == 0 && w + 2 < w1) resolve_into(w + 2, k + 2);
+
+    const int64_t ct = w % nct, col0 = ct * 128;
+    const uint4* tile4 = reinterpret_cast<const uint4*>(bufs + b * kDualTile);
+    const uint32_t* tile = reinterpret_cast<const uint32_t*>(tile4);
+
+    // ---- rowwise
+    const bool col_ok = col0 + 8 * ch < cols;
+#pragma unroll 4
+    for (int i = 0; i < 8; ++i) {
+      const int rr = rsub + 16 * i;
+      const uint4 v = tile4[rr * 16 + ch];
+      uint32_t a = bmax_abs2(bmax_abs2(v.x, v.y), bmax_abs2(v.z, v.w));
+      a = bmax_abs2(a, __shfl_xor_sync(0xffffffffu, a, 1));
+      a = bmax_abs2(a, __shfl_xor_sync(0xffffffffu, a, 2));
+      a = bmax_abs2(a, __byte_perm(a, 0, 0x1032));
+      const uint32_t sb = scale_byte_bf(a);
+      const uint32_t fm = (254u - sb) * 0x00800080u;   // 2^-s in both bf16 halves
+      uint2 o;
+      o.x = e4m3_pairs(bmul2(v.x, fm), bmul2(v.y, fm));
+      o.y = e4m3_pairs(bmul2(v.z, fm), bmul2(v.w, fm));
+      if (sb == 0xFFu) o = make_uint2(0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      if (rr < it.nrows && col_ok) *reinterpret_cast<uint2*>(q + (it.row0 + rr) * cols + col0 + 8 * ch) = o;
+      if ((ch & 3) == 0) atom_r[(rr & 31) * 16 + (rr >> 5) * 4 + (ch >> 2)] = static_cast<uint8_t>(sb);
+    }
+
+    // ---- colwise
+    const int blk = t >> 6, p = t & 63;
+    uint32_t wv[32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) wv[r] = tile[(32 * blk + r) * 64 + p];
+    uint32_t mx = wv[0];
+#pragma unroll
+    for (int r = 1; r < 32; ++r) mx = bmax_abs2(mx, wv[r]);
+    const uint32_t sb_lo = scale_byte_bf(mx), sb_hi = scale_byte_bf(mx >> 16);
+    const uint32_t fm = (((254u - sb_lo) & 0xFFu) << 7) | (((254u - sb_hi) & 0xFFu) << 23);   // (2^-s_lo, 2^-s_hi)
+    uint32_t olo[8], ohi[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      e4m3_cols(bmul2(wv[4 * j], fm), bmul2(wv[4 * j + 1], fm), bmul2(wv[4 * j + 2], fm), bmul2(wv[4 * j + 3], fm),
+                olo[j], ohi[j]);
+    if (sb_lo == 0xFFu || sb_hi == 0xFFu) {
+      const int vrows = min(32, max(0, it.nrows - 32 * blk));   // real rows of this 32-block
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (sb_lo == 0xFFu) olo[j] = nan_codes4(j, vrows);
+        if (sb_hi == 0xFFu) ohi[j] = nan_codes4(j, vrows);
+      }
+    }
+    __syncthreads();   // every thread has read the tile: it becomes the code stage; atom_r is complete
+
+    if (t < 32) {
+      const int64_t a = it.pb * pitch_r + ct;
+      reinterpret_cast<uint4*>(sf + a * 512)[t] = reinterpret_cast<const uint4*>(atom_r)[t];
+    }
+    uint4* stage = reinterpret_cast<uint4*>(bufs + b * kDualTile);   // [128 code rows][8 chunks of 16 B]
+    const int sw = p & 7;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int chunk = (2 * blk + h) ^ sw;
+      stage[(2 * p) * 8 + chunk] = make_uint4(olo[4 * h], olo[4 * h + 1], olo[4 * h + 2], olo[4 * h + 3]);
+      stage[(2 * p + 1) * 8 + chunk] = make_uint4(ohi[4 * h], ohi[4 * h + 1], ohi[4 * h + 2], ohi[4 * h + 3]);
+    }
+    {
+      const int r0 = 2 * p, r1 = 2 * p + 1;
+      atom_c[(r0 & 31) * 16 + (r0 >> 5) * 4 + blk] = static_cast<uint8_t>(sb_lo);
+      atom_c[(r1 & 31) * 16 + (r1 >> 5) * 4 + blk] = static_cast<uint8_t>(sb_hi);
+    }
+    __syncthreads();
+
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int id = t + kThreads * i, c = id >> 3, j = id & 7;
+      if (col0 + c < cols && 16 * j < it.padded)
+        *reinterpret_cast<uint4*>(qT + (col0 + c) * ldT + it.dst0 + 16 * j) = stage[c * 8 + (j ^ ((c >> 1) & 7))];
+    }
+    if (t >= 32 && t < 64) {
+      const int64_t a = ct * pitch_c + it.pb;
+      reinterpret_cast<uint4*>(sfT + a * 512)[t - 32] = reinterpret_cast<const uint4*>(atom_c)[t - 32];
     }
   }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int rr = rsub + 16 * i;
-    uint32_t a = amax_bits8(v[i]);
-    a = max(a, __shfl_xor_sync(0xffffffffu, a, 1));
-    a = max(a, __shfl_xor_sync(0xffffffffu, a, 2));
-    const uint32_t sb = scale_byte(a);
-    if (rr < br.nrows && col_ok)
-      *reinterpret_cast<uint2*>(q + (br.row0 + rr) * cols + col0 + 8 * ch) = encode8(v[i], sb);
-    if ((ch & 3) == 0) atom_r[(rr & 31) * 16 + (rr >> 5) * 4 + (ch >> 2)] = static_cast<uint8_t>(sb);
-    reinterpret_cast<uint4*>(tile)[rr * 16 + ch] = v[i];
-  }
-  __syncthreads();
-  if (t < 32) {
-    const int64_t a = static_cast<int64_t>(blockIdx.x) * pitch_r + blockIdx.y;
-    reinterpret_cast<uint4*>(sf + a * 512)[t] = reinterpret_cast<const uint4*>(atom_r)[t];
-  }
+}
 
-  const int blk = t >> 6, p = t & 63;
-  uint32_t w[32];
-  uint32_t mx = 0;
-#pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    w[r] = tile[(32 * blk + r) * 64 + p];
-    mx = __vmaxu2(mx, w[r] & 0x7FFF7FFFu);
+// Grid of the persistent dual kernel: as many CTAs as fit on the device (at
+// most one per tile of the padded bound).
+template <bool GATHER>
+cudaError_t dual_grid(int64_t tiles, int* grid) {
+  static int per_sm[64][2] = {};
+  static int sms[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (per_sm[dev][GATHER] == 0) {
+    e = cudaFuncSetAttribute(quantize_dual_kernel<GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDualSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quantize_dual_kernel<GATHER>, kThreads, kDualSmem);
+    if (e != cudaSuccess) return e;
+    per_sm[dev][GATHER] = n > 0 ? n : 1;
   }
-  const uint32_t sb_lo = scale_byte(mx & 0xFFFFu), sb_hi = scale_byte(mx >> 16);
-  const int vrows = min(32, max(0, br.nrows - 32 * blk));   // real rows of this 32-block
-  uint32_t olo[8], ohi[8];
-  {
-    const float flo = inv_scale(sb_lo == 0xFFu ? 0u : sb_lo);
-    const float fhi = inv_scale(sb_hi == 0xFFu ? 0u : sb_hi);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t a0 = cvt_e4m3x2(__fmul_rn(bf_lo(w[4 * j]), flo), __fmul_rn(bf_lo(w[4 * j + 1]), flo));
-      const uint32_t a1 = cvt_e4m3x2(__fmul_rn(bf_lo(w[4 * j + 2]), flo), __fmul_rn(bf_lo(w[4 * j + 3]), flo));
-      const uint32_t b0 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * j]), fhi), __fmul_rn(bf_hi(w[4 * j + 1]), fhi));
-      const uint32_t b1 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * j + 2]), fhi), __fmul_rn(bf_hi(w[4 * j + 3]), fhi));
-      olo[j] = sb_lo == 0xFFu ? nan_codes4(j, vrows) : (a0 | (a1 << 16));
-      ohi[j] = sb_hi == 0xFFu ? nan_codes4(j, vrows) : (b0 | (b1 << 16));
-    }
-  }
-  __syncthreads();
-
-  uint4* stage = reinterpret_cast<uint4*>(tile);
-  const int sw = p & 7;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int chunk = (2 * blk + h) ^ sw;
-    stage[(2 * p) * 8 + chunk] = make_uint4(olo[4 * h], olo[4 * h + 1], olo[4 * h + 2], olo[4 * h + 3]);
-    stage[(2 * p + 1) * 8 + chunk] = make_uint4(ohi[4 * h], ohi[4 * h + 1], ohi[4 * h + 2], ohi[4 * h + 3]);
-  }
-  {
-    const int r0 = 2 * p, r1 = 2 * p + 1;
-    atom_c[(r0 & 31) * 16 + (r0 >> 5) * 4 + blk] = static_cast<uint8_t>(sb_lo);
-    atom_c[(r1 & 31) * 16 + (r1 >> 5) * 4 + blk] = static_cast<uint8_t>(sb_hi);
-  }
-  __syncthreads();
-
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int id = t + kThreads * i, c = id >> 3, j = id & 7;
-    if (col0 + c < cols && 16 * j < br.padded)
-      *reinterpret_cast<uint4*>(qT + (col0 + c) * ldT + br.dst0 + 16 * j) = stage[c * 8 + (j ^ ((c >> 1) & 7))];
-  }
-  if (t < 32) {
-    const int64_t a = static_cast<int64_t>(blockIdx.y) * pitch_c + blockIdx.x;
-    reinterpret_cast<uint4*>(sfT + a * 512)[t] = reinterpret_cast<const uint4*>(atom_c)[t];
-  }
+  const int64_t cap = int64_t(sms[dev]) * per_sm[dev][GATHER];
+  *grid = static_cast<int>(tiles < cap ? tiles : cap);
+  return cudaSuccess;
 }
 
 int64_t block_bound(int64_t rows, int32_t G) { return rows == 0 ? 0 : (rows + 127) / 128 + G - 1; }
@@ -316,9 +532,11 @@ cudaError_t launch_quantize_dual(const uint16_t* x, int64_t rows, int64_t cols, 
                                  cudaStream_t stream) {
   const int64_t nb = block_bound(rows, G);
   if (nb == 0) return cudaSuccess;
-  const dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>((cols + 127) / 128));
-  quantize_dual_kernel<false><<<grid, kThreads, 0, stream>>>(x, rows, cols, offs, G, q, sf, (cols + 127) / 128, qT,
-                                                              ldT, sfT, nb, nullptr, rows);
+  int grid = 0;
+  cudaError_t e = dual_grid<false>(nb * ((cols + 127) / 128), &grid);
+  if (e != cudaSuccess) return e;
+  quantize_dual_kernel<false><<<grid, kThreads, kDualSmem, stream>>>(x, rows, cols, offs, G, q, sf, (cols + 127) / 128,
+                                                                    qT, ldT, sfT, nb, nullptr, rows);
   return cudaGetLastError();
 }
 
@@ -327,9 +545,11 @@ cudaError_t launch_permute_quantize_dual(const uint16_t* x, int64_t src_rows, in
                                          uint8_t* qT, int64_t ldT, uint8_t* sfT, cudaStream_t stream) {
   const int64_t nb = block_bound(rows, G);
   if (nb == 0) return cudaSuccess;
-  const dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>((cols + 127) / 128));
-  quantize_dual_kernel<true><<<grid, kThreads, 0, stream>>>(x, rows, cols, offs, G, q, sf, (cols + 127) / 128, qT,
-                                                             ldT, sfT, nb, perm, src_rows);
+  int grid = 0;
+  cudaError_t e = dual_grid<true>(nb * ((cols + 127) / 128), &grid);
+  if (e != cudaSuccess) return e;
+  quantize_dual_kernel<true><<<grid, kThreads, kDualSmem, stream>>>(x, rows, cols, offs, G, q, sf, (cols + 127) / 128,
+                                                                   qT, ldT, sfT, nb, perm, src_rows);
   return cudaGetLastError();
 }
 
