@@ -8,11 +8,12 @@
 //
 // The kernels are HBM-bound (2 bytes read, 1 + 1/32 written per element and
 // layout; the dual kernel writes both layouts from one read, 4 + 1/16 bytes).
-// A CTA owns one 128-row x 128-column tile, i.e. exactly one 512-byte scale
-// atom of the tcgen05 scale-factor layout, so scales leave the CTA as 32
-// coalesced 16-byte stores.  Rows are read with 16-byte loads, block amax is
-// an integer max over the bf16 magnitude bits (packed, two per instruction),
-// and codes come from the hardware E4M3x2 conversion.
+// The unit of work is a 128-row x 128-column tile, i.e. exactly one 512-byte
+// scale atom of the tcgen05 scale-factor layout, so scales leave as 32
+// coalesced 16-byte stores.  The rowwise and colwise kernels run one CTA per
+// tile; the dual kernel is persistent (see below).  Rows are read with
+// 16-byte loads, block amax is a max over the bf16 magnitudes (packed, two
+// per instruction), and codes come from the hardware E4M3x2 conversion.
 #include <cuda_runtime.h>
 
 #include "codec.cuh"
@@ -203,7 +204,7 @@ __global__ void __launch_bounds__(kThreads) quantize_colwise_kernel(
 // permute fused with the quantisation); a gather index outside [0, src_rows)
 // reads as a zero row.
 constexpr int kDualTile = 128 * 128 * 2;
-constexpr int kDualSmem = 2 * kDualTile + 2 * 512 + 3 * 32 + 16;
+constexpr int kDualSmem = 2 * kDualTile + 2 * 512 + 3 * 32 + 16 + 3 * 128 * 4;
 
 __device__ __forceinline__ uint32_t bmax_abs2(uint32_t a, uint32_t b) {
   uint32_t r;   // per half: max(|a|, |b|), NaN if either is NaN; the sign bits are not meaningful
@@ -317,6 +318,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_dual_kernel(
   uint8_t* atom_c = atom_r + 512;
   DualItem* slot = reinterpret_cast<DualItem*>(atom_c + 512);    // item k's block in slot k % 3
   int64_t* s_total = reinterpret_cast<int64_t*>(slot + 3);
+  int32_t* s_src = reinterpret_cast<int32_t*>(s_total + 2);      // GATHER: source rows of slot j at [128 j]
   const int t = threadIdx.x, warp = t >> 5, ch = t & 15, rsub = t >> 4;
   const int32_t nct = static_cast<int32_t>((cols + 127) / 128);
 
@@ -330,13 +332,33 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_dual_kernel(
   const int64_t w0 = total * blockIdx.x / gridDim.x, w1 = total * (blockIdx.x + 1) / gridDim.x;
   if (w0 >= w1) return;
 
-  // warp 0 keeps the last block it resolved
+  // warp 0 resolves item k into slot k % 3, one item ahead of its copies,
+  // keeping the last block it resolved; GATHER: it also stages the block's
+  // source rows (-1 = zero row), reusing the previous slot's when the block
+  // is unchanged.
   DualItem cached;
   cached.pb = -1;
   auto resolve_into = [&](int64_t w, int k) {
     const int64_t pb = w / nct;
-    if (pb != cached.pb) cached = dual_resolve(offs, G, rows, pb);
+    const bool same = pb == cached.pb;
+    if (!same) cached = dual_resolve(offs, G, rows, pb);
     if (t == 0) slot[k % 3] = cached;
+    if constexpr (GATHER) {
+      int32_t* dst = s_src + 128 * (k % 3);
+      const int32_t* prev = s_src + 128 * ((k + 2) % 3);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int rr = t + 32 * j;
+        int32_t src = -1;
+        if (same) {
+          src = prev[rr];
+        } else if (rr < cached.nrows) {
+          src = __ldg(gather + cached.row0 + rr);
+          if (src >= src_rows) src = -1;
+        }
+        dst[rr] = src;
+      }
+    }
   };
   if (warp == 0) {
     resolve_into(w0, 0);
@@ -345,34 +367,18 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_dual_kernel(
   __syncthreads();
 
   // copy issue: thread (rsub, ch) fetches rows rsub + 16 i, 16 bytes at column 8 ch
-  int64_t g_pb = -1;           // GATHER: block whose source rows are cached below
-  int32_t g_src[8];
-  auto issue = [&](const DualItem& it, int64_t w, int b) {
+  auto issue = [&](const DualItem& it, int64_t w, int k, int b) {
     const int64_t c = (w % nct) * 128 + 8 * ch;
     const bool col_ok = c < cols;
     const uint32_t sbase = smem_addr(bufs + b * kDualTile);
-    if constexpr (GATHER) {
-      if (it.pb != g_pb) {
-        g_pb = it.pb;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = rsub + 16 * i;
-          int32_t src = -1;
-          if (rr < it.nrows) {
-            src = __ldg(gather + it.row0 + rr);
-            if (src >= src_rows) src = -1;
-          }
-          g_src[i] = src;
-        }
-      }
-    }
+    const int32_t* srcs = s_src + 128 * (k % 3);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int rr = rsub + 16 * i;
       int64_t src = it.row0 + rr;
       bool ok = rr < it.nrows && col_ok;
       if constexpr (GATHER) {
-        src = g_src[i];
+        src = srcs[rr];
         ok = ok && src >= 0;
       }
       const uint16_t* gp = ok ? x + src * cols + c : x;
@@ -383,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_dual_kernel(
 
   {
     const DualItem it0 = slot[0];
-    issue(it0, w0, 0);
+    issue(it0, w0, 0, 0);
   }
 
   for (int64_t w = w0; w < w1; ++w) {
@@ -393,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_dual_kernel(
     const DualItem it = slot[k % 3];
     if (w + 1 < w1) {
       const DualItem nx = slot[(k + 1) % 3];
-      issue(nx, w + 1, b ^ 1);
+      issue(nx, w + 1, k + 1, b ^ 1);
     }
     if (warp == 0 && w + 2 < w1) resolve_into(w + 2, k + 2);
 
