@@ -332,7 +332,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     if (lane == 0) {
       for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
       mbar_init(acc_full, 1);
-      mbar_init(acc_empty, CG * 4 * 32);
+      mbar_init(acc_empty, CG * 4);   // one arrival per epilogue warp
       mbar_init(drain_bar, 1);
       fence_barrier_init();
       prefetch_tmap(&tmA);
@@ -599,12 +599,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       // Accumulator 0's last OV chunks are accumulator 1's first OV chunks:
       // drain those first, then release the accumulator to the MMA issuer.
       auto chunk_of = [&](int ci) { return buf == 0 ? (ci + 4 - C::OV) & 3 : ci; };
+      // Every lane's tcgen05.ld has completed (wait::ld) before the warp
+      // syncs; one lane then arrives for the warp.
       auto release = [&]() {
         tc_fence_before();
-        if constexpr (CG == 2) {
-          if (leader) mbar_arrive(acc_empty); else mbar_arrive_cluster(acc_empty, 0);
-        } else {
-          mbar_arrive(acc_empty);
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (CG == 2) {
+            if (leader) mbar_arrive(acc_empty); else mbar_arrive_cluster(acc_empty, 0);
+          } else {
+            mbar_arrive(acc_empty);
+          }
         }
       };
       uint32_t ra0[32], ra1[32], rb0[32], rb1[32];
