@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(wl.WORKLOADS))
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quantiser", default="dual", choices=["dual", "separate"],
                     help="dual: one fused kernel writes both layouts of X, W and dY")
@@ -226,6 +226,20 @@ class Linear:
         ]
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks: a job's time is its slowest rank's."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, ms: float, world: int) -> float:
+    """Throughput of the whole job: every rank's units over the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def run_ours(args, rank, world, local_rank):
     import mxfp8_grouped_gemm_quantize_b200 as mx
     torch.cuda.set_device(local_rank)
@@ -279,12 +293,9 @@ def run_ours(args, rank, world, local_rank):
     for s in range(K):
         for i, (kind, _) in enumerate(calls):
             per_kind.setdefault(kind, []).append(ev[s][i].elapsed_time(ev[s][i + 1]))
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / K
-    value = world * step_flops / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(step_flops, ms_step, world)
 
     pk = peaks()
     fp8_peak = pk["bf16"] * FP8_OVER_BF16
@@ -338,46 +349,77 @@ def run_ours(args, rank, world, local_rank):
 def e2e(args, mx, w, layers, dev, world):
     """Same metric through the public API with host buffers: every step copies
     the bf16 inputs (X, W, dY of both linears) and the offsets from pinned host
-    memory, runs the path and copies Y, dX and dW back to pinned host memory."""
-    stream = torch.cuda.current_stream()
-    host_in, host_out = [], []
-    for L in layers:
-        host_in += [(L.X, L.X.cpu().pin_memory()), (L.W2, L.W2.cpu().pin_memory()),
-                    (L.dY, L.dY.cpu().pin_memory()), (L.offs, L.offs.cpu().pin_memory())]
-        host_out += [(L.y, torch.empty_like(L.y, device="cpu").pin_memory()),
-                     (L.dx, torch.empty_like(L.dx, device="cpu").pin_memory()),
-                     (L.dw, torch.empty_like(L.dw, device="cpu").pin_memory())]
+    memory, runs the path and copies Y, dX and dW back to pinned host memory.
+    Steps are pipelined the way a training loop prefetches its next batch:
+    host-to-device copies on one stream, the path on the current stream and
+    device-to-host copies on a third, with two device buffer sets, so step
+    k+1's inputs and step k-1's outputs cross PCIe (one direction each) while
+    step k computes.  The timed region spans all K steps' copies and compute."""
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    in_names, out_names = ("X", "W2", "dY", "offs"), ("y", "dx", "dw")
+    sets = []   # per buffer set: {layer index: {name: device tensor}}
+    for b in range(2):
+        sets.append([{n: (getattr(L, n) if b == 0 else torch.empty_like(getattr(L, n)))
+                      for n in in_names + out_names} for L in layers])
+    host_in = [{n: getattr(L, n).cpu().pin_memory() for n in in_names} for L in layers]
+    host_out = [{n: torch.empty_like(getattr(L, n), device="cpu").pin_memory() for n in out_names} for L in layers]
     calls = [fn for L in layers for _, fn in L.launches()]
-    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
-    d2h = sum(h.numel() * h.element_size() for _, h in host_out)
+    h2d = sum(h.numel() * h.element_size() for d in host_in for h in d.values())
+    d2h = sum(h.numel() * h.element_size() for d in host_out for h in d.values())
+    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "comp", "out")}
+    used = [False, False]
 
-    def step():
-        for d, h in host_in:
-            d.copy_(h, non_blocking=True)
+    def step(k):
+        b = k % 2
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(ev["comp"][b])      # set b's inputs were read by step k-2
+            for i, d in enumerate(host_in):
+                for n, h in d.items():
+                    sets[b][i][n].copy_(h, non_blocking=True)
+            ev["in"][b].record(s_in)
+        comp.wait_event(ev["in"][b])
+        if used[b]:
+            comp.wait_event(ev["out"][b])           # set b's outputs were copied out by step k-2
+        for i, L in enumerate(layers):
+            for n in in_names + out_names:
+                setattr(L, n, sets[b][i][n])
         for fn in calls:
             fn()
-        for d, h in host_out:
-            h.copy_(d, non_blocking=True)
+        ev["comp"][b].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev["comp"][b])
+            for i, d in enumerate(host_out):
+                for n, h in d.items():
+                    h.copy_(sets[b][i][n], non_blocking=True)
+            ev["out"][b].record(s_out)
+        used[b] = True
 
-    step()
+    for k in range(2):
+        step(k)
     torch.cuda.synchronize()
     K = max(1, args.e2e_steps)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
-    a.record(stream)
-    for _ in range(K):
-        step()
-    b.record(stream)
+    a.record(comp)
+    s_in.wait_event(a)
+    s_out.wait_event(a)
+    for k in range(K):
+        step(k)
+    comp.wait_event(ev["out"][(K - 1) % 2])
+    z.record(comp)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / K
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = a.elapsed_time(z) / K
+    for i, L in enumerate(layers):
+        for n in in_names + out_names:
+            setattr(L, n, sets[0][i][n])
+    ms = max_over_ranks(ms, world, dev)
     flops = 3 * sum(L.flops_per_pass() for L in layers)
-    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": UNIT, "ms_per_step": round(ms, 3),
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": K}
+    return {"value": round(whole_job_tflops(flops, ms, world), 2), "unit": UNIT, "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": K,
+            "pipelined": "h2d / compute / d2h on three streams, two device buffer sets"}
 
 
 def quantising_epilogue(mx, L: Linear, iters=20):
