@@ -113,37 +113,39 @@ __global__ void plan_scatter_kernel(const int32_t* __restrict__ idx, int64_t n, 
   }
 }
 
-// Nearest-even bf16 bits of a double, from its bit fields: keep 8
-// significant bits (the quantum is fixed at 2^-133 below 2^-126), round the
-// dropped bits half to even, carry into the exponent, overflow to Inf.
+// Nearest-even bf16 bits of a double (one rounding: ties to even, overflow
+// to Inf, bf16 subnormals kept) by the hardware conversion; a NaN becomes the
+// quiet NaN 0x7FC0 with its sign, the definition's pattern.
 __device__ __forceinline__ uint16_t bf16_bits_rne(double v) {
-  const uint64_t b = static_cast<uint64_t>(__double_as_longlong(v));
-  const uint16_t sign = static_cast<uint16_t>((b >> 48) & 0x8000u);
-  const uint64_t mag = b & 0x7FFFFFFFFFFFFFFFull;
-  if (mag > 0x7FF0000000000000ull) return static_cast<uint16_t>(sign | 0x7FC0u);   // NaN
-  if (mag == 0x7FF0000000000000ull) return static_cast<uint16_t>(sign | 0x7F80u);  // Inf
-  const int bexp = static_cast<int>(mag >> 52);
-  if (bexp == 0) return sign;                  // double subnormal: far below half the bf16 quantum
-  const uint64_t sig = (mag & 0xFFFFFFFFFFFFFull) | (1ull << 52);   // value = sig * 2^(e2 - 52)
-  const int e2 = bexp - 1023;
-  const int qe = (e2 > -126 ? e2 : -126) - 7;  // exponent of the bf16 quantum at this magnitude
-  const int shift = qe - (e2 - 52);            // low bits of sig below the quantum (>= 45)
-  if (shift >= 64) return sign;                // value < quantum / 2^11
-  uint64_t keep = sig >> shift;
-  const uint64_t rem = sig & ((1ull << shift) - 1ull), half = 1ull << (shift - 1);
-  if (rem > half || (rem == half && (keep & 1ull))) ++keep;
-  // value = keep * 2^qe, keep <= 256
-  if (qe == -133 && keep < 128) return static_cast<uint16_t>(sign | keep);   // bf16 subnormal
-  int be = qe + 7 + 127;                       // biased exponent for keep in [128, 256)
-  if (keep == 256) { keep = 128; ++be; }
-  if (be >= 255) return static_cast<uint16_t>(sign | 0x7F80u);
-  return static_cast<uint16_t>(sign | (be << 7) | static_cast<int>(keep - 128));
+  uint16_t r;
+  asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(r) : "d"(v));
+  if (v != v) r = static_cast<uint16_t>(((__double_as_longlong(v) >> 48) & 0x8000) | 0x7FC0);
+  return r;
 }
 
 __device__ __forceinline__ double bf16_lo(uint32_t w) { return static_cast<double>(__uint_as_float(w << 16)); }
 __device__ __forceinline__ double bf16_hi(uint32_t w) { return static_cast<double>(__uint_as_float(w & 0xFFFF0000u)); }
 
 // One thread: 8 consecutive columns of one token.
+// Adds slot j's contribution w_j * yp[r_j] to the fp64 accumulators.  The
+// product of an fp32 weight and a bf16 value has at most 32 significant bits,
+// so it is exact in fp64 and one fused multiply-add rounds exactly as the
+// separate multiply and add of the definition do.
+__device__ __forceinline__ void combine_add(double (&acc)[8], double wj, const uint4& v) {
+  acc[0] = __fma_rn(wj, bf16_lo(v.x), acc[0]);
+  acc[1] = __fma_rn(wj, bf16_hi(v.x), acc[1]);
+  acc[2] = __fma_rn(wj, bf16_lo(v.y), acc[2]);
+  acc[3] = __fma_rn(wj, bf16_hi(v.y), acc[3]);
+  acc[4] = __fma_rn(wj, bf16_lo(v.z), acc[4]);
+  acc[5] = __fma_rn(wj, bf16_hi(v.z), acc[5]);
+  acc[6] = __fma_rn(wj, bf16_lo(v.w), acc[6]);
+  acc[7] = __fma_rn(wj, bf16_hi(v.w), acc[7]);
+}
+
+// Slots are summed in order 0..k-1; an unrouted slot is skipped (not added
+// as zero, which would turn -0 into +0).  The sum is bound by fp64
+// arithmetic, not by memory, so each thread keeps one slot's row in flight
+// and the SM keeps many threads resident.
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const uint16_t* __restrict__ yp, int64_t rows, int64_t cols, const int32_t* __restrict__ inv,
     const float* __restrict__ w, int64_t T, int32_t k, uint16_t* __restrict__ y) {
@@ -156,16 +158,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     for (int32_t j = 0; j < k; ++j) {
       const int32_t r = __ldg(inv + t * k + j);
       if (r < 0 || r >= rows) continue;            // an unrouted slot contributes nothing
-      const double wj = static_cast<double>(__ldg(w + t * k + j));
       const uint4 v = __ldg(reinterpret_cast<const uint4*>(yp + static_cast<int64_t>(r) * cols + c));
-      acc[0] = __dadd_rn(acc[0], __dmul_rn(wj, bf16_lo(v.x)));
-      acc[1] = __dadd_rn(acc[1], __dmul_rn(wj, bf16_hi(v.x)));
-      acc[2] = __dadd_rn(acc[2], __dmul_rn(wj, bf16_lo(v.y)));
-      acc[3] = __dadd_rn(acc[3], __dmul_rn(wj, bf16_hi(v.y)));
-      acc[4] = __dadd_rn(acc[4], __dmul_rn(wj, bf16_lo(v.z)));
-      acc[5] = __dadd_rn(acc[5], __dmul_rn(wj, bf16_hi(v.z)));
-      acc[6] = __dadd_rn(acc[6], __dmul_rn(wj, bf16_lo(v.w)));
-      acc[7] = __dadd_rn(acc[7], __dmul_rn(wj, bf16_hi(v.w)));
+      combine_add(acc, static_cast<double>(__ldg(w + t * k + j)), v);
     }
     auto pack = [](double lo, double hi) {
       return static_cast<uint32_t>(bf16_bits_rne(lo)) | (static_cast<uint32_t>(bf16_bits_rne(hi)) << 16);
