@@ -190,8 +190,8 @@ __global__ void __launch_bounds__(kThreads) quantize_colwise_kernel(
 // not per tile.  Tiles stream into shared memory with cp.async (no
 // registers held) through a two-buffer ring: tile k+1 is in flight while
 // tile k is encoded.  Per tile:
-//   rowwise: thread (rsub = t/16, ch = t%16) reads 8 columns of rows
-//            rsub + 16 i; four consecutive lanes form a 32-element block;
+//   rowwise: thread (rq = t/8, cq = t%8) reads 16 columns of rows rq + 32 i;
+//            two consecutive lanes form a 32-element block;
 //   colwise: thread (blk = t/64, p = t%64) reduces columns 2p, 2p+1 over rows
 //            32 blk..+31, and the transposed codes leave through a swizzled
 //            stage that reuses the tile's buffer.
@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_dual_kernel(
   DualItem* slot = reinterpret_cast<DualItem*>(atom_c + 512);    // item k's block in slot k % 3
   int64_t* s_total = reinterpret_cast<int64_t*>(slot + 3);
   int32_t* s_src = reinterpret_cast<int32_t*>(s_total + 2);      // GATHER: source rows of slot j at [128 j]
-  const int t = threadIdx.x, warp = t >> 5, ch = t & 15, rsub = t >> 4;
+  const int t = threadIdx.x, warp = t >> 5;
   const int32_t nct = static_cast<int32_t>((cols + 127) / 128);
 
   // Tiles (pb, ct) in row-block order, split evenly over the CTAs.
@@ -366,43 +366,32 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_dual_kernel(
   }
   __syncthreads();
 
-  // Thread mappings.  Plain rows (HBM-bound): thread (rsub = t/16, ch = t%16)
-  // copies and encodes 8 columns of rows rsub + 16 i; four lanes form a
-  // 32-element block.  Gathered rows (the source usually sits in L2, so the
-  // kernel is instruction-bound): thread (rq = t/8, cq = t%8) encodes 16
-  // columns of rows rq + 32 i (two lanes per block, 16-byte code stores) and
-  // copies chunks cq and cq + 8 of those rows; chunk c of a tile row is then
-  // stored at slot c ^ (c / 8 % 2), which keeps the 16-byte row reads and the
-  // 4-byte column reads conflict-free.  (The wide mapping measured 15 %
-  // faster on gathered rows and 4-6 % slower on plain HBM-bound ones.)
+  // Thread mapping: thread (rq = t/8, cq = t%8) encodes 16 columns of rows
+  // rq + 32 i, i = 0..3 (two lanes per 32-element block, 16-byte code stores),
+  // and copies 16-byte chunks cq and cq + 8 of those rows, so every copy
+  // instruction of a warp reads whole 128-byte row segments.  Chunk c of a
+  // tile row is stored at slot c ^ (c / 8 % 2), which keeps the 16-byte row
+  // reads and the 4-byte column reads conflict-free.  (Against 8 columns per
+  // thread and four lanes per block, this mapping issues fewer instructions
+  // per element: 3 % faster in the power-capped training step and 15 % on
+  // gathered rows, whose source sits in L2; in isolation at full clock on
+  // plain HBM-bound rows it measured up to 5 % slower.)
   const int rq = t >> 3, cq = t & 7;
   const int sl0 = (2 * cq) ^ (cq >> 2), sl1 = (2 * cq + 1) ^ (cq >> 2), cs1 = (cq + 8) ^ 1;
   auto issue = [&](const DualItem& it, int64_t w, int k, int b) {
     const uint32_t sbase = smem_addr(bufs + b * kDualTile);
     const int32_t* srcs = s_src + 128 * (k % 3);
-    if constexpr (GATHER) {
-      const int64_t c = (w % nct) * 128 + 8 * cq;
-      const bool ok0 = c < cols, ok1 = c + 64 < cols;
+    const int64_t c = (w % nct) * 128 + 8 * cq;
+    const bool ok0 = c < cols, ok1 = c + 64 < cols;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int rr = rq + 32 * i;
-        const int64_t src = srcs[rr];
-        const bool ok = rr < it.nrows && src >= 0;
-        const uint16_t* gp = ok ? x + src * cols + c : x;
-        const uint32_t sa = sbase + rr * 256;
-        cp_async16(sa + cq * 16, ok && ok0 ? gp : x, ok && ok0 ? 16u : 0u);
-        cp_async16(sa + cs1 * 16, ok && ok1 ? gp + 64 : x, ok && ok1 ? 16u : 0u);
-      }
-    } else {
-      const int64_t c = (w % nct) * 128 + 8 * ch;
-      const bool col_ok = c < cols;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int rr = rsub + 16 * i;
-        const bool ok = rr < it.nrows && col_ok;
-        const uint16_t* gp = ok ? x + (it.row0 + rr) * cols + c : x;
-        cp_async16(sbase + (rr * 16 + ch) * 16, gp, ok ? 16u : 0u);
-      }
+    for (int i = 0; i < 4; ++i) {
+      const int rr = rq + 32 * i;
+      const int64_t src = GATHER ? int64_t(srcs[rr]) : it.row0 + rr;
+      const bool ok = rr < it.nrows && src >= 0;
+      const uint16_t* gp = ok ? x + src * cols + c : x;
+      const uint32_t sa = sbase + rr * 256;
+      cp_async16(sa + cq * 16, ok && ok0 ? gp : x, ok && ok0 ? 16u : 0u);
+      cp_async16(sa + cs1 * 16, ok && ok1 ? gp + 64 : x, ok && ok1 ? 16u : 0u);
     }
     cp_async_commit();
   };
@@ -428,53 +417,32 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_dual_kernel(
     const uint32_t* tile = reinterpret_cast<const uint32_t*>(tile4);
 
     // ---- rowwise
-    if constexpr (GATHER) {
-      const bool col_ok = col0 + 16 * cq < cols;
-      uint8_t* qrow = q + (it.row0 + rq) * cols + col0 + 16 * cq;
+    const bool col_ok = col0 + 16 * cq < cols;
+    uint8_t* qrow = q + (it.row0 + rq) * cols + col0 + 16 * cq;
 #pragma unroll 2
-      for (int i = 0; i < 4; ++i) {
-        const int rr = rq + 32 * i;
-        const uint4 va = tile4[rr * 16 + sl0], vb = tile4[rr * 16 + sl1];
-        uint32_t a = bmax_abs2(bmax_abs2(bmax_abs2(va.x, va.y), bmax_abs2(va.z, va.w)),
-                               bmax_abs2(bmax_abs2(vb.x, vb.y), bmax_abs2(vb.z, vb.w)));
-        a = bmax_abs2(a, __shfl_xor_sync(0xffffffffu, a, 1));
-        a = bmax_abs2(a, __byte_perm(a, 0, 0x1032));
-        const uint32_t sb = scale_byte_bf(a);
-        const uint32_t fm = (254u - sb) * 0x00800080u;   // 2^-s in both bf16 halves
-        uint4 o;
-        o.x = e4m3_pairs(bmul2(va.x, fm), bmul2(va.y, fm));
-        o.y = e4m3_pairs(bmul2(va.z, fm), bmul2(va.w, fm));
-        o.z = e4m3_pairs(bmul2(vb.x, fm), bmul2(vb.y, fm));
-        o.w = e4m3_pairs(bmul2(vb.z, fm), bmul2(vb.w, fm));
-        if (sb == 0xFFu) o = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-        if (rr < it.nrows && col_ok) *reinterpret_cast<uint4*>(qrow + int64_t(32 * i) * cols) = o;
-        if ((cq & 1) == 0) atom_r[(rr & 31) * 16 + (rr >> 5) * 4 + (cq >> 1)] = static_cast<uint8_t>(sb);
-      }
-    } else {
-      const bool col_ok = col0 + 8 * ch < cols;
-#pragma unroll 4
-      for (int i = 0; i < 8; ++i) {
-        const int rr = rsub + 16 * i;
-        const uint4 v = tile4[rr * 16 + ch];
-        uint32_t a = bmax_abs2(bmax_abs2(v.x, v.y), bmax_abs2(v.z, v.w));
-        a = bmax_abs2(a, __shfl_xor_sync(0xffffffffu, a, 1));
-        a = bmax_abs2(a, __shfl_xor_sync(0xffffffffu, a, 2));
-        a = bmax_abs2(a, __byte_perm(a, 0, 0x1032));
-        const uint32_t sb = scale_byte_bf(a);
-        const uint32_t fm = (254u - sb) * 0x00800080u;   // 2^-s in both bf16 halves
-        uint2 o;
-        o.x = e4m3_pairs(bmul2(v.x, fm), bmul2(v.y, fm));
-        o.y = e4m3_pairs(bmul2(v.z, fm), bmul2(v.w, fm));
-        if (sb == 0xFFu) o = make_uint2(0x7F7F7F7Fu, 0x7F7F7F7Fu);
-        if (rr < it.nrows && col_ok) *reinterpret_cast<uint2*>(q + (it.row0 + rr) * cols + col0 + 8 * ch) = o;
-        if ((ch & 3) == 0) atom_r[(rr & 31) * 16 + (rr >> 5) * 4 + (ch >> 2)] = static_cast<uint8_t>(sb);
-      }
+    for (int i = 0; i < 4; ++i) {
+      const int rr = rq + 32 * i;
+      const uint4 va = tile4[rr * 16 + sl0], vb = tile4[rr * 16 + sl1];
+      uint32_t a = bmax_abs2(bmax_abs2(bmax_abs2(va.x, va.y), bmax_abs2(va.z, va.w)),
+                             bmax_abs2(bmax_abs2(vb.x, vb.y), bmax_abs2(vb.z, vb.w)));
+      a = bmax_abs2(a, __shfl_xor_sync(0xffffffffu, a, 1));
+      a = bmax_abs2(a, __byte_perm(a, 0, 0x1032));
+      const uint32_t sb = scale_byte_bf(a);
+      const uint32_t fm = (254u - sb) * 0x00800080u;   // 2^-s in both bf16 halves
+      uint4 o;
+      o.x = e4m3_pairs(bmul2(va.x, fm), bmul2(va.y, fm));
+      o.y = e4m3_pairs(bmul2(va.z, fm), bmul2(va.w, fm));
+      o.z = e4m3_pairs(bmul2(vb.x, fm), bmul2(vb.y, fm));
+      o.w = e4m3_pairs(bmul2(vb.z, fm), bmul2(vb.w, fm));
+      if (sb == 0xFFu) o = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      if (rr < it.nrows && col_ok) *reinterpret_cast<uint4*>(qrow + int64_t(32 * i) * cols) = o;
+      if ((cq & 1) == 0) atom_r[(rr & 31) * 16 + (rr >> 5) * 4 + (cq >> 1)] = static_cast<uint8_t>(sb);
     }
 
     // ---- colwise
     const int blk = t >> 6, p = t & 63;
     uint32_t wv[32];
-    const int pw = GATHER ? (p ^ ((p >> 3) & 4)) : p;   // word of column pair p in a tile row
+    const int pw = p ^ ((p >> 3) & 4);   // word of column pair p in a (swizzled) tile row
 #pragma unroll
     for (int r = 0; r < 32; ++r) wv[r] = tile[(32 * blk + r) * 64 + pw];
     uint32_t mx = wv[0];
