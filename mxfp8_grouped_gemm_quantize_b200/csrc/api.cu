@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "launch.h"
@@ -80,6 +81,10 @@ mxf8_status run_gemm(mxf8::GemmArgs& g, void* work, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   g.status = static_cast<int32_t*>(work);
   g.timeout_ns = kDefaultTimeoutNs;
+  // Test hook for the bounded-wait path: with MXF8_TEST_SKIP_FIRST_STAGE set,
+  // a 1-CTA launch leaves its first pipeline stage unfilled and the device
+  // status becomes MXF8_ERR_TIMEOUT after the wait limit.
+  g.inject_skip_stage = std::getenv("MXF8_TEST_SKIP_FIRST_STAGE") != nullptr ? 1 : 0;
   cudaError_t e = cudaMemsetAsync(work, 0, sizeof(int32_t), st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   const char* detail = nullptr;

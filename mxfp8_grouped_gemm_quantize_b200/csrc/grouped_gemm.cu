@@ -120,6 +120,7 @@ struct Params {
   int64_t out_ld;                      // output row stride (elements)
   int32_t* status;
   uint64_t timeout_ns;
+  int32_t inject_skip_stage;           // test hook: the producer leaves stage 0 unfilled (1-CTA only)
   // Quantising epilogue (fwd/dgrad): MXFP8 copies of the bf16 output, in the
   // quantisers' layouts with the GEMM's groups.  Null pointers skip a layout.
   uint8_t* qr;                         // rowwise codes [M, out_ld]
@@ -369,6 +370,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       uint32_t it = 0, s = 0, ph = 0;
       int32_t eh = 0;
       bool failed = false;
+      // Test hook: stage 0 gets neither its copies nor its arrival, so the MMA
+      // warp's bounded wait on it runs out; the drain below skips it.
+      const bool skip0 = CG == 1 && p.inject_skip_stage != 0;
       for (int32_t t = unit0; t < total && !failed; t += nunits) {
         eh = advance_group(sc, p.E, t, eh);
         const Tile tl = decode_tile<CG, FP4>(p, sc, t, eh, rank);
@@ -377,6 +381,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
             failed = true;
             break;
+          }
+          if (skip0 && it == 0) {
+            ++it;
+            if (++s == STAGES) { s = 0; ph ^= 1; }
+            continue;
           }
           const int32_t nh = min(C::KS, tl.kblocks - kb0);   // K blocks in this stage
           const uint32_t fb = full_bar(s);
@@ -420,11 +429,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           if (++s == STAGES) { s = 0; ph ^= 1; }
         }
       }
-      if (failed) {
-        // Let every copy already issued land before the CTA can exit.
+      if (failed || skip0) {
+        // Let every copy already issued land before the CTA can exit (with the
+        // test hook the MMA warp stops at stage 0 and never waits for the rest).
         if (leader) {
           for (uint32_t j = it > STAGES ? it - STAGES : 0; j < it; ++j)
-            mbar_wait(full_bar(j % STAGES), (j / STAGES) & 1, &never, lim);
+            if (!(skip0 && j == 0)) mbar_wait(full_bar(j % STAGES), (j / STAGES) & 1, &never, lim);
         } else {
           for (int i = 0; i < 100; ++i) __nanosleep(1000);
         }
@@ -879,6 +889,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   p.out_ld = out_cols;
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
+  p.inject_skip_stage = a.inject_skip_stage;
   p.qr = a.qr; p.sr = a.sr; p.qc = a.qc; p.sc = a.sc;
   p.qc_ld = a.qc_ld; p.sc_pitch = a.sc_pitch;
   p.amax_a = a.amax_a; p.amax_b = a.amax_b;

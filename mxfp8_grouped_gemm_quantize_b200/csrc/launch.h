@@ -63,6 +63,9 @@ struct GemmArgs {
   uint16_t* out;                 // bf16 output; may be null when a quantised copy is requested
   int32_t* status;
   uint64_t timeout_ns;
+  // Test hook (1-CTA launches): the producer leaves its first pipeline stage
+  // unfilled, so the MMA warp's bounded wait for it runs out (MXF8_ERR_TIMEOUT).
+  int32_t inject_skip_stage = 0;
   // fwd/dgrad only: MXFP8 copies of the output written by the epilogue, in
   // the quantisers' rowwise (qr, sr) and colwise (qc, sc) layouts over the
   // GEMM's groups; null = not written.

@@ -1,0 +1,61 @@
+"""The GEMM's bounded pipeline waits, exercised on the GPU without faulting it.
+
+With MXF8_TEST_SKIP_FIRST_STAGE set, the producer of every CTA leaves its
+first pipeline stage unfilled (no copies, no arrival): the MMA warp's wait on
+it is a flag that nothing sets.  The wait must give up after its limit, the
+kernel must drain what it had in flight and return, the device status must
+read MXF8_ERR_TIMEOUT, and the context must stay usable: the next launch
+without the hook produces the oracle's result."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mxfp8_grouped_gemm_quantize_b200 import workloads as wl
+from tests.helpers import np_u8
+
+pytestmark = pytest.mark.gpu
+
+TIMEOUT = 6   # MXF8_ERR_TIMEOUT
+
+
+@pytest.fixture(scope="module")
+def mx():
+    import mxfp8_grouped_gemm_quantize_b200 as m
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    assert m.mxfp8_device_supported(), "GPU tests need an sm_100 device"
+    return m
+
+
+def test_unfilled_stage_times_out_and_the_context_stays_usable(mx):
+    counts = [0, 150, 300, 62]
+    E, N, K = len(counts), 256, 512
+    offs = wl.offsets_from_counts(counts)
+    M = int(offs[-1])
+    X = wl.normal_bf16((M, K), 1.0, 71)
+    W = wl.normal_bf16((E * N, K), 0.05, 72)
+    od = torch.from_numpy(offs).cuda()
+    xq, xs = mx.mxfp8_quantize_rowwise(X.cuda(), od)
+    wq, ws = mx.mxfp8_quantize_rowwise(W.cuda())
+    work = mx.new_workspace(E, M, N, K)
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+
+    os.environ["MXF8_TEST_SKIP_FIRST_STAGE"] = "1"
+    try:
+        mx.mxfp8_grouped_gemm_fwd(xq, xs, wq, ws, od, N, out=y, work=work)
+        torch.cuda.synchronize()
+    finally:
+        del os.environ["MXF8_TEST_SKIP_FIRST_STAGE"]
+    assert mx.mxfp8_get_status(work) == TIMEOUT
+
+    mx.mxfp8_grouped_gemm_fwd(xq, xs, wq, ws, od, N, out=y, work=work)
+    torch.cuda.synchronize()
+    assert mx.mxfp8_get_status(work) == 0
+    Xd = oracle.dequantize_rowwise(np_u8(xq), np_u8(xs), offs)
+    Wd = oracle.dequantize_rowwise(np_u8(wq), np_u8(ws)).reshape(E, N, K)
+    ref = oracle.gemm_fwd(Xd, Wd, offs)
+    got = y.double().cpu().numpy()
+    err = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert err <= 5e-3
