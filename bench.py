@@ -56,7 +56,8 @@ def parse():
     # profiling aids (the headline line uses the defaults)
     ap.add_argument("--linears", default="all", help="comma-separated subset of the workload's linears")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the measurements outside the step (e2e, quantising epilogue, MoE dispatch)")
+                    help="skip the measurements outside the step (e2e, quantising epilogue, MoE dispatch, NVFP4, "
+                         "quantiser sweep)")
     return ap.parse_args()
 
 
@@ -343,6 +344,7 @@ def run_ours(args, rank, world, local_rank):
         out["quantising_epilogue"] = quantising_epilogue(mx, layers[0])
         out["moe_dispatch"] = moe_dispatch(mx, args, pk["hbm_gbs"])
         out["nvfp4"] = nvfp4_measure(mx, layers[0], fp8_peak, pk["hbm_gbs"])
+        out["quantiser_sweep"] = quantiser_sweep(mx, pk["hbm_gbs"])
     return out
 
 
@@ -601,11 +603,69 @@ def _cpu_sample(w: wl.Workload, budget_s: float):
     return flops, secs, desc
 
 
+def quantiser_sweep(mx, hbm_gbs, iters=10):
+    """The quantiser sweep: M in {4096, 16384, 65536} x K in {2048, 5120, 7168},
+    one group, N(0,1) with 0.1 % outliers x1000 and 1 % of aligned 32x32 tiles
+    zeroed.  Rowwise, colwise and dual kernels, each launch timed alone with L2
+    flushed before it; GB/s of algorithmic bytes (rowwise / colwise:
+    2 + 1 + 1/32 B per element, dual: 2 + 2 (1 + 1/32))."""
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
+
+    def t(fn):
+        for _ in range(3):
+            fn()
+        tot = 0.0
+        for _ in range(iters):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            tot += a.elapsed_time(b)
+        return tot / iters
+
+    rows = []
+    for M, K in wl.quantiser_sweep():
+        x = wl.sweep_tensor(M, K, device="cuda")
+        q, sf = mx.mxfp8_quantize_rowwise(x)
+        qT, sfT = mx.mxfp8_quantize_colwise(x)
+        r = {"M": M, "K": K}
+        for name, fn, bpe in (("rowwise", lambda: mx.mxfp8_quantize_rowwise(x, None, q=q, scales=sf), 3.03125),
+                              ("colwise", lambda: mx.mxfp8_quantize_colwise(x, None, qT=qT, scales=sfT), 3.03125),
+                              ("dual", lambda: mx.mxfp8_quantize_dual(x, None, q=q, scales=sf, qT=qT, scalesT=sfT),
+                               4.0625)):
+            ms = t(fn)
+            gbs = M * K * bpe / (ms * 1e-3) / 1e9
+            r[name] = {"us": round(ms * 1e3, 1), "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4)}
+        rows.append(r)
+        del x, q, sf, qT, sfT
+    torch.cuda.empty_cache()
+    return {"input": "N(0,1), 0.1 % outliers x1000, 1 % of aligned 32x32 tiles zeroed; one group",
+            "peak_gbs": hbm_gbs, "sizes": rows}
+
+
+def _cpu_quantiser(budget_s=2.0):
+    """The oracle's rowwise quantiser on the smallest sweep size (4096 x 2048):
+    GB/s of the same algorithmic bytes as the GPU sweep."""
+    import oracle
+    x = wl.sweep_tensor(4096, 2048)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.quantize_rowwise(x)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    secs = (time.perf_counter() - t0) / n
+    return {"gbs": round(4096 * 2048 * 3.03125 / secs / 1e9, 3), "kernel": "rowwise", "M": 4096, "K": 2048,
+            "seconds_per_call": round(secs, 4)}
+
+
 def cpu_baseline(w, budget_s=12.0):
     import oracle
     flops, secs, desc = _cpu_sample(w, budget_s)
     return {"value": round(flops / secs / 1e12, 5), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-            "sample": desc, "seconds": round(secs, 2)}
+            "sample": desc, "seconds": round(secs, 2), "quantiser": _cpu_quantiser()}
 
 
 def run_reference(args):

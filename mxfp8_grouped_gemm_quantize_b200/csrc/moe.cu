@@ -143,9 +143,11 @@ __device__ __forceinline__ void combine_add(double (&acc)[8], double wj, const u
 }
 
 // Slots are summed in order 0..k-1; an unrouted slot is skipped (not added
-// as zero, which would turn -0 into +0).  The sum is bound by fp64
-// arithmetic, not by memory, so each thread keeps one slot's row in flight
-// and the SM keeps many threads resident.
+// as zero, which would turn -0 into +0).  For top-k with k <= 8 a thread
+// issues all k row loads before the sums, so k independent 16-byte loads
+// are in flight instead of one dependent index -> row chain per slot.
+constexpr int kCombineSlots = 8;
+
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const uint16_t* __restrict__ yp, int64_t rows, int64_t cols, const int32_t* __restrict__ inv,
     const float* __restrict__ w, int64_t T, int32_t k, uint16_t* __restrict__ y) {
@@ -155,11 +157,28 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
        u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t t = u / per_row, c = (u - t * per_row) * 8;
     double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-    for (int32_t j = 0; j < k; ++j) {
-      const int32_t r = __ldg(inv + t * k + j);
-      if (r < 0 || r >= rows) continue;            // an unrouted slot contributes nothing
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(yp + static_cast<int64_t>(r) * cols + c));
-      combine_add(acc, static_cast<double>(__ldg(w + t * k + j)), v);
+    if (k <= kCombineSlots) {
+      int32_t r[kCombineSlots];
+      uint4 v[kCombineSlots];
+#pragma unroll
+      for (int j = 0; j < kCombineSlots; ++j) {
+        r[j] = j < k ? __ldg(inv + t * k + j) : -1;
+        if (r[j] >= rows) r[j] = -1;                // an unrouted slot contributes nothing
+      }
+#pragma unroll
+      for (int j = 0; j < kCombineSlots; ++j)
+        v[j] = r[j] >= 0 ? __ldg(reinterpret_cast<const uint4*>(yp + static_cast<int64_t>(r[j]) * cols + c))
+                         : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < kCombineSlots; ++j)
+        if (r[j] >= 0) combine_add(acc, static_cast<double>(__ldg(w + t * k + j)), v[j]);
+    } else {
+      for (int32_t j = 0; j < k; ++j) {
+        const int32_t r = __ldg(inv + t * k + j);
+        if (r < 0 || r >= rows) continue;
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(yp + static_cast<int64_t>(r) * cols + c));
+        combine_add(acc, static_cast<double>(__ldg(w + t * k + j)), v);
+      }
     }
     auto pack = [](double lo, double hi) {
       return static_cast<uint32_t>(bf16_bits_rne(lo)) | (static_cast<uint32_t>(bf16_bits_rne(hi)) << 16);
