@@ -1,0 +1,65 @@
+"""bench.py host logic that needs no GPU: the roofline's traffic figure is
+read from the committed ncu summary only while the kernel sources are the
+ones it was taken on, the peaks come from the measured file, and the clock
+sampler decodes throttle reasons from a fake NVML (it only reads)."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_traffic_is_read_while_the_sources_match():
+    t = bench.gemm_traffic()
+    assert isinstance(t, int) and 5e8 < t < 1.5e9       # DRAM bytes per GEMM launch, DS-16B gate/up
+
+
+def test_traffic_is_null_once_the_sources_change(tmp_path, monkeypatch):
+    prof = tmp_path / "profile.md"
+    text = open(bench.GEMM_PROFILE, encoding="utf-8").read()
+    prof.write_text(text)
+    monkeypatch.setattr(bench, "GEMM_PROFILE", str(prof))
+    assert bench.gemm_traffic() is not None
+    monkeypatch.setattr(bench, "gemm_sources_sha256", lambda: "0" * 64)
+    assert bench.gemm_traffic() is None
+    monkeypatch.setattr(bench, "GEMM_PROFILE", str(tmp_path / "missing.md"))
+    assert bench.gemm_traffic() is None
+
+
+def test_the_source_hash_covers_the_gemm_sources():
+    h1 = bench.gemm_sources_sha256()
+    assert len(h1) == 64 and h1 == bench.gemm_sources_sha256()
+    assert "grouped_gemm.cu" in bench.GEMM_SOURCES and "ptx.cuh" in bench.GEMM_SOURCES
+
+
+def test_peaks_come_from_the_measured_file():
+    pk = bench.peaks()
+    if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")):
+        assert pk["src"] == "measured" and pk["hbm_gbs"] > 1000 and pk["bf16"] > 100
+    else:
+        assert pk["src"] == "fallback"
+
+
+class _FakeNVML:
+    nvmlClocksThrottleReasonSwPowerCap = 0x4
+    nvmlClocksThrottleReasonHwSlowdown = 0x8
+    nvmlClocksThrottleReasonSwThermalSlowdown = 0x20
+    nvmlClocksThrottleReasonHwThermalSlowdown = 0x40
+
+
+def test_clock_reasons_are_decoded_from_the_mask():
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.nv = _FakeNVML()
+    assert s._reason_names(0x4) == {"sw_power_cap"}
+    assert s._reason_names(0x4 | 0x40) == {"sw_power_cap", "hw_thermal_slowdown"}
+    assert s._reason_names(0x0) == set()
+    assert bench.ClockSampler.BAD == {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+def test_summary_reports_the_median_clock():
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.samples, s.reasons, s.max_mhz = [1500, 1700, 1650], {"sw_power_cap"}, 1965
+    out = s.summary()
+    assert out == {"sm_mhz": 1650, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"], "samples": 3}
