@@ -84,7 +84,8 @@ typedef enum {
     MXF8_ERR_UNSUPPORTED = 3,  /* the current device is not sm_100 */
     MXF8_ERR_CUDA = 4,         /* a CUDA call failed; see mxfp8_last_cuda_error() */
     MXF8_ERR_BAD_OFFSETS = 5,  /* device side: d_offs is not a valid prefix of `rows` */
-    MXF8_ERR_TIMEOUT = 6,      /* device side: a pipeline wait ran past its limit */
+    MXF8_ERR_TIMEOUT = 6,      /* device side: a pipeline wait ran past its limit (2 s); tests provoke it
+                                  by setting MXF8_TEST_SKIP_FIRST_STAGE in the environment */
     MXF8_ERR_BAD_ROUTING = 7   /* device side: an expert id outside [0, num_experts) */
 } mxf8_status;
 
