@@ -227,6 +227,25 @@ class Linear:
         ]
 
 
+def system_info(device_index: int = 0) -> dict:
+    """GPU name, driver, CUDA and torch versions and host cores, for the JSON
+    line (reads only; every field is None when it cannot be read)."""
+    info = {"gpu": None, "driver": None, "cuda": torch.version.cuda, "torch": torch.__version__,
+            "host_cores": os.cpu_count()}
+    try:
+        info["gpu"] = torch.cuda.get_device_name(device_index)
+    except Exception:
+        pass
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        v = pynvml.nvmlSystemGetDriverVersion()
+        info["driver"] = v.decode() if isinstance(v, bytes) else v
+    except Exception:
+        pass
+    return info
+
+
 def max_over_ranks(x: float, world: int, device) -> float:
     """The largest x over all ranks: a job's time is its slowest rank's."""
     if world <= 1:
@@ -334,6 +353,7 @@ def run_ours(args, rank, world, local_rank):
         "breakdown": breakdown,
         "gpu_launches": K * n_calls,
         "clocks": clk.summary(),
+        "system": system_info(local_rank),
     }
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(w, budget_s=12.0)

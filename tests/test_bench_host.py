@@ -63,3 +63,9 @@ def test_summary_reports_the_median_clock():
     s.samples, s.reasons, s.max_mhz = [1500, 1700, 1650], {"sw_power_cap"}, 1965
     out = s.summary()
     assert out == {"sm_mhz": 1650, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"], "samples": 3}
+
+
+def test_system_info_reads_what_it_can():
+    info = bench.system_info(0)
+    assert set(info) == {"gpu", "driver", "cuda", "torch", "host_cores"}
+    assert info["torch"] and info["host_cores"] >= 1
