@@ -20,7 +20,7 @@
  *     Transformer Engine grouped GEMM): Y_e = X_e W_e^T, dX_e = dY_e W_e,
  *     dW_e = dY_e^T X_e, each per expert e over rows offs[e]..offs[e+1]-1.
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *   - an all-zero block has scale exponent -127 (byte 0x00) and zero codes;
  *   - the sign of zero survives quantisation (-0 and negative underflow
  *     encode as 0x80), as IEEE round-to-nearest-even gives;
