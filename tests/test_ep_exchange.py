@@ -111,3 +111,42 @@ def test_invalid_splits_and_ids_are_rejected_before_any_exchange():
         p.join(timeout=60)
         assert p.exitcode == 0
     assert all(e == [True, True] for _, e in got)
+
+
+def _edge(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world,
+                                         timeout=datetime.timedelta(seconds=60))
+    try:
+        from mxfp8_grouped_gemm_quantize_b200 import ep
+        E, C = 4, 8
+        if rank == 0:   # no tokens at all
+            x, idx = torch.zeros((0, C)), torch.zeros((0, 2), dtype=torch.int32)
+        else:           # every pair goes to rank 1's own experts (2 and 3)
+            x = torch.arange(5 * C, dtype=torch.float32).view(5, C)
+            idx = torch.tensor([[2, 3]] * 5, dtype=torch.int32)
+        rows, le, ex = ep.dispatch(x, idx, E)
+        back = ep.give_back(rows * 2, ex)
+        if rank == 0:
+            ok = rows.shape == (0, C) and le.numel() == 0 and back.shape == (0, C)
+        else:
+            exp = x.repeat_interleave(2, dim=0)
+            ok = torch.equal(rows, exp) and le.tolist() == [0, 1] * 5 and torch.equal(back, exp * 2)
+        q.put((rank, ok))
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+def test_a_rank_without_tokens_and_a_rank_receiving_nothing():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_edge, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(ok for _, ok in got), got
