@@ -246,6 +246,16 @@ def system_info(device_index: int = 0) -> dict:
     return info
 
 
+def workload_config(w, quantiser: str, world: int) -> dict:
+    """The `config` object of the JSON line, identical for both arms."""
+    return {"workload": f"{w.name}-like MoE layer", "experts": w.E, "routed_rows": w.M,
+            "layers": [{"name": L.name, "N": L.N, "K": L.K} for L in w.layers],
+            "routing": ("top-6 of 8192 tokens, N(0,1) logits + N(0,0.5) expert bias" if w.name == "ds-v3-16b"
+                        else w.name),
+            "l2": "inputs larger than L2 (step touches > 2 GB)", "parallelism": f"replica x{world}",
+            "quantiser": quantiser}
+
+
 def max_over_ranks(x: float, world: int, device) -> float:
     """The largest x over all ranks: a job's time is its slowest rank's."""
     if world <= 1:
@@ -334,11 +344,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)", "data": "synthetic",
-        "config": {"workload": f"{w.name}-like MoE layer", "experts": w.E, "routed_rows": w.M,
-                   "layers": [{"name": L.name, "N": L.N, "K": L.K} for L in w.layers],
-                   "routing": "top-6 of 8192 tokens, N(0,1) logits + N(0,0.5) expert bias" if w.name == "ds-v3-16b" else w.name,
-                   "l2": "inputs larger than L2 (step touches > 2 GB)", "parallelism": f"replica x{world}",
-                   "quantiser": args.quantiser},
+        "config": workload_config(w, args.quantiser, world),
         "fraction_of_fp8_peak": round(value / world / fp8_peak, 4),
         "roofline": {"kernel": "grouped_gemm_kernel (fwd+dgrad+wgrad launches)", "bound": "tensor",
                      "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
@@ -705,8 +711,7 @@ def run_reference(args):
             "warmup": warm, "ms_per_step": round(1e3 * tot_s / steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 inputs)", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": f"{w.name}-like MoE layer", "experts": w.E, "routed_rows": w.M,
-                       "layers": [{"name": L.name, "N": L.N, "K": L.K} for L in w.layers]},
+            "config": workload_config(w, args.quantiser, args.gpus),
             "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
                              "sample": desc + f"; {per_step:.2f} s per step"},
             "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

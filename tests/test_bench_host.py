@@ -69,3 +69,12 @@ def test_system_info_reads_what_it_can():
     info = bench.system_info(0)
     assert set(info) == {"gpu", "driver", "cuda", "torch", "host_cores"}
     assert info["torch"] and info["host_cores"] >= 1
+
+
+def test_both_arms_share_one_config():
+    from mxfp8_grouped_gemm_quantize_b200 import workloads as wl
+    w = wl.ds_v3_16b()
+    c = bench.workload_config(w, "dual", 1)
+    assert c["workload"] == "ds-v3-16b-like MoE layer" and c["routed_rows"] == 49152 and c["experts"] == 64
+    assert c["layers"] == [{"name": "gate_up", "N": 2816, "K": 2048}, {"name": "down", "N": 2048, "K": 1408}]
+    assert c["parallelism"] == "replica x1"
