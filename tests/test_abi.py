@@ -60,3 +60,23 @@ def test_status_strings(lib):
     import mxfp8_grouped_gemm_quantize_b200 as m
     for code in range(7):
         assert m.lib().mxfp8_status_string(code)
+
+
+def test_no_cpu_fallback_without_a_gpu_tensor():
+    """The binding only marshals device pointers: host tensors are refused
+    loudly, and nothing falls back to a CPU computation."""
+    import torch
+    import mxfp8_grouped_gemm_quantize_b200 as mx
+    x = torch.zeros((64, 64), dtype=torch.bfloat16)
+    with pytest.raises(AssertionError, match="CUDA"):
+        mx.mxfp8_quantize_rowwise(x)
+    with pytest.raises(AssertionError, match="CUDA"):
+        mx.mxfp8_quantize_dual(x)
+
+
+def test_missing_library_is_an_error(monkeypatch, tmp_path):
+    import mxfp8_grouped_gemm_quantize_b200 as mx
+    monkeypatch.setattr(mx, "_LIB", None)
+    monkeypatch.setattr(mx, "LIB_PATH", str(tmp_path / "libmxfp8.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        mx.lib()
