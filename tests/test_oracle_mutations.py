@@ -1,0 +1,113 @@
+"""The pins catch plausible mistakes.
+
+Each mutant below is the MXFP8 block rule or a grouped GEMM with one
+plausible mistake planted (an off-by-one exponent, ties rounded away from
+zero, no saturation, a lost sign of zero, a wrong clamp, a dropped term, a
+shifted group boundary, a transposed operand).  They are small CPU
+restatements, not the oracle; the test checks that the oracle passes the pins
+and that every mutant fails at least one of them, i.e. the pins would have
+caught that mistake in the oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from mxfp8_grouped_gemm_quantize_b200 import workloads as wl
+from tests.test_oracle_scalars import _bf16_bits, _golden_blocks
+
+
+def _e4m3(v, tie_even=True, saturate=True, keep_sign=True):
+    """E4M3 code of a real value (1 sign, 4 exponent bits, bias 7, 3 mantissa bits)."""
+    sign = 0x80 if (math.copysign(1.0, v) < 0 and (keep_sign or v != 0.0)) else 0x00
+    a = abs(v)
+    if a == 0.0:
+        return sign
+    e = max(math.floor(math.log2(a)), -6)                  # subnormals share the 2^-6 binade
+    q = a / 2.0 ** (e - 3)                                 # units of the last mantissa bit
+    lo = math.floor(q)
+    frac = q - lo
+    if frac > 0.5 or (frac == 0.5 and (lo % 2 == 1 if tie_even else True)):
+        lo += 1
+    mag = lo * 2.0 ** (e - 3)
+    if mag > 448.0:
+        if not saturate:
+            return sign | 0x7F                             # NaN
+        mag = 448.0
+    if mag == 0.0:
+        return sign if keep_sign else 0x00
+    e2 = max(math.floor(math.log2(mag)), -6)
+    m = int(round(mag / 2.0 ** (e2 - 3)))
+    if e2 == -6 and m < 8:
+        return sign | m                                    # subnormal
+    return sign | ((e2 + 7) << 3) | (m - 8)
+
+
+def _block(vals, emax=8, clamp_lo=-127, **enc):
+    amax = max(abs(v) for v in vals)
+    s = clamp_lo if amax == 0.0 else max(math.floor(math.log2(amax)) - emax, clamp_lo)
+    s = min(s, 127)
+    return [_e4m3(v * 2.0 ** -s, **enc) for v in vals], s + 127
+
+
+def _golden_ok(fn):
+    for name, sb, pairs in _golden_blocks():
+        vals = [v for v, _ in pairs] + [0.0] * (32 - len(pairs))
+        codes, byte = fn(vals)
+        if byte != sb or any(codes[i] != c for i, (_, c) in enumerate(pairs)):
+            return False
+    return True
+
+
+def _oracle_block(vals):
+    codes, sb = oracle.quantize_block(_bf16_bits(vals))
+    return list(codes), sb
+
+
+def test_the_oracle_and_the_restatement_pass_the_golden_blocks():
+    assert _golden_ok(_oracle_block)
+    assert _golden_ok(_block)
+
+
+@pytest.mark.parametrize("mutant", [
+    dict(emax=7),                  # scale exponent off by one
+    dict(emax=9),
+    dict(tie_even=False),          # ties rounded away from zero
+    dict(saturate=False),          # overflow to NaN instead of 448
+    dict(keep_sign=False),         # -0 and negative underflow lose the sign
+    dict(clamp_lo=-126),           # wrong lower clamp of the scale exponent
+], ids=lambda d: ",".join(f"{k}={v}" for k, v in d.items()))
+def test_block_rule_mutants_fail_a_golden_block(mutant):
+    assert not _golden_ok(lambda vals: _block(vals, **mutant))
+
+
+def _fwd_ok(fwd):
+    counts = [3, 0, 5, 4]
+    offs = wl.offsets_from_counts(counts)
+    rng = np.random.default_rng(9)
+    M, E, N, K = int(offs[-1]), len(counts), 6, 10
+    X, W = rng.standard_normal((M, K)), rng.standard_normal((E, N, K))
+    try:
+        Y = fwd(X, W, offs)
+    except Exception:
+        return False
+    ref = np.concatenate([X[offs[e]:offs[e + 1]] @ W[e].T for e in range(E)])
+    return Y.shape == ref.shape and np.allclose(Y, ref, rtol=1e-12, atol=1e-12)
+
+
+def _per_expert(op):
+    def fwd(X, W, offs):
+        return np.concatenate([op(X, W, offs, e) for e in range(W.shape[0])])
+    return fwd
+
+
+@pytest.mark.parametrize("name,mutant", [
+    ("dropped_last_k", _per_expert(lambda X, W, o, e: X[o[e]:o[e + 1], :-1] @ W[e][:, :-1].T)),
+    ("shifted_boundary", _per_expert(lambda X, W, o, e: X[max(o[e] - 1, 0):max(o[e + 1] - 1, 0)] @ W[e].T)),
+    ("wrong_expert", _per_expert(lambda X, W, o, e: X[o[e]:o[e + 1]] @ W[(e + 1) % W.shape[0]].T)),
+    ("transposed_weight", _per_expert(lambda X, W, o, e: X[o[e]:o[e + 1]] @ W[e])),
+])
+def test_gemm_mutants_fail_the_matmul_pin(name, mutant):
+    assert _fwd_ok(oracle.gemm_fwd)
+    assert not _fwd_ok(mutant), name
