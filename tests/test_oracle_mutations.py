@@ -111,3 +111,37 @@ def _per_expert(op):
 def test_gemm_mutants_fail_the_matmul_pin(name, mutant):
     assert _fwd_ok(oracle.gemm_fwd)
     assert not _fwd_ok(mutant), name
+
+
+def _swizzle(S, offset):
+    """Bytes of the logical scale matrix S [R, C] placed by an atom formula
+    offset(r, c, pitch) (R a multiple of 128, C a multiple of 4)."""
+    R, C = S.shape
+    pitch = C // 4
+    out = np.zeros(R * C, dtype=np.uint8)
+    for r in range(R):
+        for c in range(C):
+            out[offset(r, c, pitch)] = S[r, c]
+    return out
+
+
+def _atom(inner):
+    return lambda r, c, pitch: 512 * ((r // 128) * pitch + c // 4) + inner(r, c)
+
+
+@pytest.mark.parametrize("name,inner", [
+    ("quarter_and_block_swapped", lambda r, c: (r % 32) * 16 + (c % 4) * 4 + (r % 128) // 32),
+    ("rows_not_interleaved", lambda r, c: (r % 128) * 4 + c % 4),
+    ("quarter_stride_8", lambda r, c: (r % 32) * 16 + ((r % 128) // 32) * 8 % 16 + c % 4),
+])
+def test_scale_layout_mutants_fail_the_independent_layout(name, inner):
+    from tests.test_oracle_layout import _to_blocked
+    S = np.random.default_rng(3).integers(0, 255, size=(256, 8)).astype(np.uint8)
+    ref = _to_blocked(S)
+    assert np.array_equal(_swizzle(S, oracle.sf_offset), ref)         # the oracle's own formula
+    bad = _atom(inner)
+    try:
+        got = _swizzle(S, bad)
+    except IndexError:
+        return                                                       # not even a layout of the atoms
+    assert not np.array_equal(got, ref), name
