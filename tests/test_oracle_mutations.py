@@ -145,3 +145,29 @@ def test_scale_layout_mutants_fail_the_independent_layout(name, inner):
     except IndexError:
         return                                                       # not even a layout of the atoms
     assert not np.array_equal(got, ref), name
+
+
+def _double_rounded_bf16(v):
+    """Mutant: round to fp32 first, then to bf16 (two roundings)."""
+    import torch
+    return torch.tensor(v, dtype=torch.float64).to(torch.float32).to(torch.bfloat16) \
+        .view(torch.int16).numpy().view(np.uint16)
+
+
+def test_combine_rounding_mutant_rounds_twice():
+    """Just above a bf16 tie by less than fp32 can hold: one rounding goes up,
+    rounding through fp32 first lands on the tie and goes to even."""
+    v = np.array([1.0 + 2.0 ** -8 + 2.0 ** -30, -(1.0 + 2.0 ** -8 + 2.0 ** -30), 3.0 + 2.0 ** -7 + 2.0 ** -29])
+    got = oracle.bf16_from_double(v)
+    assert got.tolist() == [0x3F81, 0xBF81, 0x4041]
+    assert _double_rounded_bf16(v).tolist() != got.tolist()
+
+
+def test_unstable_dispatch_order_mutant_fails_the_stable_order():
+    rng = np.random.default_rng(4)
+    idx = np.stack([rng.permutation(6)[:2] for _ in range(50)]).astype(np.int32)
+    _, perm, _ = oracle.moe_plan(idx, 6)                          # perm: source token of each grouped row
+    flat = idx.reshape(-1)
+    assert perm.tolist() == (np.argsort(flat, kind="stable") // 2).tolist()
+    unstable = np.lexsort((-np.arange(flat.size), flat)) // 2     # equal experts: later pairs first
+    assert unstable.tolist() != perm.tolist()
