@@ -171,3 +171,52 @@ def test_unstable_dispatch_order_mutant_fails_the_stable_order():
     assert perm.tolist() == (np.argsort(flat, kind="stable") // 2).tolist()
     unstable = np.lexsort((-np.arange(flat.size), flat)) // 2     # equal experts: later pairs first
     assert unstable.tolist() != perm.tolist()
+
+
+# ---------------------------------------------------------------- NVFP4
+_E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def _e2m1(v, tie_even=True):
+    """E2M1 nibble (sign << 3 | magnitude index), nearest with the given tie rule, saturating at 6."""
+    sign = 0x8 if math.copysign(1.0, v) < 0 else 0x0
+    a = min(abs(v), 6.0)
+    best = min(range(8), key=lambda i: abs(_E2M1[i] - a))
+    lo = max(i for i in range(8) if _E2M1[i] <= a)
+    if lo < 7 and abs(a - _E2M1[lo]) == abs(_E2M1[lo + 1] - a):                # a tie
+        best = (lo if lo % 2 == 0 else lo + 1) if tie_even else lo + 1
+    return sign | best
+
+
+def _nvfp4_block(vals, S, div=6.0, tie_even=True):
+    f32 = np.float32
+    amax = max(abs(v) for v in vals)
+    sb = _e4m3(float(f32(f32(amax) * f32(S)) / f32(div)))
+    e = (sb >> 3) & 0xF
+    sf = (sb & 7) * 2.0 ** -9 if e == 0 else (1 + (sb & 7) / 8) * 2.0 ** (e - 7)
+    if sf == 0.0:
+        return [0] * len(vals), sb
+    return [_e2m1(float(f32(f32(f32(v) * f32(S)) / f32(sf))), tie_even) for v in vals], sb
+
+
+def _nvfp4_golden_ok(fn):
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "nvfp4_blocks.txt")
+    for line in open(path, encoding="utf-8"):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        name, S, sb, pairs = [s.strip() for s in line.split("|")]
+        vals = [float(p.split(":")[0]) for p in pairs.split()]
+        nibs = [int(p.split(":")[1], 16) for p in pairs.split()]
+        codes, got = fn(vals + [0.0] * (16 - len(vals)), float(S))
+        if got != int(sb, 16) or codes[:len(nibs)] != nibs:
+            return False
+    return True
+
+
+def test_nvfp4_restatement_passes_and_mutants_fail_the_golden_blocks():
+    assert _nvfp4_golden_ok(_nvfp4_block)
+    assert not _nvfp4_golden_ok(lambda v, S: _nvfp4_block(v, S, div=4.0))           # wrong E2M1 max in sf
+    assert not _nvfp4_golden_ok(lambda v, S: _nvfp4_block(v, S, tie_even=False))    # ties away from zero
+    assert not _nvfp4_golden_ok(lambda v, S: _nvfp4_block(v, 1.0))                  # tensor scale ignored
