@@ -78,3 +78,25 @@ def test_both_arms_share_one_config():
     assert c["workload"] == "ds-v3-16b-like MoE layer" and c["routed_rows"] == 49152 and c["experts"] == 64
     assert c["layers"] == [{"name": "gate_up", "N": 2816, "K": 2048}, {"name": "down", "N": 2048, "K": 1408}]
     assert c["parallelism"] == "replica x1"
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` (the oracle on the host cores) prints one
+    JSON line with the contract's keys and the same config as our arm."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    from mxfp8_grouped_gemm_quantize_b200 import workloads as wl
+    assert d["config"] == bench.workload_config(wl.ds_v3_16b(), "dual", 1)
+    assert d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
