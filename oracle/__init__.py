@@ -281,6 +281,100 @@ def gemm_wgrad(dY, X, offs) -> np.ndarray:
     return dW
 
 
+# ---------------------------------------------------------------- full-size GEMMs, one expert at a time
+# The grouped GEMM's definition (iitak.ru, "NVIDIA ... JAX", Transformer
+# Engine paragraph: every expert on its own token rows) applied per expert to
+# operands the C dequantisers above decode from the library layout; the
+# per-expert product is a library matmul in fp64 (numpy), so full workload
+# sizes finish in seconds.  Pinned against the triple-loop orc_gemm_* on
+# small inputs in the CPU tests.
+
+def _rows_prefix(counts, unit):
+    return np.concatenate([[0], np.cumsum((np.asarray(counts, np.int64) + unit - 1) // unit)]).astype(np.int64)
+
+
+def rowwise_rows(q, sf, C: int, row0: int, atom_row0: int, n: int) -> np.ndarray:
+    """fp64 [n, C]: rows row0 .. row0+n-1 of a rowwise operand whose scale
+    rows for them start at atom row atom_row0 (a group's first row, or any
+    multiple of 128 inside a one-group operand)."""
+    if n == 0:
+        return np.zeros((0, C))
+    pitch = rowwise_pitch(C)
+    a0 = atom_row0 * pitch * 512
+    a1 = (atom_row0 + (n + 127) // 128) * pitch * 512
+    return dequantize_rowwise(np.ascontiguousarray(q[row0:row0 + n]), np.ascontiguousarray(sf[a0:a1]))
+
+
+def colwise_rows(qT, sfT, pitch: int, col0: int, atom_col0: int, n: int) -> np.ndarray:
+    """fp64 [n, C] (C = qT rows): logical rows stored from code column col0
+    and scale-atom column atom_col0 of a colwise operand whose atom pitch is
+    `pitch` (a group's rows, or a 128-aligned run inside a one-group
+    operand)."""
+    C = qT.shape[0]
+    if n == 0:
+        return np.zeros((0, C))
+    sub = np.zeros((C, colwise_ld(n, 1)), dtype=np.uint8)
+    sub[:, :n] = qT[:, col0:col0 + n]
+    rb = (C + 127) // 128
+    atoms = np.asarray(sfT[:rb * pitch * 512]).reshape(rb, pitch, 512)[:, atom_col0:atom_col0 + (n + 127) // 128]
+    return dequantize_colwise(sub, np.ascontiguousarray(atoms).reshape(-1), n)
+
+
+def fwd_by_expert(xq, xs, wq, ws, offs, N: int):
+    """Yields (e, lo, hi, Y_e) with Y_e = deq(X_e) deq(W_e)^T in fp64; X
+    rowwise grouped by offs, W rowwise [E*N, K] quantised as one group."""
+    o = np.asarray(offs, np.int64)
+    cnt = np.diff(o)
+    RB = _rows_prefix(cnt, 128)
+    K = xq.shape[1]
+    for e in range(len(cnt)):
+        lo, hi = int(o[e]), int(o[e + 1])
+        if hi == lo:
+            continue
+        Xe = rowwise_rows(xq, xs, K, lo, int(RB[e]), hi - lo)
+        We = rowwise_rows(wq, ws, K, e * N, e * N // 128, N)
+        yield e, lo, hi, Xe @ We.T
+
+
+def dgrad_by_expert(dyq, dys, wqT, wsT, offs, K: int):
+    """Yields (e, lo, hi, dX_e) with dX_e = deq(dY_e) deq(W_e) in fp64; dY
+    rowwise grouped by offs, W colwise (logical [E*N, K], one group)."""
+    o = np.asarray(offs, np.int64)
+    cnt = np.diff(o)
+    RB = _rows_prefix(cnt, 128)
+    N = dyq.shape[1]
+    E = len(cnt)
+    pitch_w = colwise_pitch(E * N, 1)
+    for e in range(E):
+        lo, hi = int(o[e]), int(o[e + 1])
+        if hi == lo:
+            continue
+        dYe = rowwise_rows(dyq, dys, N, lo, int(RB[e]), hi - lo)
+        We = colwise_rows(wqT[:K], wsT, pitch_w, e * N, e * N // 128, N)
+        yield e, lo, hi, dYe @ We
+
+
+def wgrad_by_expert(dyqT, dysT, xqT, xsT, offs, M: int):
+    """Yields (e, dW_e) with dW_e = deq(dY_e)^T deq(X_e) in fp64 for every
+    expert (zero for an expert without rows); dY and X colwise grouped by
+    offs."""
+    o = np.asarray(offs, np.int64)
+    cnt = np.diff(o)
+    E = len(cnt)
+    RB = _rows_prefix(cnt, 128)
+    P = np.concatenate([[0], np.cumsum((cnt + 31) // 32 * 32)])
+    pitch = colwise_pitch(M, E)
+    N, K = dyqT.shape[0], xqT.shape[0]
+    for e in range(E):
+        m = int(cnt[e])
+        if m == 0:
+            yield e, np.zeros((N, K))
+            continue
+        dYe = colwise_rows(dyqT, dysT, pitch, int(P[e]), int(RB[e]), m)
+        Xe = colwise_rows(xqT, xsT, pitch, int(P[e]), int(RB[e]), m)
+        yield e, dYe.T @ Xe
+
+
 # ---------------------------------------------------------------- sampled outputs
 def sample_fwd(xq, xs, wq, ws, offs, N, rows, cols) -> np.ndarray:
     xq = np.ascontiguousarray(xq, np.uint8); xs = np.ascontiguousarray(xs, np.uint8)

@@ -254,10 +254,12 @@ int orc_quantize_rowwise(const uint16_t* x, int64_t R, int64_t C, const int32_t*
     group_prefixes(offs, G, R, RB, P);
     memset(sf, 0, (size_t)(RB[G] * pitch * 512));
     for (g = 0; g < G; ++g) {
-        int64_t lo, hi, r, j;
+        int64_t lo, hi, r;
         group_bounds(offs, G, R, g, &lo, &hi);
+        /* rows are independent: threads only split the loop */
+#pragma omp parallel for schedule(static)
         for (r = lo; r < hi; ++r) {
-            int64_t pr = 128 * RB[g] + (r - lo);
+            int64_t pr = 128 * RB[g] + (r - lo), j;
             for (j = 0; j < nb; ++j) {
                 uint8_t sb;
                 orc_quantize_block(x + r * C + 32 * j, 32, 1, q + r * C + 32 * j, 1, &sb);
@@ -286,10 +288,13 @@ int orc_quantize_colwise(const uint16_t* x, int64_t R, int64_t C, const int32_t*
         for (cb = 0; cb < RB[G]; ++cb)
             memset(sfT + (rb * pitch + cb) * 512, 0, 512);
     for (g = 0; g < G; ++g) {
-        int64_t lo, hi, m, t0;
+        int64_t lo, hi, m;
         group_bounds(offs, G, R, g, &lo, &hi);
         m = hi - lo;
+        /* columns are independent: threads only split the loop */
+#pragma omp parallel for schedule(static)
         for (c = 0; c < C; ++c) {
+            int64_t t0;
             for (t0 = 0; t0 < m; t0 += 32) {
                 int n = (int)(m - t0 < 32 ? m - t0 : 32);
                 uint8_t sb;
@@ -319,10 +324,11 @@ int orc_dequantize_rowwise(const uint8_t* q, const uint8_t* sf, int64_t R, int64
     P = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
     group_prefixes(offs, G, R, RB, P);
     for (g = 0; g < G; ++g) {
-        int64_t lo, hi, r, c;
+        int64_t lo, hi, r;
         group_bounds(offs, G, R, g, &lo, &hi);
+#pragma omp parallel for schedule(static)
         for (r = lo; r < hi; ++r) {
-            int64_t pr = 128 * RB[g] + (r - lo);
+            int64_t pr = 128 * RB[g] + (r - lo), c;
             for (c = 0; c < C; ++c)
                 out[r * C + c] = orc_e4m3_decode(q[r * C + c]) *
                                  orc_scale_value(sf[orc_sf_offset(pr, c / 32, pitch)]);
@@ -344,12 +350,15 @@ int orc_dequantize_colwise(const uint8_t* qT, const uint8_t* sfT, int64_t R, int
     P = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
     group_prefixes(offs, G, R, RB, P);
     for (g = 0; g < G; ++g) {
-        int64_t lo, hi, t, c;
+        int64_t lo, hi, t;
         group_bounds(offs, G, R, g, &lo, &hi);
-        for (t = 0; t < hi - lo; ++t)
+#pragma omp parallel for schedule(static)
+        for (t = 0; t < hi - lo; ++t) {
+            int64_t c;
             for (c = 0; c < C; ++c)
                 out[(lo + t) * C + c] = orc_e4m3_decode(qT[c * ldT + P[g] + t]) *
                                         orc_scale_value(sfT[orc_sf_offset(c, 4 * RB[g] + t / 32, pitch)]);
+        }
     }
     free(RB); free(P);
     return 0;

@@ -146,3 +146,71 @@ def test_fp32_baseline_tracks_fp64_definition():
     np.testing.assert_allclose(dX, oracle.gemm_dgrad(dYf, Wf, offs), rtol=1e-4, atol=1e-4)
     dW = oracle.baseline_wgrad_f32(dY, X, offs, 0, N)
     np.testing.assert_allclose(dW, oracle.gemm_wgrad(dYf, Xf, offs), rtol=1e-4, atol=1e-4)
+
+
+# ------------------------------------------------------------------ per-expert full-size forms
+def _quantised_case(seed, counts, N=256, K=320):
+    """Oracle-quantised operands (all layouts) of a grouped linear, with
+    ragged groups that cross 128-row atom boundaries and an empty expert."""
+    offs = wl.offsets_from_counts(counts)
+    M, E = int(offs[-1]), len(counts)
+    X = wl.normal_bf16((M, K), 1.0, seed + 1)
+    W = wl.normal_bf16((E, N, K), 0.5, seed + 2)
+    dY = wl.normal_bf16((M, N), 1.0, seed + 3)
+    W2 = W.reshape(E * N, K)
+    q = {"x": oracle.quantize_rowwise(X, offs), "w": oracle.quantize_rowwise(W2),
+         "dy": oracle.quantize_rowwise(dY, offs), "wT": oracle.quantize_colwise(W2),
+         "dyT": oracle.quantize_colwise(dY, offs), "xT": oracle.quantize_colwise(X, offs)}
+    return offs, M, E, N, K, q
+
+
+@pytest.mark.parametrize("seed,counts", [(0, [0, 130, 7, 300, 0, 129]), (1, [256, 1, 0, 40])])
+def test_row_and_column_slices_equal_the_full_dequantisation(seed, counts):
+    """rowwise_rows / colwise_rows of one group (or of a 128-aligned run of a
+    one-group operand) equal the matching rows of the whole-tensor
+    dequantisation."""
+    offs, M, E, N, K, q = _quantised_case(seed, counts)
+    cnt = np.diff(offs.astype(np.int64))
+    RB = np.concatenate([[0], np.cumsum((cnt + 127) // 128)])
+    P = np.concatenate([[0], np.cumsum((cnt + 31) // 32 * 32)])
+    Xd = oracle.dequantize_rowwise(*q["x"], offs)
+    Xc = oracle.dequantize_colwise(*q["xT"], M, offs)
+    Wd = oracle.dequantize_rowwise(*q["w"])
+    WdT = oracle.dequantize_colwise(*q["wT"], E * N)
+    for e in range(E):
+        lo, hi = int(offs[e]), int(offs[e + 1])
+        np.testing.assert_array_equal(oracle.rowwise_rows(*q["x"], K, lo, int(RB[e]), hi - lo), Xd[lo:hi])
+        np.testing.assert_array_equal(
+            oracle.colwise_rows(*q["xT"], oracle.colwise_pitch(M, E), int(P[e]), int(RB[e]), hi - lo), Xc[lo:hi])
+        np.testing.assert_array_equal(oracle.rowwise_rows(*q["w"], K, e * N, e * N // 128, N), Wd[e * N:(e + 1) * N])
+        np.testing.assert_array_equal(
+            oracle.colwise_rows(*q["wT"], oracle.colwise_pitch(E * N, 1), e * N, e * N // 128, N),
+            WdT[e * N:(e + 1) * N])
+
+
+@pytest.mark.parametrize("seed,counts", [(2, [0, 130, 7, 300, 0, 129]), (3, [5, 0, 0, 251])])
+def test_per_expert_gemms_equal_the_triple_loop(seed, counts):
+    """The per-expert BLAS forms used at full workload sizes give the
+    triple-loop grouped GEMM of the whole dequantised operands (to fp64
+    summation-order rounding), every expert, empty ones included."""
+    offs, M, E, N, K, q = _quantised_case(seed, counts)
+    Xd = oracle.dequantize_rowwise(*q["x"], offs)
+    Wd = oracle.dequantize_rowwise(*q["w"]).reshape(E, N, K)
+    dYd = oracle.dequantize_rowwise(*q["dy"], offs)
+    WdT = oracle.dequantize_colwise(*q["wT"], E * N).reshape(E, N, K)
+    dYc = oracle.dequantize_colwise(*q["dyT"], M, offs)
+    Xc = oracle.dequantize_colwise(*q["xT"], M, offs)
+    Y, dX, dW = oracle.gemm_fwd(Xd, Wd, offs), oracle.gemm_dgrad(dYd, WdT, offs), oracle.gemm_wgrad(dYc, Xc, offs)
+    seen = set()
+    for e, lo, hi, ye in oracle.fwd_by_expert(*q["x"], *q["w"], offs, N):
+        np.testing.assert_allclose(ye, Y[lo:hi], rtol=1e-12, atol=1e-9)
+        seen.add(e)
+    assert seen == {e for e in range(E) if offs[e + 1] > offs[e]}
+    for e, lo, hi, dxe in oracle.dgrad_by_expert(*q["dy"], *q["wT"], offs, K):
+        np.testing.assert_allclose(dxe, dX[lo:hi], rtol=1e-12, atol=1e-9)
+    got = dict(oracle.wgrad_by_expert(*q["dyT"], *q["xT"], offs, M))
+    assert sorted(got) == list(range(E))
+    for e in range(E):
+        np.testing.assert_allclose(got[e], dW[e], rtol=1e-12, atol=1e-9)
+        if offs[e + 1] == offs[e]:
+            assert np.all(got[e] == 0.0)
