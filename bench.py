@@ -2,13 +2,18 @@
 """Benchmark of the MXFP8 MoE expert-layer hot path on B200.
 
 One step = one pass of the whole path over one synthetic routed batch of the
-DeepSeek-V3-16B-like MoE layer (64 experts, top-6 of 8192 tokens = 49152
-rows; gate/up N = 2816, K = 2048; down N = 2048, K = 1408): for each of the
-two grouped linears, rowwise + colwise MXFP8 quantisation of X, W and dY
-(by default one fused dual-layout kernel per tensor; --quantiser separate
-runs the rowwise and colwise kernels), then the forward, dgrad and wgrad
-grouped GEMMs.  The metric is algorithmic
+DeepSeek-V3-671B-like MoE layer (one GPU's share: 32 local experts, 16384
+routed rows with Zipf(1.1)-skewed counts; gate/up N = 4096, K = 7168; down
+N = 7168, K = 2048): for each of the two grouped linears, rowwise + colwise
+MXFP8 quantisation of X, W and dY (one fused dual-layout kernel per tensor
+by default; --quantiser separate runs the rowwise and colwise kernels),
+then the forward, dgrad and wgrad grouped GEMMs.  The metric is algorithmic
 GEMM TFLOP/s (3 passes x 2*M*N*K per linear over real tokens) per step.
+
+The same JSON line also carries ``per_config``: every grouped GEMM pass of
+the three MoE workloads (DeepSeek-V3-16B-like, DeepSeek-V3-671B-like,
+Llama-4-Scout-like), each launch timed alone with L2 flushed before it, and
+the dual quantiser on their X, W and dY.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -38,7 +43,7 @@ from mxfp8_grouped_gemm_quantize_b200 import workloads as wl  # noqa: E402
 
 METRIC = "MoE grouped-GEMM MXFP8 TFLOP/s (fwd+dgrad+wgrad) and % of B200 FP8 peak"
 UNIT = "TFLOP/s"
-WORKLOAD = "ds-v3-16b"
+WORKLOAD = "ds-v3-671b"
 FP8_OVER_BF16 = 2.0   # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
 
 
@@ -56,12 +61,18 @@ def parse():
     # profiling aids (the headline line uses the defaults)
     ap.add_argument("--linears", default="all", help="comma-separated subset of the workload's linears")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the measurements outside the step (e2e, quantising epilogue, MoE dispatch, NVFP4, "
-                         "quantiser sweep)")
+                    help="skip the measurements outside the step (e2e, per-config passes, quantising epilogue, MoE "
+                         "dispatch, NVFP4, quantiser sweep)")
+    ap.add_argument("--per-config-iters", type=int, default=10)
     return ap.parse_args()
 
 
-GEMM_PROFILE = os.path.join(ROOT, "profiles", "grouped_gemm_ds-v3-16b_gate_up.md")
+# DRAM traffic of one grouped_gemm_kernel launch from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum, mean over the fwd, dgrad and
+# wgrad launches of the workload named below).  The figure belongs to the
+# kernel sources it was taken on: when their hash differs the line reports
+# null instead.
+GEMM_TRAFFIC = {"bytes_per_launch": None, "workload": None, "sources_sha256": None}
 GEMM_SOURCES = ("grouped_gemm.cu", "ptx.cuh", "codec.cuh", "launch.h", "tmap.cu")
 
 
@@ -75,20 +86,11 @@ def gemm_sources_sha256() -> str:
 
 
 def gemm_traffic():
-    """DRAM bytes per GEMM launch from the committed ncu summary (the mean over
-    the gate/up linear's fwd, dgrad and wgrad launches), or None when the
-    summary is missing or the kernel sources changed since it was taken."""
-    try:
-        kv = {}
-        for line in open(GEMM_PROFILE, encoding="utf-8"):
-            if ":" in line and line.split(":")[0].strip() in ("traffic_bytes_per_launch", "kernel_sources_sha256"):
-                k, v = line.split(":", 1)
-                kv[k.strip()] = v.strip().strip("`")
-        if kv.get("kernel_sources_sha256") != gemm_sources_sha256():
-            return None
-        return int(kv["traffic_bytes_per_launch"])
-    except (OSError, KeyError, ValueError):
-        return None
+    """(bytes per GEMM launch, workload it was captured on), or (None, None)
+    when no capture exists for the current kernel sources."""
+    if GEMM_TRAFFIC["sources_sha256"] != gemm_sources_sha256():
+        return None, None
+    return GEMM_TRAFFIC["bytes_per_launch"], GEMM_TRAFFIC["workload"]
 
 
 def peaks():
@@ -191,10 +193,10 @@ class Linear:
         reads = 1 if self.quantiser == "dual" else 2
         return el * (2 * reads + 2 * (1 + 1 / 32))
 
-    def launches(self):
-        """(kind, callable) for one pass of the path; kind is 'quant' or 'gemm:<pass>'."""
+    def passes(self):
+        """{pass: callable} for the three grouped GEMMs of this linear."""
         mx = self.mx
-        gemms = {
+        return {
             "fwd": lambda: mx.mxfp8_grouped_gemm_fwd(self.xq, self.xs, self.wq, self.ws, self.offs, self.N,
                                                      out=self.y, work=self.work),
             "dgrad": lambda: mx.mxfp8_grouped_gemm_dgrad(self.dyq, self.dys, self.wqT, self.wsT, self.offs, self.K,
@@ -202,28 +204,36 @@ class Linear:
             "wgrad": lambda: mx.mxfp8_grouped_gemm_wgrad(self.dyqT, self.dysT, self.xqT, self.xsT, self.offs, self.M,
                                                          out=self.dw, work=self.work),
         }
+
+    def dual_quantisations(self):
+        """The three dual quantisations (X, W, dY: both layouts from one read)."""
+        mx = self.mx
+        return [
+            lambda: mx.mxfp8_quantize_dual(self.X, self.offs, q=self.xq, scales=self.xs, qT=self.xqT,
+                                           scalesT=self.xsT),
+            lambda: mx.mxfp8_quantize_dual(self.W2, None, q=self.wq, scales=self.ws, qT=self.wqT, scalesT=self.wsT),
+            lambda: mx.mxfp8_quantize_dual(self.dY, self.offs, q=self.dyq, scales=self.dys, qT=self.dyqT,
+                                           scalesT=self.dysT),
+        ]
+
+    def launches(self):
+        """(kind, callable) for one pass of the path; kind is 'quant' or 'gemm:<pass>'."""
+        mx = self.mx
+        g = self.passes()
         if self.quantiser == "dual":
-            return [
-                ("quant", lambda: mx.mxfp8_quantize_dual(self.X, self.offs, q=self.xq, scales=self.xs, qT=self.xqT,
-                                                         scalesT=self.xsT)),
-                ("quant", lambda: mx.mxfp8_quantize_dual(self.W2, None, q=self.wq, scales=self.ws, qT=self.wqT,
-                                                         scalesT=self.wsT)),
-                ("gemm:fwd", gemms["fwd"]),
-                ("quant", lambda: mx.mxfp8_quantize_dual(self.dY, self.offs, q=self.dyq, scales=self.dys,
-                                                         qT=self.dyqT, scalesT=self.dysT)),
-                ("gemm:dgrad", gemms["dgrad"]),
-                ("gemm:wgrad", gemms["wgrad"]),
-            ]
+            qx, qw, qdy = self.dual_quantisations()
+            return [("quant", qx), ("quant", qw), ("gemm:fwd", g["fwd"]), ("quant", qdy),
+                    ("gemm:dgrad", g["dgrad"]), ("gemm:wgrad", g["wgrad"])]
         return [
             ("quant", lambda: mx.mxfp8_quantize_rowwise(self.X, self.offs, q=self.xq, scales=self.xs)),
             ("quant", lambda: mx.mxfp8_quantize_rowwise(self.W2, None, q=self.wq, scales=self.ws)),
-            ("gemm:fwd", gemms["fwd"]),
+            ("gemm:fwd", g["fwd"]),
             ("quant", lambda: mx.mxfp8_quantize_rowwise(self.dY, self.offs, q=self.dyq, scales=self.dys)),
             ("quant", lambda: mx.mxfp8_quantize_colwise(self.W2, None, qT=self.wqT, scales=self.wsT)),
-            ("gemm:dgrad", gemms["dgrad"]),
+            ("gemm:dgrad", g["dgrad"]),
             ("quant", lambda: mx.mxfp8_quantize_colwise(self.dY, self.offs, qT=self.dyqT, scales=self.dysT)),
             ("quant", lambda: mx.mxfp8_quantize_colwise(self.X, self.offs, qT=self.xqT, scales=self.xsT)),
-            ("gemm:wgrad", gemms["wgrad"]),
+            ("gemm:wgrad", g["wgrad"]),
         ]
 
 
@@ -246,14 +256,22 @@ def system_info(device_index: int = 0) -> dict:
     return info
 
 
+ROUTING = {
+    "tiny": "counts [0, 7, 21, 36]",
+    "ds-v3-16b": "top-6 of 64 experts over 8192 tokens; N(0,1) logits + N(0,0.5) expert bias",
+    "ds-v3-671b": "one GPU's share of top-8 of 256 experts over 16384 tokens: 32 local experts, 16384 rows, "
+                  "Multinomial counts with Zipf(1.1) weights in a seeded order",
+    "llama4-scout": "top-1 of 16 experts over 16384 tokens; N(0,1) logits",
+}
+
+
 def workload_config(w, quantiser: str, world: int) -> dict:
     """The `config` object of the JSON line, identical for both arms."""
     return {"workload": f"{w.name}-like MoE layer", "experts": w.E, "routed_rows": w.M,
             "layers": [{"name": L.name, "N": L.N, "K": L.K} for L in w.layers],
-            "routing": ("top-6 of 8192 tokens, N(0,1) logits + N(0,0.5) expert bias" if w.name == "ds-v3-16b"
-                        else w.name),
-            "l2": "inputs larger than L2 (step touches > 2 GB)", "parallelism": f"replica x{world}",
-            "quantiser": quantiser}
+            "routing": ROUTING.get(w.name, w.name),
+            "l2": "inputs larger than L2 (126 MB): the step's operands are several GB",
+            "parallelism": f"replica x{world}", "quantiser": quantiser}
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -329,6 +347,7 @@ def run_ours(args, rank, world, local_rank):
 
     pk = peaks()
     fp8_peak = pk["bf16"] * FP8_OVER_BF16
+    traffic, traffic_wl = gemm_traffic()
     gemm_ms = sum(sum(v) for k, v in per_kind.items() if k.startswith("gemm")) / K
     gemm_launches = sum(len(v) for k, v in per_kind.items() if k.startswith("gemm"))
     gemm_tflops = step_flops / (gemm_ms * 1e-3) / 1e12
@@ -348,10 +367,10 @@ def run_ours(args, rank, world, local_rank):
         "fraction_of_fp8_peak": round(value / world / fp8_peak, 4),
         "roofline": {"kernel": "grouped_gemm_kernel (fwd+dgrad+wgrad launches)", "bound": "tensor",
                      "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(gemm_tflops / fp8_peak, 4), "traffic": gemm_traffic(),
-                     "traffic_source": "mean DRAM read+write bytes per launch over the gate/up linear's fwd, dgrad "
-                                       "and wgrad launches, ncu (profiles/grouped_gemm_ds-v3-16b_gate_up.md); null "
-                                       "if the kernel sources changed since",
+                     "frac": round(gemm_tflops / fp8_peak, 4), "traffic": traffic,
+                     "traffic_source": (f"ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, mean over the "
+                                        f"fwd, dgrad and wgrad launches of {traffic_wl}" if traffic is not None else
+                                        "no ncu capture of the current kernel sources"),
                      "peak_source": f"{pk['src']} bf16 burst x {FP8_OVER_BF16} (nominal FP8/BF16)",
                      "launches_timed": gemm_launches},
         "quantiser": {"achieved_gbs": round(quant_gbs, 1), "peak_gbs": pk["hbm_gbs"],
@@ -367,11 +386,86 @@ def run_ours(args, rank, world, local_rank):
         out["config"]["linears_timed"] = [L.name for L in layers]
     if not args.no_extras:
         out["e2e"] = e2e(args, mx, w, layers, dev, world)
+        out["per_config"] = per_config(mx, args, fp8_peak, pk["hbm_gbs"], dev, local_rank)
+        c2 = out["per_config"].get("ds-v3-671b")
+        if c2 is not None:
+            out["fwd_frac"] = {"workload": "ds-v3-671b-like MoE layer, both linears, forward launches timed alone",
+                               "tflops": c2["passes"]["fwd"]["tflops"], "frac": c2["passes"]["fwd"]["frac"],
+                               "target": 0.60, "peak": round(fp8_peak, 1)}
         out["quantising_epilogue"] = quantising_epilogue(mx, layers[0])
         out["moe_dispatch"] = moe_dispatch(mx, args, pk["hbm_gbs"])
         out["nvfp4"] = nvfp4_measure(mx, layers[0], fp8_peak, pk["hbm_gbs"])
         out["quantiser_sweep"] = quantiser_sweep(mx, pk["hbm_gbs"])
     return out
+
+
+def timed_alone(fn, flush, iters):
+    """Median CUDA-event time (ms) of one launch with L2 flushed before it."""
+    for _ in range(2):
+        fn()
+    ts = []
+    for _ in range(iters):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def per_config(mx, args, fp8_peak, hbm_gbs, dev, device_index):
+    """Every grouped GEMM pass (fwd, dgrad, wgrad of both linears) of the three
+    MoE workloads, each launch timed alone with L2 flushed before it (median
+    of --per-config-iters), and the dual quantiser on each linear's X, W and
+    dY timed the same way.  TFLOP/s are algorithmic (2*M*N*K over real
+    tokens); fractions are of the FP8 peak of the roofline."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * max(l2, 64 << 20), dtype=torch.uint8, device=dev)
+    it = max(3, args.per_config_iters)
+    res = {}
+    with ClockSampler(device_index) as clk:
+        for name in ("ds-v3-16b", "ds-v3-671b", "llama4-scout"):
+            w = wl.WORKLOADS[name]()
+            cfg = {"routing": ROUTING[name], "experts": w.E, "routed_rows": w.M, "linears": {}}
+            tot = {p: [0.0, 0.0] for p in ("fwd", "dgrad", "wgrad")}
+            q_bytes, q_ms = 0.0, 0.0
+            for layer in w.layers:
+                L = Linear(mx, w, layer, dev, "dual")
+                for fn in L.dual_quantisations():
+                    fn()
+                r = {"N": L.N, "K": L.K}
+                for p, fn in L.passes().items():
+                    ms = timed_alone(fn, flush, it)
+                    fl = L.flops_per_pass()
+                    tot[p][0] += fl
+                    tot[p][1] += ms
+                    r[p] = {"ms": round(ms, 4), "tflops": round(fl / (ms * 1e-3) / 1e12, 1),
+                            "frac": round(fl / (ms * 1e-3) / 1e12 / fp8_peak, 4)}
+                if mx.mxfp8_get_status(L.work) != 0:
+                    raise SystemExit(f"bench: device status error in the {name} {layer.name} passes")
+                for fn in L.dual_quantisations():
+                    q_ms += timed_alone(fn, flush, it)
+                q_bytes += L.quant_bytes()
+                cfg["linears"][layer.name] = r
+                del L
+                torch.cuda.empty_cache()
+            cfg["passes"] = {p: {"tflops": round(f / (ms * 1e-3) / 1e12, 1),
+                                 "frac": round(f / (ms * 1e-3) / 1e12 / fp8_peak, 4)} for p, (f, ms) in tot.items()}
+            f_all, ms_all = sum(v[0] for v in tot.values()), sum(v[1] for v in tot.values())
+            cfg["all_passes"] = {"tflops": round(f_all / (ms_all * 1e-3) / 1e12, 1),
+                                 "frac": round(f_all / (ms_all * 1e-3) / 1e12 / fp8_peak, 4)}
+            gbs = q_bytes / (q_ms * 1e-3) / 1e9
+            cfg["quantiser"] = {"kernel": "quantize_dual_kernel (X, W, dY of both linears)", "ms": round(q_ms, 4),
+                                "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4)}
+            res[name] = cfg
+    del flush
+    torch.cuda.empty_cache()
+    res["method"] = (f"each launch alone, L2 flushed before it ({2 * max(l2, 64 << 20) >> 20} MiB written), "
+                     f"median of {it}")
+    res["clocks"] = clk.summary()
+    return res
 
 
 def e2e(args, mx, w, layers, dev, world):

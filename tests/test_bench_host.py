@@ -1,6 +1,5 @@
 """bench.py host logic that needs no GPU: the roofline's traffic figure is
-read from the committed ncu summary only while the kernel sources are the
-ones it was taken on, the peaks come from the measured file, and the clock
+reported only while the kernel sources are the ones it was taken on, the peaks come from the measured file, and the clock
 sampler decodes throttle reasons from a fake NVML (it only reads)."""
 import os
 import sys
@@ -11,21 +10,18 @@ sys.path.insert(0, ROOT)
 import bench  # noqa: E402
 
 
-def test_traffic_is_read_while_the_sources_match():
-    t = bench.gemm_traffic()
-    assert isinstance(t, int) and 5e8 < t < 1.5e9       # DRAM bytes per GEMM launch, DS-16B gate/up
-
-
-def test_traffic_is_null_once_the_sources_change(tmp_path, monkeypatch):
-    prof = tmp_path / "profile.md"
-    text = open(bench.GEMM_PROFILE, encoding="utf-8").read()
-    prof.write_text(text)
-    monkeypatch.setattr(bench, "GEMM_PROFILE", str(prof))
-    assert bench.gemm_traffic() is not None
+def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(monkeypatch):
+    monkeypatch.setattr(bench, "GEMM_TRAFFIC", {"bytes_per_launch": 123456789, "workload": "w",
+                                                "sources_sha256": bench.gemm_sources_sha256()})
+    assert bench.gemm_traffic() == (123456789, "w")
     monkeypatch.setattr(bench, "gemm_sources_sha256", lambda: "0" * 64)
-    assert bench.gemm_traffic() is None
-    monkeypatch.setattr(bench, "GEMM_PROFILE", str(tmp_path / "missing.md"))
-    assert bench.gemm_traffic() is None
+    assert bench.gemm_traffic() == (None, None)
+
+
+def test_the_committed_traffic_figure_is_consistent():
+    t = bench.GEMM_TRAFFIC
+    if t["sources_sha256"] is not None:
+        assert len(t["sources_sha256"]) == 64 and 1e8 < t["bytes_per_launch"] < 1e10 and t["workload"]
 
 
 def test_the_source_hash_covers_the_gemm_sources():
@@ -98,5 +94,14 @@ def test_reference_arm_prints_one_contract_line():
     assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     from mxfp8_grouped_gemm_quantize_b200 import workloads as wl
-    assert d["config"] == bench.workload_config(wl.ds_v3_16b(), "dual", 1)
+    assert d["config"] == bench.workload_config(wl.ds_v3_671b(), "dual", 1)
     assert d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+
+
+def test_the_headline_is_the_671b_like_layer():
+    from mxfp8_grouped_gemm_quantize_b200 import workloads as wl
+    assert bench.WORKLOAD == "ds-v3-671b"
+    c = bench.workload_config(wl.ds_v3_671b(), "dual", 1)
+    assert c["workload"] == "ds-v3-671b-like MoE layer" and c["routed_rows"] == 16384 and c["experts"] == 32
+    assert c["layers"] == [{"name": "gate_up", "N": 4096, "K": 7168}, {"name": "down", "N": 7168, "K": 2048}]
+    assert "Zipf" in c["routing"]
