@@ -85,7 +85,7 @@ typedef enum {
     MXF8_ERR_CUDA = 4,         /* a CUDA call failed; see mxfp8_last_cuda_error() */
     MXF8_ERR_BAD_OFFSETS = 5,  /* device side: d_offs is not a valid prefix of `rows` */
     MXF8_ERR_TIMEOUT = 6,      /* device side: a pipeline wait ran past its limit (2 s); tests provoke it
-                                  by setting MXF8_TEST_SKIP_FIRST_STAGE in the environment */
+                                  with mxfp8_testing_stall_first_stage */
     MXF8_ERR_BAD_ROUTING = 7   /* device side: an expert id outside [0, num_experts) */
 } mxf8_status;
 
@@ -233,6 +233,9 @@ MXF8_API mxf8_status mxfp8_grouped_gemm_dgrad_quant(const uint8_t* dyq, const ui
  * every GPU that loads the library until the process exits.
  *   - The first call on a device looks up that array's device address (with
  *     the device current); make that first call before any stream capture.
+ *     The address is kept for the life of the process: after a
+ *     cudaDeviceReset on that device it is stale, so do not call this entry
+ *     point on a device that has been reset.
  *   - Every call on a device shares the one array; its status word is cleared
  *     at the start of each call, but calls that overlap on the GPU (other
  *     streams, other host threads) race on it.
@@ -247,6 +250,27 @@ MXF8_API mxf8_status mxfp8_grouped_gemm_fwd_noalloc(const uint8_t* xq, const uin
                                                     const int32_t* d_offs, int32_t E, int64_t M, int64_t N,
                                                     int64_t K, uint16_t* y, int32_t* host_status,
                                                     void* stream);
+
+/* ---------------------------------------------------------------- tuning and testing switches */
+
+/* Overrides, for the calling process, the tile configuration the grouped
+ * GEMMs (MXFP8) choose per pass.  The pages fix no tiling; these are this
+ * library's own pipeline shapes.
+ *   cta_pair  -1 = the library's rule, 0 = 1-CTA 128x256 tiles,
+ *             1 = CTA-pair 256x256 tiles (cta_group::2)
+ *   stage_k   -1 = the library's rule, 1 = 128-deep K stages, 2 = 256-deep
+ * Results are the same under every setting (same products, same fp32
+ * accumulation order within a 32-element step); only speed changes.  Returns
+ * MXF8_ERR_INVALID_ARG for any other value.  Not thread-safe against
+ * concurrent GEMM calls. */
+MXF8_API mxf8_status mxfp8_set_gemm_tiling(int32_t cta_pair, int32_t stage_k);
+
+/* Test switch for the bounded pipeline waits: while enabled (enable != 0),
+ * every grouped GEMM launch leaves its first pipeline stage unfilled, so the
+ * MMA warp's wait on it runs out after the 2 s limit; the kernel drains what
+ * it issued, frees tensor memory and returns with MXF8_ERR_TIMEOUT in the
+ * workspace status.  Off by default; meant only for tests of that path. */
+MXF8_API void mxfp8_testing_stall_first_stage(int32_t enable);
 
 /* ---------------------------------------------------------------- MoE dispatch / combine */
 /* The steps around the grouped GEMM in a Mixture-of-Experts layer on one

@@ -40,7 +40,8 @@ EXPORTED = ("mxfp8_rowwise_scale_bytes", "mxfp8_colwise_pitch", "mxfp8_colwise_s
             "mxfp8_permute_quantize_dual", "mxfp8_moe_combine", "mxfp8_nvfp4_rowwise_scale_bytes",
             "mxfp8_nvfp4_colwise_pitch", "mxfp8_nvfp4_colwise_scale_bytes", "mxfp8_nvfp4_colwise_ld",
             "mxfp8_nvfp4_amax", "mxfp8_nvfp4_quantize_rowwise", "mxfp8_nvfp4_quantize_colwise",
-            "mxfp8_nvfp4_grouped_gemm_fwd", "mxfp8_nvfp4_grouped_gemm_dgrad", "mxfp8_nvfp4_grouped_gemm_wgrad")
+            "mxfp8_nvfp4_grouped_gemm_fwd", "mxfp8_nvfp4_grouped_gemm_dgrad", "mxfp8_nvfp4_grouped_gemm_wgrad",
+            "mxfp8_set_gemm_tiling", "mxfp8_testing_stall_first_stage")
 
 
 class MXFP8Error(RuntimeError):
@@ -116,6 +117,10 @@ def lib() -> ctypes.CDLL:
         L.mxfp8_status_string.argtypes = [_i32]
         L.mxfp8_last_cuda_error.restype = ctypes.c_char_p
         L.mxfp8_device_supported.restype = _i32
+        L.mxfp8_set_gemm_tiling.restype = _i32
+        L.mxfp8_set_gemm_tiling.argtypes = [_i32, _i32]
+        L.mxfp8_testing_stall_first_stage.restype = None
+        L.mxfp8_testing_stall_first_stage.argtypes = [_i32]
         _LIB = L
     return _LIB
 
@@ -314,6 +319,20 @@ def mxfp8_get_status(work: torch.Tensor, stream=None) -> int:
 
 def mxfp8_device_supported() -> bool:
     return bool(lib().mxfp8_device_supported())
+
+
+def mxfp8_set_gemm_tiling(cta_pair: int = -1, stage_k: int = -1) -> None:
+    """Process-wide override of the grouped GEMMs' tile configuration
+    (-1 = the library's rule; cta_pair 0/1 = 1-CTA / CTA-pair tiles; stage_k
+    1/2 = 128- / 256-deep K stages).  Results do not change, only speed."""
+    _check(lib().mxfp8_set_gemm_tiling(int(cta_pair), int(stage_k)), "mxfp8_set_gemm_tiling")
+
+
+def mxfp8_testing_stall_first_stage(enable: bool) -> None:
+    """Test switch: while on, every grouped GEMM launch leaves its first
+    pipeline stage unfilled and ends with MXF8_ERR_TIMEOUT after its 2 s
+    bounded wait (the workspace status reports it)."""
+    lib().mxfp8_testing_stall_first_stage(1 if enable else 0)
 
 
 # ------------------------------------------------------------------ MoE dispatch / combine

@@ -2,9 +2,11 @@
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import subprocess
 import sys
+import tempfile
 from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
@@ -38,7 +40,9 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return OUT
-    objdir = os.path.join(ROOT, "_build")
+    # object files go outside the source tree (only the library lives in-tree)
+    tag = hashlib.sha256(PKG.encode()).hexdigest()[:12]
+    objdir = os.path.join(tempfile.gettempdir(), f"mxfp8_build_{tag}")
     os.makedirs(objdir, exist_ok=True)
     extra = ["-Xptxas", "-v"] if verbose else []
 

@@ -3,6 +3,7 @@
 // allocates device memory.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -15,7 +16,7 @@ namespace {
 thread_local char g_last_error[256] = "";
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;   // a pipeline wait gives up after 2 s
-constexpr int64_t kWorkspaceBytes = 256;                 // status word + reserve
+constexpr int64_t kWorkspaceBytes = mxf8::kGemmWorkspaceBytes;   // status word + reserve
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int64_t round_up(int64_t a, int64_t b) { return cdiv(a, b) * b; }
@@ -23,9 +24,13 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int64_t blocks128_bound(int64_t rows, int32_t G) { return rows <= 0 ? 0 : cdiv(rows, 128) + G - 1; }
 
+// Switches set through mxfp8_testing_stall_first_stage / mxfp8_set_gemm_tiling.
+std::atomic<int> g_stall_first_stage{0};
+std::atomic<int> g_tiling_cta_pair{-1};
+std::atomic<int> g_tiling_stage_k{-1};
+
 mxf8_status cuda_fail(cudaError_t e, const char* where, const char* detail = nullptr) {
-  std::snprintf(g_last_error, sizeof g_last_error, "%s: %s%s%s", where, cudaGetErrorString(e),
-                detail ? " -- " : "", detail ? detail : "");
+  mxf8::record_cuda_error(e, where, detail);
   return MXF8_ERR_CUDA;
 }
 
@@ -81,10 +86,10 @@ mxf8_status run_gemm(mxf8::GemmArgs& g, void* work, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   g.status = static_cast<int32_t*>(work);
   g.timeout_ns = kDefaultTimeoutNs;
-  // Test hook for the bounded-wait path: with MXF8_TEST_SKIP_FIRST_STAGE set,
-  // a 1-CTA launch leaves its first pipeline stage unfilled and the device
+  // Test switch for the bounded-wait path (mxfp8_testing_stall_first_stage):
+  // the launch leaves its first pipeline stage unfilled and the device
   // status becomes MXF8_ERR_TIMEOUT after the wait limit.
-  g.inject_skip_stage = std::getenv("MXF8_TEST_SKIP_FIRST_STAGE") != nullptr ? 1 : 0;
+  g.inject_skip_stage = g_stall_first_stage.load(std::memory_order_relaxed);
   cudaError_t e = cudaMemsetAsync(work, 0, sizeof(int32_t), st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   const char* detail = nullptr;
@@ -116,7 +121,32 @@ mxf8_status attach_quant_outputs(mxf8::GemmArgs& g, int64_t C, const uint16_t* o
 
 }  // namespace
 
+namespace mxf8 {
+
+void record_cuda_error(cudaError_t e, const char* where, const char* detail) {
+  std::snprintf(g_last_error, sizeof g_last_error, "%s: %s%s%s", where, cudaGetErrorString(e),
+                detail ? " -- " : "", detail ? detail : "");
+}
+
+void gemm_tiling_override(int* cta_pair, int* stage_k) {
+  *cta_pair = g_tiling_cta_pair.load(std::memory_order_relaxed);
+  *stage_k = g_tiling_stage_k.load(std::memory_order_relaxed);
+}
+
+}  // namespace mxf8
+
 extern "C" {
+
+mxf8_status mxfp8_set_gemm_tiling(int32_t cta_pair, int32_t stage_k) {
+  if (cta_pair < -1 || cta_pair > 1 || stage_k < -1 || stage_k == 0 || stage_k > 2) return MXF8_ERR_INVALID_ARG;
+  g_tiling_cta_pair.store(cta_pair, std::memory_order_relaxed);
+  g_tiling_stage_k.store(stage_k, std::memory_order_relaxed);
+  return MXF8_OK;
+}
+
+void mxfp8_testing_stall_first_stage(int32_t enable) {
+  g_stall_first_stage.store(enable != 0 ? 1 : 0, std::memory_order_relaxed);
+}
 
 int64_t mxfp8_rowwise_scale_bytes(int64_t rows, int64_t cols, int32_t num_groups) {
   if (rows < 0 || cols <= 0 || num_groups < 1) return 0;

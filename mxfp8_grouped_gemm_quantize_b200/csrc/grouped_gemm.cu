@@ -839,11 +839,11 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   // rows per group in fwd/dgrad).  Stage depth: 128-deep stages (4-stage
   // ring) except for long K loops -- fwd/dgrad with at least 64 K blocks,
   // wgrad with at least 1024 rows per group on average -- where 256-deep
-  // stages (2-stage ring) measured faster.  MXF8_GEMM_CTA_PAIR=1/0 and
-  // MXF8_GEMM_KS=1/2 override the choices.
-  int cg = 1;
-  const char* env = std::getenv("MXF8_GEMM_CTA_PAIR");
-  if (env && std::strcmp(env, "1") == 0) cg = 2;
+  // stages (2-stage ring) measured faster.  mxfp8_set_gemm_tiling overrides
+  // either choice.
+  int force_cg = -1, force_ks = -1;
+  gemm_tiling_override(&force_cg, &force_ks);
+  int cg = force_cg == 1 ? 2 : 1;
   int ks = 1;
   if (a.mode == kWgrad) {
     if (a.M >= int64_t(1024) * a.E) ks = 2;
@@ -851,9 +851,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
     const int64_t kblocks = ((a.mode == kFwd ? a.K : a.N) + BK - 1) / BK;
     if (kblocks >= 64) ks = 2;
   }
-  env = std::getenv("MXF8_GEMM_KS");
-  if (env && std::strcmp(env, "1") == 0) ks = 1;
-  if (env && std::strcmp(env, "2") == 0) ks = 2;
+  if (force_ks == 1 || force_ks == 2) ks = force_ks;
   if (a.fp4) { cg = 1; ks = 1; }   // NVFP4: one configuration (1-CTA, 3 x 128-byte stages)
   const uint32_t sf_box_rows = 4 * ks * (a.fp4 ? 4 : 1);
   const int64_t out_rows = a.mode == kWgrad ? int64_t(a.E) * a.N : a.M;

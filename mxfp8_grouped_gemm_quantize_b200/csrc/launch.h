@@ -6,6 +6,10 @@
 
 namespace mxf8 {
 
+// Bytes of the workspace every grouped GEMM takes: its status word and a
+// reserve (mxfp8_workspace_bytes).
+constexpr int64_t kGemmWorkspaceBytes = 256;
+
 // 2D TMA map over a row-major matrix [rows, cols] of `esize`-byte elements
 // with row stride `ld` elements; box = box_cols x box_rows; zero fill
 // outside the matrix.  False if the driver rejects it.
@@ -82,5 +86,11 @@ struct GemmArgs {
 // Returns cudaSuccess or the CUDA error; *detail gets a short reason for
 // failures detected before the launch (tensor-map encoding).
 cudaError_t launch_grouped_gemm(const GemmArgs& args, cudaStream_t stream, const char** detail);
+
+// Process-wide tile overrides set through mxfp8_set_gemm_tiling (-1 = rule).
+void gemm_tiling_override(int* cta_pair, int* stage_k);
+
+// Records a CUDA failure for mxfp8_last_cuda_error (thread-local text).
+void record_cuda_error(cudaError_t e, const char* where, const char* detail);
 
 }  // namespace mxf8

@@ -12,7 +12,11 @@
 
 #include <mutex>
 
+#include "launch.h"
 #include "mxfp8.h"
+
+static_assert(MXF8_NOALLOC_SCRATCH_BYTES >= mxf8::kGemmWorkspaceBytes,
+              "the static scratch must hold a grouped GEMM workspace");
 
 namespace {
 
@@ -55,7 +59,10 @@ extern "C" mxf8_status mxfp8_grouped_gemm_fwd_noalloc(const uint8_t* xq, const u
   if (mxfp8_workspace_bytes(E, M, N, K) > MXF8_NOALLOC_SCRATCH_BYTES) return MXF8_ERR_INVALID_ARG;
   cudaError_t err = cudaSuccess;
   void* scratch = scratch_for_current_device(&err);
-  if (!scratch) return MXF8_ERR_CUDA;
+  if (!scratch) {
+    mxf8::record_cuda_error(err, "mxfp8_grouped_gemm_fwd_noalloc: scratch address lookup", nullptr);
+    return MXF8_ERR_CUDA;
+  }
   // The forward entry point clears the status word in the scratch before its
   // launch, so the last call's contents never leak into this one.
   mxf8_status s = mxfp8_grouped_gemm_fwd(xq, xs, xs_bytes, wq, ws, ws_bytes, d_offs, E, M, N, K, y, scratch,

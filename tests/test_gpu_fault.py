@@ -1,13 +1,11 @@
 """The GEMM's bounded pipeline waits, exercised on the GPU without faulting it.
 
-With MXF8_TEST_SKIP_FIRST_STAGE set, the producer of every CTA leaves its
-first pipeline stage unfilled (no copies, no arrival): the MMA warp's wait on
-it is a flag that nothing sets.  The wait must give up after its limit, the
+With the library's test switch mxfp8_testing_stall_first_stage on, the
+producer of every CTA leaves its first pipeline stage unfilled (no copies, no
+arrival): the MMA warp's wait on it is a flag that nothing sets.  The wait must give up after its limit, the
 kernel must drain what it had in flight and return, the device status must
 read MXF8_ERR_TIMEOUT, and the context must stay usable: the next launch
 without the hook produces the oracle's result."""
-import os
-
 import numpy as np
 import pytest
 import torch
@@ -42,12 +40,12 @@ def test_unfilled_stage_times_out_and_the_context_stays_usable(mx):
     work = mx.new_workspace(E, M, N, K)
     y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
 
-    os.environ["MXF8_TEST_SKIP_FIRST_STAGE"] = "1"
+    mx.mxfp8_testing_stall_first_stage(True)
     try:
         mx.mxfp8_grouped_gemm_fwd(xq, xs, wq, ws, od, N, out=y, work=work)
         torch.cuda.synchronize()
     finally:
-        del os.environ["MXF8_TEST_SKIP_FIRST_STAGE"]
+        mx.mxfp8_testing_stall_first_stage(False)
     assert mx.mxfp8_get_status(work) == TIMEOUT
 
     mx.mxfp8_grouped_gemm_fwd(xq, xs, wq, ws, od, N, out=y, work=work)

@@ -20,18 +20,18 @@ POISON = 0x7FC0  # bf16 NaN: any output element the kernel fails to write stays 
 
 
 @pytest.fixture(params=["default", "1cta-ks1", "1cta-ks2", "pair-ks1", "pair-ks2"])
-def tile_config(request, monkeypatch):
+def tile_config(request):
     """Runs a test under the per-pass default tile configuration and under
     each forced one: 1-CTA 128x256 or CTA-pair 256x256 tiles, with 128-deep
     (ks1) or 256-deep (ks2) pipeline stages."""
+    import mxfp8_grouped_gemm_quantize_b200 as m
     if request.param == "default":
-        monkeypatch.delenv("MXF8_GEMM_CTA_PAIR", raising=False)
-        monkeypatch.delenv("MXF8_GEMM_KS", raising=False)
+        m.mxfp8_set_gemm_tiling(-1, -1)
     else:
         tiles, ks = request.param.split("-")
-        monkeypatch.setenv("MXF8_GEMM_CTA_PAIR", "1" if tiles == "pair" else "0")
-        monkeypatch.setenv("MXF8_GEMM_KS", ks[-1])
-    return request.param
+        m.mxfp8_set_gemm_tiling(1 if tiles == "pair" else 0, int(ks[-1]))
+    yield request.param
+    m.mxfp8_set_gemm_tiling(-1, -1)
 
 
 @pytest.fixture(scope="module")
