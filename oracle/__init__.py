@@ -74,6 +74,9 @@ def lib():
         L.orc_bf16_from_double.restype = ctypes.c_uint16
         L.orc_bf16_from_double.argtypes = [ctypes.c_double]
         L.orc_bf16_from_double_array.argtypes = [_vp, _i64, _vp]
+        L.orc_silu.restype = ctypes.c_double
+        L.orc_silu.argtypes = [ctypes.c_double]
+        L.orc_swiglu.argtypes = [_vp, _i64, _i64, _vp]
         L.orc_e2m1_decode.restype = ctypes.c_double
         L.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
         L.orc_e2m1_encode.restype = ctypes.c_uint8
@@ -589,3 +592,20 @@ def nvfp4_dequantize_colwise(qT, sf, R: int, S, offs=None) -> np.ndarray:
     _check(lib().orc_nvfp4_dequantize_colwise(_p(qT), _p(np.ascontiguousarray(sf)), R, C, _p(o), G, float(S),
                                               _p(out)), "nvfp4_dequantize_colwise")
     return out
+
+
+# ---------------------------------------------------------------- SwiGLU between the two linears
+def silu(g: float) -> float:
+    """silu(g) = g / (1 + exp(-g)) in fp64."""
+    return lib().orc_silu(float(g))
+
+
+def swiglu(Y) -> np.ndarray:
+    """Y: fp64 [M, 2I] gate/up output (gate = columns 0..I-1, up = I..2I-1)
+    -> bf16 bits [M, I] of silu(gate) * up, fp64 then one nearest-even rounding."""
+    Y = np.ascontiguousarray(np.asarray(Y, dtype=np.float64))
+    M, N2 = Y.shape
+    assert N2 % 2 == 0
+    h = np.zeros((M, N2 // 2), dtype=np.uint16)
+    _check(lib().orc_swiglu(_p(Y), M, N2 // 2, _p(h)), "swiglu")
+    return h

@@ -721,6 +721,34 @@ void orc_bf16_from_double_array(const double* v, int64_t n, uint16_t* out)
 }
 
 /* ------------------------------------------------------------------ */
+/* SwiGLU between the two grouped linears of an expert                  */
+/* ------------------------------------------------------------------ */
+/* The MXFP8 speed-up comes from the expert pipeline as a whole
+ * (opensourcebeat.com, section "Двухсторонняя атака: MXFP8 и DeepEP"); the
+ * DeepSeek-V3 and Llama 4 experts the workloads model apply SwiGLU between
+ * their gate/up and down projections.  The pages give no formula, so the
+ * plainest reading: the gate/up output Y [M, 2I] holds the gate in columns
+ * 0 .. I-1 and the up projection in columns I .. 2I-1, and
+ *   h[i, j] = silu(g) * u = g * u / (1 + exp(-g)),  g = Y[i, j], u = Y[i, I + j],
+ * evaluated in fp64 and rounded once to bf16 (nearest even). */
+double orc_silu(double g) { return g / (1.0 + exp(-g)); }
+
+int orc_swiglu(const double* Y, int64_t M, int64_t I, uint16_t* h)
+{
+    int64_t i;
+    if (M < 0 || I <= 0) return 1;
+#pragma omp parallel for schedule(static)
+    for (i = 0; i < M; ++i) {
+        int64_t j;
+        for (j = 0; j < I; ++j) {
+            double g = Y[i * 2 * I + j], u = Y[i * 2 * I + I + j];
+            h[i * I + j] = orc_bf16_from_double(orc_silu(g) * u);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* NVFP4: 4-bit E2M1 elements, 16-element blocks with E4M3 scales and   */
 /* one fp32 scale per tensor                                             */
 /* ------------------------------------------------------------------ */
