@@ -781,11 +781,15 @@ def _cpu_quantiser(budget_s=2.0):
             "seconds_per_call": round(secs, 4)}
 
 
+CPU_BUILD = ("oracle/baseline_f32.c: bf16 inputs, fp32 accumulation, OpenMP over experts x 8-row blocks, "
+             "gcc -O3 -march=x86-64-v3 -ffp-contract=fast")
+
+
 def cpu_baseline(w, budget_s=12.0):
     import oracle
     flops, secs, desc = _cpu_sample(w, budget_s)
     return {"value": round(flops / secs / 1e12, 5), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-            "sample": desc, "seconds": round(secs, 2), "quantiser": _cpu_quantiser()}
+            "sample": desc, "seconds": round(secs, 2), "build": CPU_BUILD, "quantiser": _cpu_quantiser()}
 
 
 def run_reference(args):
@@ -807,7 +811,7 @@ def run_reference(args):
             "impl": "reference",
             "config": workload_config(w, args.quantiser, args.gpus),
             "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-                             "sample": desc + f"; {per_step:.2f} s per step"},
+                             "sample": desc + f"; {per_step:.2f} s per step", "build": CPU_BUILD},
             "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 

@@ -540,8 +540,6 @@ int orc_sample_wgrad(const uint8_t* dyqT, const uint8_t* dysT, const uint8_t* xq
 /* CPU baseline: bf16 inputs, fp32 accumulation, rows split over threads */
 /* ------------------------------------------------------------------ */
 
-static float bf16f(uint16_t b) { uint32_t u = (uint32_t)b << 16; float f; memcpy(&f, &u, 4); return f; }
-
 int orc_threads(void)
 {
 #ifdef _OPENMP
@@ -551,63 +549,8 @@ int orc_threads(void)
 #endif
 }
 
-/* Y = X_e W_e^T for rows [row_lo, row_hi) only (a bounded sample). */
-int orc_baseline_fwd_f32(const uint16_t* X, const uint16_t* W, const int32_t* offs, int32_t E,
-                         int64_t M, int64_t N, int64_t K, int64_t row_lo, int64_t row_hi, float* Y)
-{
-    int64_t i;
-    if (orc_check_offsets(offs, E, M)) return 1;
-#pragma omp parallel for schedule(dynamic, 4)
-    for (i = row_lo; i < row_hi; ++i) {
-        int32_t e = group_of_row(offs, E, i);
-        int64_t n, k;
-        for (n = 0; n < N; ++n) {
-            float acc = 0.0f;
-            for (k = 0; k < K; ++k) acc += bf16f(X[i * K + k]) * bf16f(W[((int64_t)e * N + n) * K + k]);
-            Y[i * N + n] = acc;
-        }
-    }
-    return 0;
-}
-
-/* dX = dY_e W_e for rows [row_lo, row_hi). */
-int orc_baseline_dgrad_f32(const uint16_t* dY, const uint16_t* W, const int32_t* offs, int32_t E,
-                           int64_t M, int64_t N, int64_t K, int64_t row_lo, int64_t row_hi, float* dX)
-{
-    int64_t i;
-    if (orc_check_offsets(offs, E, M)) return 1;
-#pragma omp parallel for schedule(dynamic, 4)
-    for (i = row_lo; i < row_hi; ++i) {
-        int32_t e = group_of_row(offs, E, i);
-        int64_t n, k;
-        for (k = 0; k < K; ++k) dX[i * K + k] = 0.0f;
-        for (n = 0; n < N; ++n) {
-            float d = bf16f(dY[i * N + n]);
-            for (k = 0; k < K; ++k) dX[i * K + k] += d * bf16f(W[((int64_t)e * N + n) * K + k]);
-        }
-    }
-    return 0;
-}
-
-/* dW_e = dY_e^T X_e for output rows n in [n_lo, n_hi) of every expert. */
-int orc_baseline_wgrad_f32(const uint16_t* dY, const uint16_t* X, const int32_t* offs, int32_t E,
-                           int64_t M, int64_t N, int64_t K, int64_t n_lo, int64_t n_hi, float* dW)
-{
-    int64_t en;
-    if (orc_check_offsets(offs, E, M)) return 1;
-#pragma omp parallel for schedule(dynamic, 1)
-    for (en = 0; en < (int64_t)E * (n_hi - n_lo); ++en) {
-        int32_t e = (int32_t)(en / (n_hi - n_lo));
-        int64_t n = n_lo + en % (n_hi - n_lo), i, k;
-        float* out = dW + ((int64_t)e * N + n) * K;
-        for (k = 0; k < K; ++k) out[k] = 0.0f;
-        for (i = offs[e]; i < offs[e + 1]; ++i) {
-            float d = bf16f(dY[i * N + n]);
-            for (k = 0; k < K; ++k) out[k] += d * bf16f(X[i * K + k]);
-        }
-    }
-    return 0;
-}
+/* The timed fp32 baselines (orc_baseline_fwd/dgrad/wgrad_f32) live in
+ * baseline_f32.c, built with optimisation flags of their own. */
 
 /* Whole-tensor quantiser timing helper for the CPU baseline: rowwise over
  * rows [row_lo, row_hi) of a single-group tensor (codes and logical scales). */
