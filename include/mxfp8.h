@@ -223,6 +223,28 @@ MXF8_API mxf8_status mxfp8_grouped_gemm_dgrad_quant(const uint8_t* dyq, const ui
                                                     uint8_t* scalesT, int64_t scaleT_bytes, void* work,
                                                     int64_t work_bytes, void* stream);
 
+/* Forward gate/up grouped GEMM fused with SwiGLU and MXFP8 quantisation of
+ * its result, for the down projection that follows.  The pages credit the
+ * MXFP8 speed-up to the expert pipeline as a whole (opensourcebeat.com,
+ * section "Двухсторонняя атака: MXFP8 и DeepEP"), and the DeepSeek-V3 and
+ * Llama 4 experts apply SwiGLU between their two linears; the pages give no
+ * formula, so the plainest reading is used:
+ *   Y_e = X_e W_e^T        (W_e: [N, K], N = 2I; Y accumulated in fp32, never written)
+ *   h[i, j] = silu(Y[i, j]) * Y[i, I + j],  silu(g) = g / (1 + exp(-g)),
+ * evaluated in fp32 from the accumulator and rounded once to bf16 (nearest
+ * even).  h is [M, I]; it is written as bf16 (`h`, nullable) and/or as
+ * MXFP8 exactly as mxfp8_quantize_rowwise / _colwise(h, d_offs) would encode
+ * that bf16 h (q/scales and qT/ldT/scalesT, each pair nullable; at least one
+ * of the three outputs).  N % 256 == 0 (I % 128 == 0), otherwise
+ * MXF8_ERR_INVALID_ARG; every other argument and error is that of
+ * mxfp8_grouped_gemm_fwd_quant with C = I. */
+MXF8_API mxf8_status mxfp8_grouped_gemm_fwd_swiglu(const uint8_t* xq, const uint8_t* xs, int64_t xs_bytes,
+                                                   const uint8_t* wq, const uint8_t* ws, int64_t ws_bytes,
+                                                   const int32_t* d_offs, int32_t E, int64_t M, int64_t N, int64_t K,
+                                                   uint16_t* h, uint8_t* q, uint8_t* scales, int64_t scale_bytes,
+                                                   uint8_t* qT, int64_t ldT, uint8_t* scalesT, int64_t scaleT_bytes,
+                                                   void* work, int64_t work_bytes, void* stream);
+
 /* Forward grouped GEMM that allocates nothing and takes no workspace.
  * The paper has no counterpart to this entry point; it exists for callers
  * that cannot call cudaMalloc (for example a plugin inside an engine that owns
@@ -256,14 +278,16 @@ MXF8_API mxf8_status mxfp8_grouped_gemm_fwd_noalloc(const uint8_t* xq, const uin
 /* Overrides, for the calling process, the tile configuration the grouped
  * GEMMs (MXFP8) choose per pass.  The pages fix no tiling; these are this
  * library's own pipeline shapes.
- *   cta_pair  -1 = the library's rule, 0 = 1-CTA 128x256 tiles,
- *             1 = CTA-pair 256x256 tiles (cta_group::2)
- *   stage_k   -1 = the library's rule, 1 = 128-deep K stages, 2 = 256-deep
+ *   cta_pair     -1 = the library's rule, 0 = 1-CTA 128x256 tiles,
+ *                1 = CTA-pair 256x256 tiles (cta_group::2)
+ *   stage_k      -1 = the library's rule, 1 = 128-deep K stages, 2 = 256-deep
+ *   l2_prefetch  -1 = the library's rule, 0 = none, 1..64 = K blocks the
+ *                producer prefetches into L2 ahead of its loads
  * Results are the same under every setting (same products, same fp32
  * accumulation order within a 32-element step); only speed changes.  Returns
  * MXF8_ERR_INVALID_ARG for any other value.  Not thread-safe against
  * concurrent GEMM calls. */
-MXF8_API mxf8_status mxfp8_set_gemm_tiling(int32_t cta_pair, int32_t stage_k);
+MXF8_API mxf8_status mxfp8_set_gemm_tiling(int32_t cta_pair, int32_t stage_k, int32_t l2_prefetch);
 
 /* Test switch for the bounded pipeline waits: while enabled (enable != 0),
  * every grouped GEMM launch leaves its first pipeline stage unfilled, so the

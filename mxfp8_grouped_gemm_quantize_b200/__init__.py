@@ -41,7 +41,7 @@ EXPORTED = ("mxfp8_rowwise_scale_bytes", "mxfp8_colwise_pitch", "mxfp8_colwise_s
             "mxfp8_nvfp4_colwise_pitch", "mxfp8_nvfp4_colwise_scale_bytes", "mxfp8_nvfp4_colwise_ld",
             "mxfp8_nvfp4_amax", "mxfp8_nvfp4_quantize_rowwise", "mxfp8_nvfp4_quantize_colwise",
             "mxfp8_nvfp4_grouped_gemm_fwd", "mxfp8_nvfp4_grouped_gemm_dgrad", "mxfp8_nvfp4_grouped_gemm_wgrad",
-            "mxfp8_set_gemm_tiling", "mxfp8_testing_stall_first_stage")
+            "mxfp8_set_gemm_tiling", "mxfp8_testing_stall_first_stage", "mxfp8_grouped_gemm_fwd_swiglu")
 
 
 class MXFP8Error(RuntimeError):
@@ -79,7 +79,7 @@ def lib() -> ctypes.CDLL:
         for n in ("mxfp8_grouped_gemm_fwd", "mxfp8_grouped_gemm_dgrad", "mxfp8_grouped_gemm_wgrad"):
             getattr(L, n).restype = _i32
             getattr(L, n).argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp, _vp, _i64, _vp]
-        for n in ("mxfp8_grouped_gemm_fwd_quant", "mxfp8_grouped_gemm_dgrad_quant"):
+        for n in ("mxfp8_grouped_gemm_fwd_quant", "mxfp8_grouped_gemm_dgrad_quant", "mxfp8_grouped_gemm_fwd_swiglu"):
             getattr(L, n).restype = _i32
             getattr(L, n).argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i64,
                                       _vp, _i64, _vp, _i64, _vp, _i64, _vp]
@@ -118,7 +118,7 @@ def lib() -> ctypes.CDLL:
         L.mxfp8_last_cuda_error.restype = ctypes.c_char_p
         L.mxfp8_device_supported.restype = _i32
         L.mxfp8_set_gemm_tiling.restype = _i32
-        L.mxfp8_set_gemm_tiling.argtypes = [_i32, _i32]
+        L.mxfp8_set_gemm_tiling.argtypes = [_i32, _i32, _i32]
         L.mxfp8_testing_stall_first_stage.restype = None
         L.mxfp8_testing_stall_first_stage.argtypes = [_i32]
         _LIB = L
@@ -296,6 +296,19 @@ def mxfp8_grouped_gemm_dgrad_quant(dyq, dys, wqT, wsT, offs, K: int, out=True, r
                        colwise, work, stream)
 
 
+def mxfp8_grouped_gemm_fwd_swiglu(xq, xs, wq, ws, offs, N: int, out=True, rowwise=True, colwise=True, work=None,
+                                  stream=None):
+    """Gate/up forward GEMM fused with SwiGLU: h = silu(Y[:, :N/2]) * Y[:, N/2:]
+    for Y = X_e W_e^T, written as bf16 [M, N/2] and/or MXFP8 (the bytes
+    mxfp8_quantize_rowwise / _colwise(h, offs) give).  Arguments as
+    mxfp8_grouped_gemm_fwd_quant.  Returns (h, q, scales, qT, scalesT)."""
+    M, K = xq.shape
+    if out is True:
+        out = torch.empty((M, N // 2), dtype=torch.bfloat16, device=xq.device)
+    return _gemm_quant("mxfp8_grouped_gemm_fwd_swiglu", xq, xs, wq, ws, offs, M, N, K, N // 2,
+                       out if isinstance(out, torch.Tensor) else None, rowwise, colwise, work, stream)
+
+
 def mxfp8_grouped_gemm_fwd_noalloc(xq, xs, wq, ws, offs, N: int, out=None, stream=None, want_status=False):
     """Forward grouped GEMM with the library's static scratch instead of a
     workspace, for callers that cannot allocate device memory.  With
@@ -321,11 +334,12 @@ def mxfp8_device_supported() -> bool:
     return bool(lib().mxfp8_device_supported())
 
 
-def mxfp8_set_gemm_tiling(cta_pair: int = -1, stage_k: int = -1) -> None:
+def mxfp8_set_gemm_tiling(cta_pair: int = -1, stage_k: int = -1, l2_prefetch: int = -1) -> None:
     """Process-wide override of the grouped GEMMs' tile configuration
     (-1 = the library's rule; cta_pair 0/1 = 1-CTA / CTA-pair tiles; stage_k
-    1/2 = 128- / 256-deep K stages).  Results do not change, only speed."""
-    _check(lib().mxfp8_set_gemm_tiling(int(cta_pair), int(stage_k)), "mxfp8_set_gemm_tiling")
+    1/2 = 128- / 256-deep K stages; l2_prefetch = K blocks prefetched into L2
+    ahead of the loads, 0 = none).  Results do not change, only speed."""
+    _check(lib().mxfp8_set_gemm_tiling(int(cta_pair), int(stage_k), int(l2_prefetch)), "mxfp8_set_gemm_tiling")
 
 
 def mxfp8_testing_stall_first_stage(enable: bool) -> None:

@@ -28,6 +28,7 @@ int64_t blocks128_bound(int64_t rows, int32_t G) { return rows <= 0 ? 0 : cdiv(r
 std::atomic<int> g_stall_first_stage{0};
 std::atomic<int> g_tiling_cta_pair{-1};
 std::atomic<int> g_tiling_stage_k{-1};
+std::atomic<int> g_tiling_l2_prefetch{-1};
 
 mxf8_status cuda_fail(cudaError_t e, const char* where, const char* detail = nullptr) {
   mxf8::record_cuda_error(e, where, detail);
@@ -128,19 +129,22 @@ void record_cuda_error(cudaError_t e, const char* where, const char* detail) {
                 detail ? " -- " : "", detail ? detail : "");
 }
 
-void gemm_tiling_override(int* cta_pair, int* stage_k) {
+void gemm_tiling_override(int* cta_pair, int* stage_k, int* l2_prefetch) {
   *cta_pair = g_tiling_cta_pair.load(std::memory_order_relaxed);
   *stage_k = g_tiling_stage_k.load(std::memory_order_relaxed);
+  *l2_prefetch = g_tiling_l2_prefetch.load(std::memory_order_relaxed);
 }
 
 }  // namespace mxf8
 
 extern "C" {
 
-mxf8_status mxfp8_set_gemm_tiling(int32_t cta_pair, int32_t stage_k) {
+mxf8_status mxfp8_set_gemm_tiling(int32_t cta_pair, int32_t stage_k, int32_t l2_prefetch) {
   if (cta_pair < -1 || cta_pair > 1 || stage_k < -1 || stage_k == 0 || stage_k > 2) return MXF8_ERR_INVALID_ARG;
+  if (l2_prefetch < -1 || l2_prefetch > 64) return MXF8_ERR_INVALID_ARG;
   g_tiling_cta_pair.store(cta_pair, std::memory_order_relaxed);
   g_tiling_stage_k.store(stage_k, std::memory_order_relaxed);
+  g_tiling_l2_prefetch.store(l2_prefetch, std::memory_order_relaxed);
   return MXF8_OK;
 }
 
@@ -311,6 +315,33 @@ mxf8_status mxfp8_grouped_gemm_fwd_quant(const uint8_t* xq, const uint8_t* xs, i
   g.sfa = xs; g.sfa_pitch = cdiv(K, 128); g.sfa_atoms = xs_bytes / 512;
   g.sfb = ws; g.sfb_pitch = cdiv(K, 128); g.sfb_atoms = ws_bytes / 512;
   g.out = y;
+  return run_gemm(g, work, stream);
+}
+
+mxf8_status mxfp8_grouped_gemm_fwd_swiglu(const uint8_t* xq, const uint8_t* xs, int64_t xs_bytes, const uint8_t* wq,
+                                          const uint8_t* ws, int64_t ws_bytes, const int32_t* d_offs, int32_t E,
+                                          int64_t M, int64_t N, int64_t K, uint16_t* h, uint8_t* q, uint8_t* scales,
+                                          int64_t scale_bytes, uint8_t* qT, int64_t ldT, uint8_t* scalesT,
+                                          int64_t scaleT_bytes, void* work, int64_t work_bytes, void* stream) {
+  const void* any_out = h ? static_cast<const void*>(h) : (q ? static_cast<const void*>(q) : qT);
+  mxf8_status s = check_gemm_args({xq, xs, xs_bytes, wq, ws, ws_bytes, d_offs, E, M, N, K, any_out, work, work_bytes});
+  if (s != MXF8_OK) return s;
+  if (N % 256 != 0) return MXF8_ERR_INVALID_ARG;   // gate and up halves in whole 128-column tiles
+  if (xs_bytes < mxfp8_rowwise_scale_bytes(M, K, E) || ws_bytes < mxfp8_rowwise_scale_bytes(E * N, K, 1))
+    return MXF8_ERR_INVALID_ARG;
+  mxf8::GemmArgs g{};
+  g.mode = mxf8::kFwd; g.E = E; g.M = M; g.N = N; g.K = K; g.offs = d_offs;
+  g.swiglu = true;
+  if ((s = attach_quant_outputs(g, N / 2, h, q, scales, scale_bytes, qT, ldT, scalesT, scaleT_bytes)) != MXF8_OK)
+    return s;
+  if ((s = check_device()) != MXF8_OK) return s;
+  if (M == 0) return cudaMemsetAsync(work, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) == cudaSuccess
+                         ? MXF8_OK : cuda_fail(cudaGetLastError(), "cudaMemsetAsync(status)");
+  g.a = xq; g.lda = K; g.a_rows = M; g.a_cols = K;
+  g.b = wq; g.ldb = K; g.b_rows = E * N; g.b_cols = K;
+  g.sfa = xs; g.sfa_pitch = cdiv(K, 128); g.sfa_atoms = xs_bytes / 512;
+  g.sfb = ws; g.sfb_pitch = cdiv(K, 128); g.sfb_atoms = ws_bytes / 512;
+  g.out = h;
   return run_gemm(g, work, stream);
 }
 

@@ -121,6 +121,7 @@ struct Params {
   int32_t* status;
   uint64_t timeout_ns;
   int32_t inject_skip_stage;           // test hook: the producer leaves stage 0 unfilled (1-CTA only)
+  int32_t l2_prefetch;                 // K blocks the producer prefetches into L2 ahead of its loads (0: none)
   // Quantising epilogue (fwd/dgrad): MXFP8 copies of the bf16 output, in the
   // quantisers' layouts with the GEMM's groups.  Null pointers skip a layout.
   uint8_t* qr;                         // rowwise codes [M, out_ld]
@@ -160,6 +161,11 @@ struct Tile {
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 __device__ __forceinline__ int32_t cdiv32(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
 
+// SwiGLU of one gate/up pair from the fp32 accumulators: silu(g) * u with
+// silu(g) = g / (1 + exp(-g)) (g -> -inf gives -0: the division by an
+// infinite denominator returns zero).
+__device__ __forceinline__ float swiglu_f32(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
 template <int CG>
 __device__ __forceinline__ int32_t group_m_units(const Params& p, int32_t m) {
   return cdiv32(p.mode == kWgrad ? cdiv32(p.N, BM) : cdiv32(m, BM), CG);
@@ -178,7 +184,10 @@ __device__ __forceinline__ int32_t advance_group(const Sched& s, int32_t E, int3
 }
 
 // Tile t (a pair tile when CG = 2) of group e as seen by CTA `rank` of its pair.
-template <int CG, bool FP4 = false>
+// SG (SwiGLU, fwd only): output tile nt covers columns 128nt..128nt+127 of
+// h [M, N/2]; its B rows are gate rows e*N + 128nt.. and up rows
+// e*N + N/2 + 128nt.. (CTA pairs: rank 0 stages the gate rows, rank 1 the up rows).
+template <int CG, bool FP4 = false, bool SG = false>
 __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int32_t t, int32_t e, uint32_t rank) {
   // K blocks are 128 bytes of codes: 128 E4M3 or 256 E2M1 elements; MMA steps
   // take 32 (E4M3) or 64 (E2M1) elements.  TMA x coordinates count bytes.
@@ -194,21 +203,31 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int
   const int64_t L = p.mode == kFwd ? p.K : (p.mode == kDgrad ? p.N : m);
   tl.kblocks = static_cast<int32_t>((L + KE - 1) / KE);
   tl.ksteps_last = tl.kblocks > 0 ? static_cast<int32_t>((L - int64_t(KE) * (tl.kblocks - 1) + KSTEP - 1) / KSTEP) : 0;
-  int64_t sfa_row, sfa_col, sfb_row, sfb_col, out_cols;
+  int64_t sfa_row, sfa_col, sfb_row, sfb_row1, sfb_col, out_cols;
   if (p.mode == kFwd) {
     tl.a_x = 0;                              tl.a_y = row0 + BM * mt;
-    tl.b_x = 0;                              tl.b_y = static_cast<int32_t>(e * p.N) + BN * nt + b_half;
+    tl.b_x = 0;
+    if constexpr (SG) {
+      const int64_t I = p.N / 2;
+      tl.b_y = static_cast<int32_t>(e * p.N + 128 * nt + (CG == 2 ? int64_t(rank) * I : 0));
+      sfb_row = e * (p.N / 128) + nt;        sfb_row1 = sfb_row + I / 128;
+      out_cols = I;
+    } else {
+      tl.b_y = static_cast<int32_t>(e * p.N) + BN * nt + b_half;
+      sfb_row = e * (p.N / 128) + 2 * nt;    sfb_row1 = sfb_row + 1;
+      out_cols = p.N;
+    }
     sfa_row = s.rb[e] + mt;                  sfa_col = 0;
-    sfb_row = e * (p.N / 128) + 2 * nt;      sfb_col = 0;
+    sfb_col = 0;
     tl.q_rb = s.rb[e] + mt;                  tl.q_p = s.p[e] + BM * mt;
     tl.out_row = int64_t(row0) + BM * mt;
     tl.rows = static_cast<int32_t>(min64(BM, m - BM * mt));
-    out_cols = p.N;
   } else if (p.mode == kDgrad) {
     tl.a_x = 0;                              tl.a_y = row0 + BM * mt;
     tl.b_x = static_cast<int32_t>(e * p.N / EB); tl.b_y = BN * nt + b_half;
     sfa_row = s.rb[e] + mt;                  sfa_col = 0;
     sfb_row = 2 * nt;                        sfb_col = e * (p.N / RPA);
+    sfb_row1 = sfb_row + 1;
     tl.q_rb = s.rb[e] + mt;                  tl.q_p = s.p[e] + BM * mt;
     tl.out_row = int64_t(row0) + BM * mt;
     tl.rows = static_cast<int32_t>(min64(BM, m - BM * mt));
@@ -218,17 +237,19 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int
     tl.b_x = s.p[e] / EB;                    tl.b_y = BN * nt + b_half;
     sfa_row = mt;                            sfa_col = FP4 ? s.q[e] : s.rb[e];
     sfb_row = 2 * nt;                        sfb_col = FP4 ? s.q[e] : s.rb[e];
+    sfb_row1 = sfb_row + 1;
     tl.q_rb = 0;                             tl.q_p = 0;
     tl.out_row = int64_t(e) * p.N + BM * mt;
     tl.rows = static_cast<int32_t>(min64(BM, p.N - int64_t(BM) * mt));
     out_cols = p.K;
   }
   if (tl.rows < 0) tl.rows = 0;
-  tl.out_col = int64_t(BN) * nt;
-  tl.cols = static_cast<int32_t>(min64(BN, out_cols - tl.out_col));
+  constexpr int OUT_W = SG ? BN / 2 : BN;   // output columns per tile
+  tl.out_col = int64_t(OUT_W) * nt;
+  tl.cols = static_cast<int32_t>(min64(OUT_W, out_cols - tl.out_col));
   tl.sfa_atom = sfa_row * p.sfa_pitch + sfa_col;
   tl.sfb_atom0 = sfb_row * p.sfb_pitch + sfb_col;
-  tl.sfb_atom1 = (sfb_row + 1) * p.sfb_pitch + sfb_col;
+  tl.sfb_atom1 = sfb_row1 * p.sfb_pitch + sfb_col;
   return tl;
 }
 
@@ -298,7 +319,7 @@ __device__ __forceinline__ void tmem_wait_regs(uint32_t (&r)[32]) {
                : "memory");
 }
 
-template <int CG, int KS, bool QE, bool FP4>
+template <int CG, int KS, bool QE, bool FP4, bool SG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
@@ -375,7 +396,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const bool skip0 = CG == 1 && p.inject_skip_stage != 0;
       for (int32_t t = unit0; t < total && !failed; t += nunits) {
         eh = advance_group(sc, p.E, t, eh);
-        const Tile tl = decode_tile<CG, FP4>(p, sc, t, eh, rank);
+        const Tile tl = decode_tile<CG, FP4, SG>(p, sc, t, eh, rank);
+        Tile tl_next;                 // decoded on demand for the L2 prefetch
+        bool next_ok = false, has_next = false;
         for (int32_t kb0 = 0; kb0 < tl.kblocks; kb0 += C::KS) {
           if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, lim)) {
             record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
@@ -411,9 +434,36 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if constexpr (CG == 2) {
               tma_load_2d_pair(sa, &tmA, tl.a_x + kx, tl.a_y, fb);
               tma_load_2d_pair(sb, &tmB, tl.b_x + kx, tl.b_y, fb);
+            } else if constexpr (SG) {
+              // gate rows, then the up rows N/2 further (two 128-row boxes)
+              tma_load_2d(sa, &tmA, tl.a_x + kx, tl.a_y, fb);
+              tma_load_2d(sb, &tmB, tl.b_x + kx, tl.b_y, fb);
+              tma_load_2d(sb + 128 * BK, &tmB, tl.b_x + kx, tl.b_y + static_cast<int32_t>(p.N / 2), fb);
             } else {
               tma_load_2d(sa, &tmA, tl.a_x + kx, tl.a_y, fb);
               tma_load_2d(sb, &tmB, tl.b_x + kx, tl.b_y, fb);
+            }
+          }
+          if (p.l2_prefetch > 0) {
+            // L2 prefetch of the A and B boxes l2_prefetch K blocks ahead, in
+            // this tile or (near its end) in this CTA's next tile
+            for (int32_t h = 0; h < nh; ++h) {
+              int32_t kp = kb0 + h + p.l2_prefetch;
+              const Tile* tp = &tl;
+              if (kp >= tl.kblocks) {
+                if (!next_ok) {
+                  next_ok = true;
+                  has_next = t + nunits < total;
+                  if (has_next) tl_next = decode_tile<CG, FP4, SG>(p, sc, t + nunits, advance_group(sc, p.E, t + nunits, eh), rank);
+                }
+                kp -= tl.kblocks;
+                tp = &tl_next;
+                if (!has_next || kp >= tl_next.kblocks) continue;
+              }
+              const int32_t kx = BK * kp;
+              tma_prefetch_l2_2d(&tmA, tp->a_x + kx, tp->a_y);
+              tma_prefetch_l2_2d(&tmB, tp->b_x + kx, tp->b_y);
+              if constexpr (SG && CG == 1) tma_prefetch_l2_2d(&tmB, tp->b_x + kx, tp->b_y + static_cast<int32_t>(p.N / 2));
             }
           }
           if constexpr (CG == 2) {
@@ -586,7 +636,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     for (int32_t t = unit0; t < total; t += nunits) {
       eh = advance_group(sc, p.E, t, eh);
-      const Tile tl = decode_tile<CG, FP4>(p, sc, t, eh, rank);
+      const Tile tl = decode_tile<CG, FP4, SG>(p, sc, t, eh, rank);
       const int32_t vr = max(0, min(32, tl.rows - row_base));       // valid rows of this warp's slice
       uint16_t* out_tile = p.out + tl.out_row * p.out_ld + tl.out_col;
       if (tl.kblocks == 0) {
@@ -606,9 +656,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       tc_fence_after();
       const uint32_t buf = j & 1;
       const uint32_t tbase = tmem + ((32 * quarter) << 16) + buf * C::ACC_STRIDE;
-      // Accumulator 0's last OV chunks are accumulator 1's first OV chunks:
-      // drain those first, then release the accumulator to the MMA issuer.
-      auto chunk_of = [&](int ci) { return buf == 0 ? (ci + 4 - C::OV) & 3 : ci; };
       // Every lane's tcgen05.ld has completed (wait::ld) before the warp
       // syncs; one lane then arrives for the warp.
       auto release = [&]() {
@@ -622,38 +669,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           }
         }
       };
-      uint32_t ra0[32], ra1[32], rb0[32], rb1[32];
-      tmem_ld_32x32b_x32(tbase + 64 * chunk_of(0), ra0);
-      tmem_ld_32x32b_x32(tbase + 64 * chunk_of(0) + 32, ra1);
-      tmem_wait_regs(ra0);
-      tmem_wait_regs(ra1);
-      if (C::OV == 1) release();
-#pragma unroll
-      for (int ci = 0; ci < 4; ++ci) {
-        uint32_t(&c0)[32] = (ci & 1) ? rb0 : ra0;
-        uint32_t(&c1)[32] = (ci & 1) ? rb1 : ra1;
-        uint32_t(&n0)[32] = (ci & 1) ? ra0 : rb0;
-        uint32_t(&n1)[32] = (ci & 1) ? ra1 : rb1;
-        if (ci < 3) {   // next chunk's tensor-memory load overlaps this chunk's conversion and store
-          tmem_ld_32x32b_x32(tbase + 64 * chunk_of(ci + 1), n0);
-          tmem_ld_32x32b_x32(tbase + 64 * chunk_of(ci + 1) + 32, n1);
-        }
-        const int c = chunk_of(ci);
+      // Writes output chunk c (64 columns from tl.out_col + 64c, this warp's
+      // 32 rows) from 64 packed bf16 values per lane: the bf16 output through
+      // a swizzled stage (TMA store for a full slice, masked stores for a
+      // group's ragged slice) and, in a quantising epilogue, its MXFP8 copies.
+      auto emit = [&](const uint32_t (&pk)[32], int c) {
         uint32_t rs = 0, cs0 = 0, cs1 = 0;   // quantising epilogue: scale bytes (0 = pad)
         if (vr > 0 && 64 * c < tl.cols) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            if constexpr (FP4) {
-              pk[i] = cvt_bf16x2(__fmul_rn(__uint_as_float(c0[2 * i]), oscale),
-                                 __fmul_rn(__uint_as_float(c0[2 * i + 1]), oscale));
-              pk[16 + i] = cvt_bf16x2(__fmul_rn(__uint_as_float(c1[2 * i]), oscale),
-                                      __fmul_rn(__uint_as_float(c1[2 * i + 1]), oscale));
-            } else {
-              pk[i] = cvt_bf16x2(__uint_as_float(c0[2 * i]), __uint_as_float(c0[2 * i + 1]));
-              pk[16 + i] = cvt_bf16x2(__uint_as_float(c1[2 * i]), __uint_as_float(c1[2 * i + 1]));
-            }
-          }
           uint8_t* stg = stage_base + (ec % C::EPI_BUFS) * EPI_STAGE;
           uint4* st4 = reinterpret_cast<uint4*>(stg);
           if (lane == 0) bulk_wait_read<C::EPI_BUFS - 1>();   // the buffer's previous store has read it
@@ -719,13 +741,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               const float f0 = inv_scale(cs0 == 0xFFu ? 0u : cs0), f1 = inv_scale(cs1 == 0xFFu ? 0u : cs1);
               uint32_t o0[8], o1[8];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const uint32_t a0 = cvt_e4m3x2(__fmul_rn(bf_lo(w[4 * j]), f0), __fmul_rn(bf_lo(w[4 * j + 1]), f0));
-                const uint32_t a1 = cvt_e4m3x2(__fmul_rn(bf_lo(w[4 * j + 2]), f0), __fmul_rn(bf_lo(w[4 * j + 3]), f0));
-                const uint32_t b0 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * j]), f1), __fmul_rn(bf_hi(w[4 * j + 1]), f1));
-                const uint32_t b1 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * j + 2]), f1), __fmul_rn(bf_hi(w[4 * j + 3]), f1));
-                o0[j] = cs0 == 0xFFu ? nan_codes4(j, vr) : (a0 | (a1 << 16));
-                o1[j] = cs1 == 0xFFu ? nan_codes4(j, vr) : (b0 | (b1 << 16));
+              for (int jj = 0; jj < 8; ++jj) {
+                const uint32_t a0 = cvt_e4m3x2(__fmul_rn(bf_lo(w[4 * jj]), f0), __fmul_rn(bf_lo(w[4 * jj + 1]), f0));
+                const uint32_t a1 = cvt_e4m3x2(__fmul_rn(bf_lo(w[4 * jj + 2]), f0), __fmul_rn(bf_lo(w[4 * jj + 3]), f0));
+                const uint32_t b0 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * jj]), f1), __fmul_rn(bf_hi(w[4 * jj + 1]), f1));
+                const uint32_t b1 = cvt_e4m3x2(__fmul_rn(bf_hi(w[4 * jj + 2]), f1), __fmul_rn(bf_hi(w[4 * jj + 3]), f1));
+                o0[jj] = cs0 == 0xFFu ? nan_codes4(jj, vr) : (a0 | (a1 << 16));
+                o1[jj] = cs1 == 0xFFu ? nan_codes4(jj, vr) : (b0 | (b1 << 16));
               }
               uint8_t* qcol = p.qc + (tl.out_col + 64 * c + 2 * lane) * p.qc_ld + tl.q_p + row_base;
               reinterpret_cast<uint4*>(qcol)[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
@@ -753,10 +775,75 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
           }
         }
-        if (ci < 3) {
-          tmem_wait_regs(n0);
-          tmem_wait_regs(n1);
-          if (ci + 2 == C::OV) release();   // chunk ci + 1 (the last shared one) is now in registers
+      };
+      if constexpr (SG) {
+        // SwiGLU: accumulator columns 0-127 hold the gate, 128-255 the up
+        // projection of the same 128 output columns; output chunk cc pairs
+        // gate chunk cc with up chunk cc + 2.  The chunk shared with the other
+        // accumulator goes first, so the release comes as early as it can.
+        const int first = buf == 0 ? 1 : 0;
+#pragma unroll 1
+        for (int it = 0; it < 2; ++it) {
+          const int cc = it == 0 ? first : 1 - first;
+          uint32_t g0[32], g1[32], u0[32], u1[32];
+          tmem_ld_32x32b_x32(tbase + 64 * cc, g0);
+          tmem_ld_32x32b_x32(tbase + 64 * cc + 32, g1);
+          tmem_ld_32x32b_x32(tbase + 64 * (cc + 2), u0);
+          tmem_ld_32x32b_x32(tbase + 64 * (cc + 2) + 32, u1);
+          tmem_wait_regs(g0);
+          tmem_wait_regs(g1);
+          tmem_wait_regs(u0);
+          tmem_wait_regs(u1);
+          if ((C::OV == 1 && it == 0) || it == 1) release();
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            pk[i] = cvt_bf16x2(swiglu_f32(__uint_as_float(g0[2 * i]), __uint_as_float(u0[2 * i])),
+                               swiglu_f32(__uint_as_float(g0[2 * i + 1]), __uint_as_float(u0[2 * i + 1])));
+            pk[16 + i] = cvt_bf16x2(swiglu_f32(__uint_as_float(g1[2 * i]), __uint_as_float(u1[2 * i])),
+                                    swiglu_f32(__uint_as_float(g1[2 * i + 1]), __uint_as_float(u1[2 * i + 1])));
+          }
+          emit(pk, cc);
+        }
+      } else {
+        // Accumulator 0's last OV chunks are accumulator 1's first OV chunks:
+        // drain those first, then release the accumulator to the MMA issuer.
+        auto chunk_of = [&](int ci) { return buf == 0 ? (ci + 4 - C::OV) & 3 : ci; };
+        uint32_t ra0[32], ra1[32], rb0[32], rb1[32];
+        tmem_ld_32x32b_x32(tbase + 64 * chunk_of(0), ra0);
+        tmem_ld_32x32b_x32(tbase + 64 * chunk_of(0) + 32, ra1);
+        tmem_wait_regs(ra0);
+        tmem_wait_regs(ra1);
+        if (C::OV == 1) release();
+#pragma unroll
+        for (int ci = 0; ci < 4; ++ci) {
+          uint32_t(&c0)[32] = (ci & 1) ? rb0 : ra0;
+          uint32_t(&c1)[32] = (ci & 1) ? rb1 : ra1;
+          uint32_t(&n0)[32] = (ci & 1) ? ra0 : rb0;
+          uint32_t(&n1)[32] = (ci & 1) ? ra1 : rb1;
+          if (ci < 3) {   // next chunk's tensor-memory load overlaps this chunk's conversion and store
+            tmem_ld_32x32b_x32(tbase + 64 * chunk_of(ci + 1), n0);
+            tmem_ld_32x32b_x32(tbase + 64 * chunk_of(ci + 1) + 32, n1);
+          }
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if constexpr (FP4) {
+              pk[i] = cvt_bf16x2(__fmul_rn(__uint_as_float(c0[2 * i]), oscale),
+                                 __fmul_rn(__uint_as_float(c0[2 * i + 1]), oscale));
+              pk[16 + i] = cvt_bf16x2(__fmul_rn(__uint_as_float(c1[2 * i]), oscale),
+                                      __fmul_rn(__uint_as_float(c1[2 * i + 1]), oscale));
+            } else {
+              pk[i] = cvt_bf16x2(__uint_as_float(c0[2 * i]), __uint_as_float(c0[2 * i + 1]));
+              pk[16 + i] = cvt_bf16x2(__uint_as_float(c1[2 * i]), __uint_as_float(c1[2 * i + 1]));
+            }
+          }
+          emit(pk, chunk_of(ci));
+          if (ci < 3) {
+            tmem_wait_regs(n0);
+            tmem_wait_regs(n1);
+            if (ci + 2 == C::OV) release();   // chunk ci + 1 (the last shared one) is now in registers
+          }
         }
       }
       ++j;
@@ -777,28 +864,32 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 }
 
 // ---------------------------------------------------------------- host side
+// Per device: SM count and, per kernel variant, whether its attributes are
+// set and how many CTA pairs fit (cluster launches).
+constexpr int kVariants = 32;   // CG x KS x QE x FP4 x SG
 struct DeviceSetup {
-  bool done[2][2][2][2] = {};    // [CG - 1][KS - 1][QE][FP4]
+  bool done[kVariants] = {};
   int num_sms = 0;
-  int max_pairs[2][2][2] = {};   // [KS - 1][QE][FP4]
+  int max_pairs[kVariants] = {};
 };
 DeviceSetup g_setup[64];
 
-template <int CG, int KS, bool QE, bool FP4 = false>
+template <int CG, int KS, bool QE, bool FP4 = false, bool SG = false>
 cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_t stream) {
   using C = Cfg<CG, KS, FP4>;
+  constexpr int V = (CG - 1) * 16 + (KS - 1) * 8 + int(QE) * 4 + int(FP4) * 2 + int(SG);
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   DeviceSetup& ds = g_setup[dev];
-  auto kernel = grouped_gemm_kernel<CG, KS, QE, FP4>;
+  auto kernel = grouped_gemm_kernel<CG, KS, QE, FP4, SG>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  if (!ds.done[CG - 1][KS - 1][QE][FP4]) {
+  if (!ds.done[V]) {
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     err = cudaDeviceGetAttribute(&ds.num_sms, cudaDevAttrMultiProcessorCount, dev);
@@ -813,16 +904,16 @@ cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_
       int clusters = 0;
       err = cudaOccupancyMaxActiveClusters(&clusters, kernel, &q);
       if (err != cudaSuccess) return err;
-      ds.max_pairs[KS - 1][QE][FP4] = clusters > 0 ? clusters : 1;
+      ds.max_pairs[V] = clusters > 0 ? clusters : 1;
     }
-    ds.done[CG - 1][KS - 1][QE][FP4] = true;
+    ds.done[V] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
   if (CG == 2) {
-    cfg.gridDim = dim3(2 * ds.max_pairs[KS - 1][QE][FP4]);
+    cfg.gridDim = dim3(2 * ds.max_pairs[V]);
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   } else {
@@ -840,9 +931,9 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   // ring) except for long K loops -- fwd/dgrad with at least 64 K blocks,
   // wgrad with at least 1024 rows per group on average -- where 256-deep
   // stages (2-stage ring) measured faster.  mxfp8_set_gemm_tiling overrides
-  // either choice.
-  int force_cg = -1, force_ks = -1;
-  gemm_tiling_override(&force_cg, &force_ks);
+  // either choice and sets the L2 prefetch distance (default: none).
+  int force_cg = -1, force_ks = -1, force_pf = -1;
+  gemm_tiling_override(&force_cg, &force_ks, &force_pf);
   int cg = force_cg == 1 ? 2 : 1;
   int ks = 1;
   if (a.mode == kWgrad) {
@@ -855,12 +946,15 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   if (a.fp4) { cg = 1; ks = 1; }   // NVFP4: one configuration (1-CTA, 3 x 128-byte stages)
   const uint32_t sf_box_rows = 4 * ks * (a.fp4 ? 4 : 1);
   const int64_t out_rows = a.mode == kWgrad ? int64_t(a.E) * a.N : a.M;
-  const int64_t out_cols = a.mode == kFwd ? a.N : a.K;
+  const int64_t out_cols = a.mode == kFwd ? (a.swiglu ? a.N / 2 : a.N) : a.K;
+  // B boxes: 128 rows when a CTA stages half of a 256-row B tile (pairs) or
+  // the gate and up halves separately (SwiGLU), else the whole tile.
+  const uint32_t b_box_rows = (cg == 2 || a.swiglu) ? BN / 2 : BN;
   CUtensorMap maps[5];
   const bool ok =
       make_tensor_map(&maps[0], a.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.a_rows, a.a_cols, a.lda, BK, BM,
                CU_TENSOR_MAP_SWIZZLE_128B) &&
-      make_tensor_map(&maps[1], a.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b_rows, a.b_cols, a.ldb, BK, BN / cg,
+      make_tensor_map(&maps[1], a.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.b_rows, a.b_cols, a.ldb, BK, b_box_rows,
                CU_TENSOR_MAP_SWIZZLE_128B) &&
       make_tensor_map(&maps[2], a.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.sfa_atoms * 4, 128, 128, 128, sf_box_rows,
                CU_TENSOR_MAP_SWIZZLE_NONE) &&
@@ -888,10 +982,16 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
   p.inject_skip_stage = a.inject_skip_stage;
+  p.l2_prefetch = force_pf > 0 ? force_pf : 0;
   p.qr = a.qr; p.sr = a.sr; p.qc = a.qc; p.sc = a.sc;
   p.qc_ld = a.qc_ld; p.sc_pitch = a.sc_pitch;
   p.amax_a = a.amax_a; p.amax_b = a.amax_b;
   if (a.fp4) return launch_cg<1, 1, false, true>(p, maps, stream);
+  if (a.swiglu) {
+    if (cg == 2) return ks == 2 ? launch_cg<2, 2, true, false, true>(p, maps, stream)
+                                : launch_cg<2, 1, true, false, true>(p, maps, stream);
+    return ks == 2 ? launch_cg<1, 2, true, false, true>(p, maps, stream) : launch_cg<1, 1, true, false, true>(p, maps, stream);
+  }
   const bool qe = a.qr != nullptr || a.qc != nullptr;
   if (qe) {
     if (cg == 2) return ks == 2 ? launch_cg<2, 2, true>(p, maps, stream) : launch_cg<2, 1, true>(p, maps, stream);
@@ -902,4 +1002,3 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
 }
 
 }  // namespace mxf8
-

@@ -81,6 +81,10 @@ struct GemmArgs {
   bool fp4 = false;
   const float* amax_a = nullptr;
   const float* amax_b = nullptr;
+  // fwd only: the epilogue applies SwiGLU to the gate/up output (gate =
+  // columns 0..N/2-1, up = N/2..N-1) and writes h [M, N/2] (bf16 `out`
+  // and/or the MXFP8 copies above); requires N % 256 == 0.
+  bool swiglu = false;
 };
 
 // Returns cudaSuccess or the CUDA error; *detail gets a short reason for
@@ -88,7 +92,7 @@ struct GemmArgs {
 cudaError_t launch_grouped_gemm(const GemmArgs& args, cudaStream_t stream, const char** detail);
 
 // Process-wide tile overrides set through mxfp8_set_gemm_tiling (-1 = rule).
-void gemm_tiling_override(int* cta_pair, int* stage_k);
+void gemm_tiling_override(int* cta_pair, int* stage_k, int* l2_prefetch);
 
 // Records a CUDA failure for mxfp8_last_cuda_error (thread-local text).
 void record_cuda_error(cudaError_t e, const char* where, const char* detail);
