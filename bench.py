@@ -589,6 +589,44 @@ def quantising_epilogue(mx, L: Linear, iters=20):
             raise SystemExit(f"bench: device status {st} in the quantising-epilogue measurement")
         r["tflops"] = round(L.flops_per_pass() / (r["quantising_epilogue_ms"] * 1e-3) / 1e12, 1)
         res[mode] = r
+    if L.N % 256 == 0:
+        # gate/up forward fused with SwiGLU and MXFP8 of h [M, N/2] (both
+        # layouts, no bf16 h), against the unfused path's lower bound: the
+        # GEMM writing bf16 Y [M, N], then the dual quantiser on an h-sized
+        # tensor (the elementwise SwiGLU pass itself is not counted)
+        I = L.N // 2
+        h = torch.empty((M, I), dtype=torch.bfloat16, device=dev)
+        row = (torch.empty((M, I), dtype=torch.uint8, device=dev),
+               torch.empty(mx.mxfp8_rowwise_scale_bytes(M, I, E), dtype=torch.uint8, device=dev))
+        col = (torch.empty((I, ld), dtype=torch.uint8, device=dev),
+               torch.empty(mx.mxfp8_colwise_scale_bytes(M, I, E), dtype=torch.uint8, device=dev))
+        variants = {
+            "gemm_then_dual_quantiser_ms": lambda: (
+                mx.mxfp8_grouped_gemm_fwd(L.xq, L.xs, L.wq, L.ws, L.offs, L.N, out=L.y, work=L.work),
+                mx.mxfp8_quantize_dual(h, L.offs, q=row[0], scales=row[1], qT=col[0], scalesT=col[1])),
+            "fused_swiglu_ms": lambda: mx.mxfp8_grouped_gemm_fwd_swiglu(L.xq, L.xs, L.wq, L.ws, L.offs, L.N, out=None,
+                                                                      rowwise=row, colwise=col, work=L.work),
+            "fused_swiglu_with_bf16_h_ms": lambda: mx.mxfp8_grouped_gemm_fwd_swiglu(
+                L.xq, L.xs, L.wq, L.ws, L.offs, L.N, out=h, rowwise=row, colwise=col, work=L.work),
+        }
+        r = {}
+        for name, fn in variants.items():
+            for _ in range(3):
+                fn()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record()
+            for _ in range(iters):
+                fn()
+            b.record()
+            torch.cuda.synchronize()
+            r[name] = round(a.elapsed_time(b) / iters, 4)
+        if mx.mxfp8_get_status(L.work) != 0:
+            raise SystemExit("bench: device status error in the SwiGLU measurement")
+        r["tflops"] = round(L.flops_per_pass() / (r["fused_swiglu_ms"] * 1e-3) / 1e12, 1)
+        r["unfused_note"] = "lower bound of the unfused path: GEMM to bf16 Y, then the dual quantiser on an [M, N/2] tensor"
+        res["swiglu_fwd"] = r
+        del h, row, col
     return res
 
 
