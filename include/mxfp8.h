@@ -278,16 +278,14 @@ MXF8_API mxf8_status mxfp8_grouped_gemm_fwd_noalloc(const uint8_t* xq, const uin
 /* Overrides, for the calling process, the tile configuration the grouped
  * GEMMs (MXFP8) choose per pass.  The pages fix no tiling; these are this
  * library's own pipeline shapes.
- *   cta_pair     -1 = the library's rule, 0 = 1-CTA 128x256 tiles,
- *                1 = CTA-pair 256x256 tiles (cta_group::2)
- *   stage_k      -1 = the library's rule, 1 = 128-deep K stages, 2 = 256-deep
- *   l2_prefetch  -1 = the library's rule, 0 = none, 1..64 = K blocks the
- *                producer prefetches into L2 ahead of its loads
+ *   cta_pair  -1 = the library's rule, 0 = 1-CTA 128x256 tiles,
+ *             1 = CTA-pair 256x256 tiles (cta_group::2)
+ *   stage_k   -1 = the library's rule, 1 = 128-deep K stages, 2 = 256-deep
  * Results are the same under every setting (same products, same fp32
  * accumulation order within a 32-element step); only speed changes.  Returns
  * MXF8_ERR_INVALID_ARG for any other value.  Not thread-safe against
  * concurrent GEMM calls. */
-MXF8_API mxf8_status mxfp8_set_gemm_tiling(int32_t cta_pair, int32_t stage_k, int32_t l2_prefetch);
+MXF8_API mxf8_status mxfp8_set_gemm_tiling(int32_t cta_pair, int32_t stage_k);
 
 /* Test switch for the bounded pipeline waits: while enabled (enable != 0),
  * every grouped GEMM launch leaves its first pipeline stage unfilled, so the

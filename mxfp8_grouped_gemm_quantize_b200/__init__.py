@@ -118,7 +118,7 @@ def lib() -> ctypes.CDLL:
         L.mxfp8_last_cuda_error.restype = ctypes.c_char_p
         L.mxfp8_device_supported.restype = _i32
         L.mxfp8_set_gemm_tiling.restype = _i32
-        L.mxfp8_set_gemm_tiling.argtypes = [_i32, _i32, _i32]
+        L.mxfp8_set_gemm_tiling.argtypes = [_i32, _i32]
         L.mxfp8_testing_stall_first_stage.restype = None
         L.mxfp8_testing_stall_first_stage.argtypes = [_i32]
         _LIB = L
@@ -334,12 +334,11 @@ def mxfp8_device_supported() -> bool:
     return bool(lib().mxfp8_device_supported())
 
 
-def mxfp8_set_gemm_tiling(cta_pair: int = -1, stage_k: int = -1, l2_prefetch: int = -1) -> None:
+def mxfp8_set_gemm_tiling(cta_pair: int = -1, stage_k: int = -1) -> None:
     """Process-wide override of the grouped GEMMs' tile configuration
     (-1 = the library's rule; cta_pair 0/1 = 1-CTA / CTA-pair tiles; stage_k
-    1/2 = 128- / 256-deep K stages; l2_prefetch = K blocks prefetched into L2
-    ahead of the loads, 0 = none).  Results do not change, only speed."""
-    _check(lib().mxfp8_set_gemm_tiling(int(cta_pair), int(stage_k), int(l2_prefetch)), "mxfp8_set_gemm_tiling")
+    1/2 = 128- / 256-deep K stages).  Results do not change, only speed."""
+    _check(lib().mxfp8_set_gemm_tiling(int(cta_pair), int(stage_k)), "mxfp8_set_gemm_tiling")
 
 
 def mxfp8_testing_stall_first_stage(enable: bool) -> None:

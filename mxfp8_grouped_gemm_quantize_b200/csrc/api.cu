@@ -28,7 +28,6 @@ int64_t blocks128_bound(int64_t rows, int32_t G) { return rows <= 0 ? 0 : cdiv(r
 std::atomic<int> g_stall_first_stage{0};
 std::atomic<int> g_tiling_cta_pair{-1};
 std::atomic<int> g_tiling_stage_k{-1};
-std::atomic<int> g_tiling_l2_prefetch{-1};
 
 mxf8_status cuda_fail(cudaError_t e, const char* where, const char* detail = nullptr) {
   mxf8::record_cuda_error(e, where, detail);
@@ -129,22 +128,19 @@ void record_cuda_error(cudaError_t e, const char* where, const char* detail) {
                 detail ? " -- " : "", detail ? detail : "");
 }
 
-void gemm_tiling_override(int* cta_pair, int* stage_k, int* l2_prefetch) {
+void gemm_tiling_override(int* cta_pair, int* stage_k) {
   *cta_pair = g_tiling_cta_pair.load(std::memory_order_relaxed);
   *stage_k = g_tiling_stage_k.load(std::memory_order_relaxed);
-  *l2_prefetch = g_tiling_l2_prefetch.load(std::memory_order_relaxed);
 }
 
 }  // namespace mxf8
 
 extern "C" {
 
-mxf8_status mxfp8_set_gemm_tiling(int32_t cta_pair, int32_t stage_k, int32_t l2_prefetch) {
+mxf8_status mxfp8_set_gemm_tiling(int32_t cta_pair, int32_t stage_k) {
   if (cta_pair < -1 || cta_pair > 1 || stage_k < -1 || stage_k == 0 || stage_k > 2) return MXF8_ERR_INVALID_ARG;
-  if (l2_prefetch < -1 || l2_prefetch > 64) return MXF8_ERR_INVALID_ARG;
   g_tiling_cta_pair.store(cta_pair, std::memory_order_relaxed);
   g_tiling_stage_k.store(stage_k, std::memory_order_relaxed);
-  g_tiling_l2_prefetch.store(l2_prefetch, std::memory_order_relaxed);
   return MXF8_OK;
 }
 

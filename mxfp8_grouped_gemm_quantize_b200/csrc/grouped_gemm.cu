@@ -54,7 +54,7 @@ constexpr int EPI_STAGE = 32 * 128;        // one epilogue buffer: 32 rows x 64 
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_STRIDE = 12;        // per stage: SFA 4 columns, then SFB 8 columns
 constexpr int MAXG = MXF8_GEMM_MAX_GROUPS;
-constexpr int SCHED_INTS = 5 * (MAXG + 1);
+constexpr int SCHED_INTS = 6 * (MAXG + 1);
 
 constexpr int round_up_c(int a, int b) { return (a + b - 1) / b * b; }
 
@@ -70,17 +70,22 @@ constexpr int round_up_c(int a, int b) { return (a + b - 1) / b * b; }
 template <int CG, int KS_, bool FP4 = false>
 struct Cfg {
   static constexpr int KS = KS_;
-  static constexpr int STAGES = FP4 ? 3 : (CG == 2 ? (KS == 2 ? 3 : 5) : (KS == 2 ? 2 : 4));
+  static constexpr int STAGES = FP4 ? 3 : (CG == 2 ? (KS == 2 ? 3 : 6) : (KS == 2 ? 2 : 4));
   static constexpr int APK = FP4 ? 4 : 1;              // scale atoms per K block and 128 rows
   static constexpr int SFA_T = SFA_TILE * APK, SFB_T = SFB_TILE * APK;
   static constexpr int SLOTS = STAGES * KS;            // 128-wide K-block slots in the ring
   static constexpr int B_ROWS = BN / CG;               // B rows staged by each CTA
   static constexpr int A_TILE = BM * BK;               // 16 KB of E4M3 codes
   static constexpr int B_TILE = B_ROWS * BK;
-  static constexpr int EPI_BUFS = (CG == 2 && KS == 1) ? 2 : 1;
+  static constexpr int EPI_BUFS = 1;
   // The two 128x256 accumulators overlap in OV 64-column chunks: accumulator 1
-  // starts at column ACC_STRIDE, and the scale sets of all slots follow it.
-  static constexpr int SF_SETS = FP4 ? 2 : SLOTS;      // scale sets in tensor memory
+  // starts at column ACC_STRIDE, and the scale sets follow it.  Scale sets
+  // either rotate with the ring's K-block slots or, where the ring is deep
+  // (NVFP4, pairs with 6 x 128-deep stages), alternate between two sets: the
+  // copies and MMAs of one thread execute in issue order, so the copy into a
+  // set follows the MMAs of the K block before last that read it.
+  static constexpr bool SF_ALT = FP4 || SLOTS > 4;
+  static constexpr int SF_SETS = SF_ALT ? 2 : SLOTS;   // scale sets in tensor memory
   static constexpr int SF_SET_COLS = SF_STRIDE * APK;  // columns of one set
   static constexpr int OV = (SF_SETS * SF_SET_COLS <= 64) ? 1 : 2;
   static constexpr uint32_t ACC_STRIDE = 256 - 64 * OV;
@@ -121,7 +126,6 @@ struct Params {
   int32_t* status;
   uint64_t timeout_ns;
   int32_t inject_skip_stage;           // test hook: the producer leaves stage 0 unfilled (1-CTA only)
-  int32_t l2_prefetch;                 // K blocks the producer prefetches into L2 ahead of its loads (0: none)
   // Quantising epilogue (fwd/dgrad): MXFP8 copies of the bf16 output, in the
   // quantisers' layouts with the GEMM's groups.  Null pointers skip a layout.
   uint8_t* qr;                         // rowwise codes [M, out_ld]
@@ -135,9 +139,13 @@ struct Params {
   const float* amax_b;
 };
 
-// Per-CTA schedule, built from the offsets by warp 0.
+// Per-CTA schedule, built from the offsets by warp 0.  Tiles are numbered
+// slot by slot; slot i holds the tiles of expert slot[i] (fwd/dgrad: slot i
+// is expert i; wgrad: experts by decreasing token count, so the long K loops
+// run first and the short ones fill the end of the schedule).
 struct Sched {
-  int32_t* tile0;   // [E+1] first tile of each group (prefix)
+  int32_t* tile0;   // [E+1] first tile of each slot (prefix)
+  int32_t* slot;    // [E]   expert of each slot
   int32_t* off;     // [E+1] row offsets
   int32_t* rb;      // [E]   RB_e: 128-row blocks before group e (rowwise scale rows,
                     //       colwise scale block-columns / 4)
@@ -175,28 +183,29 @@ __device__ __forceinline__ int32_t n_tiles(const Params& p) {
   return p.mode == kFwd ? cdiv32(p.N, BN) : cdiv32(p.K, BN);
 }
 
-// Group of tile t: the last group whose first tile is <= t.  A CTA visits
-// its tiles in increasing order, so the search advances from the previous
-// answer `e` (start at 0) instead of bisecting every time.
-__device__ __forceinline__ int32_t advance_group(const Sched& s, int32_t E, int32_t t, int32_t e) {
-  while (e + 1 < E && s.tile0[e + 1] <= t) ++e;
-  return e;
+// Slot of tile t: the last slot whose first tile is <= t.  A CTA visits its
+// tiles in increasing order, so the search advances from the previous answer
+// `i` (start at 0) instead of bisecting every time.
+__device__ __forceinline__ int32_t advance_group(const Sched& s, int32_t E, int32_t t, int32_t i) {
+  while (i + 1 < E && s.tile0[i + 1] <= t) ++i;
+  return i;
 }
 
-// Tile t (a pair tile when CG = 2) of group e as seen by CTA `rank` of its pair.
+// Tile t (a pair tile when CG = 2) of slot `si` as seen by CTA `rank` of its pair.
 // SG (SwiGLU, fwd only): output tile nt covers columns 128nt..128nt+127 of
 // h [M, N/2]; its B rows are gate rows e*N + 128nt.. and up rows
 // e*N + N/2 + 128nt.. (CTA pairs: rank 0 stages the gate rows, rank 1 the up rows).
 template <int CG, bool FP4 = false, bool SG = false>
-__device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int32_t t, int32_t e, uint32_t rank) {
+__device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int32_t t, int32_t si, uint32_t rank) {
   // K blocks are 128 bytes of codes: 128 E4M3 or 256 E2M1 elements; MMA steps
   // take 32 (E4M3) or 64 (E2M1) elements.  TMA x coordinates count bytes.
   constexpr int KE = FP4 ? 256 : 128, KSTEP = FP4 ? 64 : 32, EB = FP4 ? 2 : 1;   // EB: elements per byte
   constexpr int RPA = FP4 ? 64 : 128;   // colwise rows per scale atom column
   Tile tl;
+  const int32_t e = s.slot[si];
   const int32_t row0 = s.off[e], m = s.off[e + 1] - s.off[e];
   const int32_t munits = group_m_units<CG>(p, m);
-  const int32_t local = t - s.tile0[e];
+  const int32_t local = t - s.tile0[si];
   const int32_t mt = CG * (local % munits) + static_cast<int32_t>(rank);   // this CTA's 128-row block
   const int32_t nt = local / munits;
   const int32_t b_half = (CG == 2) ? BN / 2 * static_cast<int32_t>(rank) : 0;
@@ -303,6 +312,41 @@ __device__ int32_t build_schedule(const Params& p, const Sched& s) {
     if (lane == 0 && blockIdx.x == 0) atomicCAS(p.status, 0, static_cast<int32_t>(MXF8_ERR_BAD_OFFSETS));
     return 0;
   }
+  if (p.mode != kWgrad) {
+    for (int32_t h = lane; h < p.E; h += 32) s.slot[h] = h;
+    return carry_t;
+  }
+  // wgrad: slot order = decreasing rows (ties by expert index), then the
+  // tile prefix in slot order
+  __syncwarp();
+  for (int32_t h = lane; h < p.E; h += 32) {
+    const int32_t mh = s.off[h + 1] - s.off[h];
+    int32_t r = 0;
+    for (int32_t g = 0; g < p.E; ++g) {
+      const int32_t mg = s.off[g + 1] - s.off[g];
+      r += (mg > mh || (mg == mh && g < h)) ? 1 : 0;
+    }
+    s.slot[r] = h;
+  }
+  __syncwarp();
+  carry_t = 0;
+  for (int32_t base = 0; base < p.E; base += 32) {
+    const int32_t i = base + lane;
+    int32_t tiles = 0;
+    if (i < p.E) {
+      const int32_t e = s.slot[i];
+      tiles = group_m_units<CG>(p, s.off[e + 1] - s.off[e]) * ntl;
+    }
+    int32_t st = tiles;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int32_t x = __shfl_up_sync(0xffffffffu, st, d);
+      if (lane >= d) st += x;
+    }
+    if (i < p.E) s.tile0[i] = carry_t + st - tiles;
+    if (i == p.E - 1) s.tile0[p.E] = carry_t + st;
+    carry_t = __shfl_sync(0xffffffffu, carry_t + st, 31);
+  }
   return carry_t;
 }
 
@@ -349,6 +393,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   sc.rb = sched + 2 * (MAXG + 1);
   sc.p = sched + 3 * (MAXG + 1);
   sc.q = sched + 4 * (MAXG + 1);
+  sc.slot = sched + 5 * (MAXG + 1);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -397,8 +442,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       for (int32_t t = unit0; t < total && !failed; t += nunits) {
         eh = advance_group(sc, p.E, t, eh);
         const Tile tl = decode_tile<CG, FP4, SG>(p, sc, t, eh, rank);
-        Tile tl_next;                 // decoded on demand for the L2 prefetch
-        bool next_ok = false, has_next = false;
         for (int32_t kb0 = 0; kb0 < tl.kblocks; kb0 += C::KS) {
           if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, lim)) {
             record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
@@ -442,28 +485,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             } else {
               tma_load_2d(sa, &tmA, tl.a_x + kx, tl.a_y, fb);
               tma_load_2d(sb, &tmB, tl.b_x + kx, tl.b_y, fb);
-            }
-          }
-          if (p.l2_prefetch > 0) {
-            // L2 prefetch of the A and B boxes l2_prefetch K blocks ahead, in
-            // this tile or (near its end) in this CTA's next tile
-            for (int32_t h = 0; h < nh; ++h) {
-              int32_t kp = kb0 + h + p.l2_prefetch;
-              const Tile* tp = &tl;
-              if (kp >= tl.kblocks) {
-                if (!next_ok) {
-                  next_ok = true;
-                  has_next = t + nunits < total;
-                  if (has_next) tl_next = decode_tile<CG, FP4, SG>(p, sc, t + nunits, advance_group(sc, p.E, t + nunits, eh), rank);
-                }
-                kp -= tl.kblocks;
-                tp = &tl_next;
-                if (!has_next || kp >= tl_next.kblocks) continue;
-              }
-              const int32_t kx = BK * kp;
-              tma_prefetch_l2_2d(&tmA, tp->a_x + kx, tp->a_y);
-              tma_prefetch_l2_2d(&tmB, tp->b_x + kx, tp->b_y);
-              if constexpr (SG && CG == 1) tma_prefetch_l2_2d(&tmB, tp->b_x + kx, tp->b_y + static_cast<int32_t>(p.N / 2));
             }
           }
           if constexpr (CG == 2) {
@@ -523,7 +544,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         int32_t kblocks = kb_fixed, ksteps_last = ks_fixed;
         if (p.mode == kWgrad) {
           eh = advance_group(sc, p.E, t, eh);
-          const int32_t m = sc.off[eh + 1] - sc.off[eh];
+          const int32_t e = sc.slot[eh];
+          const int32_t m = sc.off[e + 1] - sc.off[e];
           kblocks = (m + KE - 1) / KE;
           if (kblocks == 0) continue;
           ksteps_last = (m - KE * (kblocks - 1) + KSTEP - 1) / KSTEP;
@@ -575,7 +597,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
                 ++kbc;
               } else {
-                const uint32_t sfa_t = sf_t0 + SF_STRIDE * q, sfb_t = sfa_t + 4;
+                const uint32_t sfa_t = sf_t0 + SF_STRIDE * (C::SF_ALT ? (kbc & 1) : q), sfb_t = sfa_t + 4;
+                ++kbc;
                 const uint64_t dsa = dsa0 + (SFA_TILE >> 4) * q;
                 const uint64_t dsb = dsb0 + (SFB_TILE >> 4) * C::KS * s + (512 >> 4) * h;
                 if constexpr (CG == 2) {
@@ -931,9 +954,9 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   // ring) except for long K loops -- fwd/dgrad with at least 64 K blocks,
   // wgrad with at least 1024 rows per group on average -- where 256-deep
   // stages (2-stage ring) measured faster.  mxfp8_set_gemm_tiling overrides
-  // either choice and sets the L2 prefetch distance (default: none).
-  int force_cg = -1, force_ks = -1, force_pf = -1;
-  gemm_tiling_override(&force_cg, &force_ks, &force_pf);
+  // either choice.
+  int force_cg = -1, force_ks = -1;
+  gemm_tiling_override(&force_cg, &force_ks);
   int cg = force_cg == 1 ? 2 : 1;
   int ks = 1;
   if (a.mode == kWgrad) {
@@ -982,7 +1005,6 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
   p.inject_skip_stage = a.inject_skip_stage;
-  p.l2_prefetch = force_pf > 0 ? force_pf : 0;
   p.qr = a.qr; p.sr = a.sr; p.qc = a.qc; p.sc = a.sc;
   p.qc_ld = a.qc_ld; p.sc_pitch = a.sc_pitch;
   p.amax_a = a.amax_a; p.amax_b = a.amax_b;

@@ -92,7 +92,7 @@ struct GemmArgs {
 cudaError_t launch_grouped_gemm(const GemmArgs& args, cudaStream_t stream, const char** detail);
 
 // Process-wide tile overrides set through mxfp8_set_gemm_tiling (-1 = rule).
-void gemm_tiling_override(int* cta_pair, int* stage_k, int* l2_prefetch);
+void gemm_tiling_override(int* cta_pair, int* stage_k);
 
 // Records a CUDA failure for mxfp8_last_cuda_error (thread-local text).
 void record_cuda_error(cudaError_t e, const char* where, const char* detail);
