@@ -38,6 +38,7 @@
 
 #include <cstdlib>
 #include <cstring>
+#include <type_traits>
 
 #include "codec.cuh"
 #include "launch.h"
@@ -558,73 +559,83 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
         tc_fence_after();
         uint32_t acc = 0;
-        for (int32_t kb0 = 0; kb0 < kblocks; kb0 += C::KS) {
+        // One K block of slot q (stage s, position h): its scale copies and
+        // MMAs.  FULL (compile time): all four MMA steps, no predicates --
+        // every K block but a tile's last; the tile's last takes nk steps.
+        auto issue_kb = [&](uint32_t q, uint32_t st, int h, int32_t nk, auto full_tag) {
+          constexpr bool FULL = decltype(full_tag)::value;
+          const uint64_t da = da0 + (C::A_TILE >> 4) * q, db = db0 + (C::B_TILE >> 4) * q;
+          if constexpr (FP4) {
+            // four MMAs of K = 64, each with its own atoms: SFA atom i of the
+            // stage's SFA box, SFB atoms i of its two SFB boxes
+            const uint32_t set0 = sf_t0 + C::SF_SET_COLS * (kbc & 1);
+            const uint64_t dsa = dsa0 + (C::SFA_T >> 4) * q;
+            const uint64_t dsb = dsb0 + (C::SFB_T >> 4) * C::KS * st + (C::APK * 512 >> 4) * h;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if (FULL || i < nk) {
+                const uint32_t sfa_t = set0 + SF_STRIDE * i, sfb_t = sfa_t + 4;
+                tc_cp_32x128b_x4(sfa_t, dsa + (512 >> 4) * i);
+                tc_cp_32x128b_x4(sfb_t, dsb + (512 >> 4) * i);
+                tc_cp_32x128b_x4(sfb_t + 4, dsb + (512 >> 4) * (C::KS * C::APK + i));
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if (FULL || i < nk) {
+                const uint32_t sfa_t = set0 + SF_STRIDE * i, sfb_t = sfa_t + 4;
+                tc_mma_nvf4(d_tmem, da + 2 * i, db + 2 * i, idesc0, sfa_t, sfb_t, acc);
+                acc = 1;
+              }
+            }
+            ++kbc;
+          } else {
+            const uint32_t sfa_t = sf_t0 + SF_STRIDE * (C::SF_ALT ? (kbc & 1) : q), sfb_t = sfa_t + 4;
+            ++kbc;
+            const uint64_t dsa = dsa0 + (SFA_TILE >> 4) * q;
+            const uint64_t dsb = dsb0 + (SFB_TILE >> 4) * C::KS * st + (512 >> 4) * h;
+            if constexpr (CG == 2) {
+              tc_cp_32x128b_x4_pair(sfa_t, dsa);
+              tc_cp_32x128b_x4_pair(sfb_t, dsb);
+              tc_cp_32x128b_x4_pair(sfb_t + 4, dsb + (512 >> 4) * C::KS);
+            } else {
+              tc_cp_32x128b_x4(sfa_t, dsa);
+              tc_cp_32x128b_x4(sfb_t, dsb);
+              tc_cp_32x128b_x4(sfb_t + 4, dsb + (512 >> 4) * C::KS);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              if (FULL || k < nk) {
+                // +2 per step: the start-address field counts 16-byte units, one step is 32 bytes of K
+                const uint32_t idesc = idesc0 | (uint32_t(k) << 4) | (uint32_t(k) << 29);
+                if constexpr (CG == 2)
+                  tc_mma_mxf8_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
+                                   sfb_t | (uint32_t(k) << 30), acc);
+                else
+                  tc_mma_mxf8(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
+                              sfb_t | (uint32_t(k) << 30), acc);
+                acc = 1;
+              }
+            }
+          }
+        };
+        // Stages before the tile's last hold only full-depth K blocks.
+        const int32_t last0 = ((kblocks - 1) / C::KS) * C::KS;   // first K block of the last stage
+        for (int32_t kb0 = 0; kb0 <= last0; kb0 += C::KS) {
           if (!mbar_wait(full_bar(s), ph, abort_flag, lim)) {
             record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
             failed = true;
             break;
           }
           tc_fence_after();
+          if (kb0 < last0) {
 #pragma unroll
-          for (int h = 0; h < C::KS; ++h) {
-            const int32_t kb = kb0 + h;
-            if (kb < kblocks) {
-              const uint32_t q = s * C::KS + h;
-              const uint64_t da = da0 + (C::A_TILE >> 4) * q, db = db0 + (C::B_TILE >> 4) * q;
-              const int32_t nk = (kb == kblocks - 1) ? ksteps_last : 4;
-              if constexpr (FP4) {
-                // four MMAs of K = 64, each with its own atoms: SFA atom i of the
-                // stage's SFA box, SFB atoms i of its two SFB boxes
-                const uint32_t set0 = sf_t0 + C::SF_SET_COLS * (kbc & 1);
-                const uint64_t dsa = dsa0 + (C::SFA_T >> 4) * q;
-                const uint64_t dsb = dsb0 + (C::SFB_T >> 4) * C::KS * s + (C::APK * 512 >> 4) * h;
+            for (int h = 0; h < C::KS; ++h) issue_kb(s * C::KS + h, s, h, 4, std::true_type{});
+          } else {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  if (i < nk) {
-                    const uint32_t sfa_t = set0 + SF_STRIDE * i, sfb_t = sfa_t + 4;
-                    tc_cp_32x128b_x4(sfa_t, dsa + (512 >> 4) * i);
-                    tc_cp_32x128b_x4(sfb_t, dsb + (512 >> 4) * i);
-                    tc_cp_32x128b_x4(sfb_t + 4, dsb + (512 >> 4) * (C::KS * C::APK + i));
-                  }
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  if (i < nk) {
-                    const uint32_t sfa_t = set0 + SF_STRIDE * i, sfb_t = sfa_t + 4;
-                    tc_mma_nvf4(d_tmem, da + 2 * i, db + 2 * i, idesc0, sfa_t, sfb_t, acc);
-                    acc = 1;
-                  }
-                }
-                ++kbc;
-              } else {
-                const uint32_t sfa_t = sf_t0 + SF_STRIDE * (C::SF_ALT ? (kbc & 1) : q), sfb_t = sfa_t + 4;
-                ++kbc;
-                const uint64_t dsa = dsa0 + (SFA_TILE >> 4) * q;
-                const uint64_t dsb = dsb0 + (SFB_TILE >> 4) * C::KS * s + (512 >> 4) * h;
-                if constexpr (CG == 2) {
-                  tc_cp_32x128b_x4_pair(sfa_t, dsa);
-                  tc_cp_32x128b_x4_pair(sfb_t, dsb);
-                  tc_cp_32x128b_x4_pair(sfb_t + 4, dsb + (512 >> 4) * C::KS);
-                } else {
-                  tc_cp_32x128b_x4(sfa_t, dsa);
-                  tc_cp_32x128b_x4(sfb_t, dsb);
-                  tc_cp_32x128b_x4(sfb_t + 4, dsb + (512 >> 4) * C::KS);
-                }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  if (k < nk) {
-                    // +2 per step: the start-address field counts 16-byte units, one step is 32 bytes of K
-                    const uint32_t idesc = idesc0 | (uint32_t(k) << 4) | (uint32_t(k) << 29);
-                    if constexpr (CG == 2)
-                      tc_mma_mxf8_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
-                                       sfb_t | (uint32_t(k) << 30), acc);
-                    else
-                      tc_mma_mxf8(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
-                                  sfb_t | (uint32_t(k) << 30), acc);
-                    acc = 1;
-                  }
-                }
-              }
+            for (int h = 0; h < C::KS; ++h) {
+              const int32_t kb = kb0 + h;
+              if (kb < kblocks) issue_kb(s * C::KS + h, s, h, kb == kblocks - 1 ? ksteps_last : 4, std::false_type{});
             }
           }
           if constexpr (CG == 2) tc_commit_pair(empty_bar(s), 0x3);
