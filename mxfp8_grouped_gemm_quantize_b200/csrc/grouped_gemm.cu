@@ -959,23 +959,21 @@ cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_
 }  // namespace
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** detail) {
-  // Tile configuration: 1-CTA 128x256 tiles by default -- on B200 they beat
-  // CTA pairs on the DeepSeek-V3-like layers (pairs also waste up to 128
-  // rows per group in fwd/dgrad).  Stage depth: 128-deep stages (4-stage
-  // ring) except for long K loops -- fwd/dgrad with at least 64 K blocks,
-  // wgrad with at least 1024 rows per group on average -- where 256-deep
-  // stages (2-stage ring) measured faster.  mxfp8_set_gemm_tiling overrides
-  // either choice.
+  // Tile configuration, from sizes the host knows (the group sizes stay on
+  // the device): fwd/dgrad over long contractions (>= 40 K blocks) of groups
+  // averaging >= 768 rows run CTA pairs with 256-deep stages -- pairs move
+  // 2/3 of the operand bytes per FLOP and their 256-row padding is then a
+  // small share; everything else runs 1-CTA 128x256 tiles with 128-deep
+  // stages (on B200 these won every other pass of the three MoE layers).
+  // mxfp8_set_gemm_tiling overrides either choice.
   int force_cg = -1, force_ks = -1;
   gemm_tiling_override(&force_cg, &force_ks);
-  int cg = force_cg == 1 ? 2 : 1;
-  int ks = 1;
-  if (a.mode == kWgrad) {
-    if (a.M >= int64_t(1024) * a.E) ks = 2;
-  } else {
+  int cg = 1, ks = 1;
+  if (a.mode != kWgrad) {
     const int64_t kblocks = ((a.mode == kFwd ? a.K : a.N) + BK - 1) / BK;
-    if (kblocks >= 64) ks = 2;
+    if (kblocks >= 40 && a.M >= int64_t(768) * a.E) { cg = 2; ks = 2; }
   }
+  if (force_cg == 0 || force_cg == 1) cg = force_cg == 1 ? 2 : 1;
   if (force_ks == 1 || force_ks == 2) ks = force_ks;
   if (a.fp4) { cg = 1; ks = 1; }   // NVFP4: one configuration (1-CTA, 3 x 128-byte stages)
   const uint32_t sf_box_rows = 4 * ks * (a.fp4 ? 4 : 1);
