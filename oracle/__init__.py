@@ -74,6 +74,12 @@ def lib():
         L.orc_bf16_from_double.restype = ctypes.c_uint16
         L.orc_bf16_from_double.argtypes = [ctypes.c_double]
         L.orc_bf16_from_double_array.argtypes = [_vp, _i64, _vp]
+        L.orc_ep_plan.restype = _i64
+        L.orc_ep_plan.argtypes = [_vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]
+        L.orc_ep_record_bytes.restype = _i64
+        L.orc_ep_record_bytes.argtypes = [_i64]
+        L.orc_ep_pack.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp]
+        L.orc_ep_unpack.argtypes = [_vp, _i64, _i64, _vp, _vp, _i32, _vp, _i64, _vp, _i32, _vp, _vp]
         L.orc_silu.restype = ctypes.c_double
         L.orc_silu.argtypes = [ctypes.c_double]
         L.orc_swiglu.argtypes = [_vp, _i64, _i64, _vp]
@@ -492,6 +498,85 @@ def moe_combine(yp, inv, w) -> np.ndarray:
     y = np.zeros((T, C), dtype=np.uint16)
     _check(lib().orc_moe_combine(_p(ypu), rows, C, _p(inv), _p(w), T, k, _p(y)), "moe_combine")
     return y
+
+
+# ---------------------------------------------------------------- expert-parallel dispatch
+class EpPlan:
+    """The send side of one dispatch (see orc_ep_plan)."""
+
+    def __init__(self, counts, rec_token, pair_expert, pair_rec, ret_pos, bad):
+        self.counts, self.rec_token, self.pair_expert, self.pair_rec = counts, rec_token, pair_expert, pair_rec
+        self.ret_pos, self.bad = ret_pos, bad
+
+    @property
+    def num_ranks(self) -> int:
+        return self.counts.size // 2
+
+    def records_to(self, p: int) -> slice:
+        c = self.counts[: self.num_ranks]
+        return slice(int(c[:p].sum()), int(c[: p + 1].sum()))
+
+    def pairs_to(self, p: int) -> slice:
+        c = self.counts[self.num_ranks:]
+        return slice(int(c[:p].sum()), int(c[: p + 1].sum()))
+
+
+def ep_plan(idx, E: int, P: int) -> EpPlan:
+    """idx: int [T, k] global expert ids; P ranks owning E/P consecutive experts each."""
+    idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int32))
+    T, k = idx.shape
+    cap = max(T * k, 1)
+    counts = np.zeros(2 * P, dtype=np.int32)
+    rec_token = np.zeros(cap, dtype=np.int32)
+    pair_expert = np.zeros(cap, dtype=np.int32)
+    pair_rec = np.zeros(cap, dtype=np.int32)
+    ret_pos = np.zeros((T, k), dtype=np.int32)
+    bad = lib().orc_ep_plan(_p(idx), T, k, E, P, _p(counts), _p(rec_token), _p(pair_expert), _p(pair_rec),
+                            _p(ret_pos))
+    if bad < 0:
+        raise ValueError("ep_plan: P < 1 or E not a positive multiple of P")
+    R, S = int(counts[:P].sum()), int(counts[P:].sum())
+    return EpPlan(counts, rec_token[:R].copy(), pair_expert[:S].copy(), pair_rec[:S].copy(), ret_pos, int(bad))
+
+
+def ep_record_bytes(C: int) -> int:
+    return int(lib().orc_ep_record_bytes(C))
+
+
+def ep_pack(x, rec_token) -> np.ndarray:
+    """x: bf16 [T, C] -> records uint8 [R, ep_record_bytes(C)] (rowwise MXFP8 of row rec_token[i])."""
+    xu = _u16(x)
+    T, C = xu.shape
+    rt = np.ascontiguousarray(np.asarray(rec_token, dtype=np.int32))
+    out = np.zeros((rt.size, ep_record_bytes(C)), dtype=np.uint8)
+    _check(lib().orc_ep_pack(_p(xu), T, C, _p(rt), rt.size, _p(out)), "ep_pack")
+    return out
+
+
+def ep_source_bases(recv_counts) -> np.ndarray:
+    """recv_counts int [2P] (records from each source, then pairs from each
+    source) -> src_base int32 [2(P+1)]: pair bases then record bases."""
+    c = np.asarray(recv_counts, dtype=np.int64)
+    P = c.size // 2
+    rec, pairs = c[:P], c[P:]
+    return np.concatenate([[0], np.cumsum(pairs), [0], np.cumsum(rec)]).astype(np.int32)
+
+
+def ep_unpack(records, C: int, pair_rec, src_base, perm, offs):
+    """Received records + pair entries -> rowwise MXFP8 (q [M, C], sf) of the
+    grouped rows, as quantize_rowwise would write them."""
+    rec = np.ascontiguousarray(records, dtype=np.uint8)
+    R = rec.shape[0]
+    pr = np.ascontiguousarray(np.asarray(pair_rec, dtype=np.int32))
+    sb = np.ascontiguousarray(np.asarray(src_base, dtype=np.int32))
+    pm = np.ascontiguousarray(np.asarray(perm, dtype=np.int32))
+    M = pm.size
+    o, G = _offs(offs, M)
+    P = sb.size // 2 - 1
+    q = np.zeros((M, C), dtype=np.uint8)
+    sf = np.zeros(max(rowwise_scale_bytes(M, C, G), 512), dtype=np.uint8)
+    _check(lib().orc_ep_unpack(_p(rec), R, C, _p(pr), _p(sb), P, _p(pm), M, _p(o), G, _p(q), _p(sf)), "ep_unpack")
+    return q, sf
 
 
 # ---------------------------------------------------------------- NVFP4

@@ -692,6 +692,130 @@ int orc_swiglu(const double* Y, int64_t M, int64_t I, uint16_t* h)
 }
 
 /* ------------------------------------------------------------------ */
+/* Expert-parallel dispatch: the plan, and MXFP8 rows sent once per rank */
+/* ------------------------------------------------------------------ */
+/* Each MoE layer sends every token to the GPUs holding its experts and
+ * brings the results back (opensourcebeat.com, section "Двухсторонняя
+ * атака: MXFP8 и DeepEP"); a token needed by several experts of one
+ * destination crosses the network once and is copied there (iitak.ru,
+ * "NVIDIA ... JAX", paragraph on NCCL EP).  Readings where the pages are
+ * silent: P ranks own E/P consecutive experts each (rank p owns experts
+ * p*E/P .. (p+1)*E/P - 1); a token travels as one record per destination
+ * rank, carrying the token's row as rowwise MXFP8 (its codes, then its
+ * 32-block scale bytes); each (token, slot) pair routed to that rank travels
+ * as a pair entry (local expert id, record index).  Send order: destination
+ * rank, then token, then slot, all ascending. */
+
+/* idx: int32 [T, k] global expert ids.  Outputs, in send order:
+ *   counts[p]         records sent to rank p;  counts[P + p]  pairs sent to p
+ *   rec_token[i]      token of record i (records of rank p after those of
+ *                     ranks < p)
+ *   pair_expert[s]    local expert id (e mod E/P) of pair s
+ *   pair_rec[s]       record of pair s, counted from the first record sent
+ *                     to the same rank
+ *   ret_pos[t*k + j]  pair index s of slot (t, j) -- the row at which its
+ *                     expert output comes back -- or -1 when the id is
+ *                     outside [0, E) (such a slot is not sent).
+ * Returns the number of slots with an id outside [0, E), or -1 when P < 1
+ * or E is not a positive multiple of P. */
+int64_t orc_ep_plan(const int32_t* idx, int64_t T, int32_t k, int32_t E, int32_t P, int32_t* counts,
+                    int32_t* rec_token, int32_t* pair_expert, int32_t* pair_rec, int32_t* ret_pos)
+{
+    int64_t t, rec = 0, pair = 0, bad = 0;
+    int32_t p, j, epr;
+    if (P < 1 || E < 1 || E % P != 0 || k < 1) return -1;
+    epr = E / P;
+    for (t = 0; t < T * k; ++t) {
+        ret_pos[t] = -1;
+        if (idx[t] < 0 || idx[t] >= E) bad += 1;
+    }
+    for (p = 0; p < P; ++p) {
+        int64_t rec0 = rec, pair0 = pair;
+        for (t = 0; t < T; ++t) {
+            int64_t mine = -1;   /* this token's record for rank p, once made */
+            for (j = 0; j < k; ++j) {
+                int32_t e = idx[t * k + j];
+                if (e < 0 || e >= E || e / epr != p) continue;
+                if (mine < 0) {
+                    mine = rec - rec0;
+                    rec_token[rec++] = (int32_t)t;
+                }
+                pair_expert[pair] = e % epr;
+                pair_rec[pair] = (int32_t)mine;
+                ret_pos[t * k + j] = (int32_t)pair;
+                pair += 1;
+            }
+        }
+        counts[p] = (int32_t)(rec - rec0);
+        counts[P + p] = (int32_t)(pair - pair0);
+    }
+    return bad;
+}
+
+/* Bytes of one record holding a row of C elements: C codes, C/32 scale
+ * bytes, zero padding to a multiple of 16. */
+int64_t orc_ep_record_bytes(int64_t C) { return rup(C + C / 32, 16); }
+
+/* x: bf16 [T, C], C % 32 == 0.  Record i holds the MXFP8 rowwise encoding
+ * of row rec_token[i]: byte 32b + n is the code of element 32b + n, byte
+ * C + b the scale byte of block b, the rest zero.  A token index outside
+ * [0, T) gives an all-zero record. */
+int orc_ep_pack(const uint16_t* x, int64_t T, int64_t C, const int32_t* rec_token, int64_t R, uint8_t* rec)
+{
+    int64_t stride = orc_ep_record_bytes(C), i;
+    if (C % 32 != 0 || C <= 0) return 1;
+#pragma omp parallel for schedule(static)
+    for (i = 0; i < R; ++i) {
+        uint8_t* r = rec + i * stride;
+        int64_t t = rec_token[i], b;
+        memset(r, 0, (size_t)stride);
+        if (t < 0 || t >= T) continue;
+        for (b = 0; b < C / 32; ++b) orc_quantize_block(x + t * C + 32 * b, 32, 1, r + 32 * b, 1, r + C + b);
+    }
+    return 0;
+}
+
+/* Receiving side: R records and M pairs arrived from P source ranks, each
+ * source's records and pairs after those of lower ranks.  src_base[q] is
+ * the first pair and src_base[P + 1 + q] the first record from source q
+ * (src_base[P], src_base[2P + 1] the totals).  Grouped row r (rows grouped
+ * by local expert with offs, G groups) is pair perm[r]; its record is
+ * src_base[P + 1 + q] + pair_rec[perm[r]] for the source q whose pairs hold
+ * perm[r].  Writes the rowwise MXFP8 layout of the grouped rows: codes
+ * q [M, C] and scale atoms (pitch ceil(C/128), the first RB_G * pitch * 512
+ * bytes).  Returns 1 on bad sizes, offsets or an index out of range. */
+int orc_ep_unpack(const uint8_t* rec, int64_t R, int64_t C, const int32_t* pair_rec, const int32_t* src_base,
+                  int32_t P, const int32_t* perm, int64_t M, const int32_t* offs, int32_t G, uint8_t* q,
+                  uint8_t* sf)
+{
+    int64_t stride = orc_ep_record_bytes(C), pitch = orc_rowwise_pitch(C), nb = C / 32;
+    int64_t *RB, *Pp;
+    int32_t g;
+    int bad = 0;
+    if (C % 32 != 0 || C <= 0 || G < 1 || P < 1 || orc_check_offsets(offs, G, M)) return 1;
+    if (src_base[P] != M || src_base[2 * P + 1] != R) return 1;
+    RB = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
+    Pp = (int64_t*)malloc(sizeof(int64_t) * (G + 1));
+    group_prefixes(offs, G, M, RB, Pp);
+    memset(sf, 0, (size_t)(RB[G] * pitch * 512));
+    for (g = 0; g < G; ++g) {
+        int64_t lo, hi, r;
+        group_bounds(offs, G, M, g, &lo, &hi);
+        for (r = lo; r < hi; ++r) {
+            int64_t s = perm[r], i, j, src = 0;
+            if (s < 0 || s >= M) { bad = 1; continue; }
+            while (src + 1 < P && src_base[src + 1] <= s) src += 1;
+            i = (int64_t)src_base[P + 1 + src] + pair_rec[s];
+            if (i < 0 || i >= R) { bad = 1; continue; }
+            memcpy(q + r * C, rec + i * stride, (size_t)C);
+            for (j = 0; j < nb; ++j) sf[orc_sf_offset(128 * RB[g] + (r - lo), j, pitch)] = rec[i * stride + C + j];
+        }
+    }
+    free(RB); free(Pp);
+    return bad;
+}
+
+/* ------------------------------------------------------------------ */
 /* NVFP4: 4-bit E2M1 elements, 16-element blocks with E4M3 scales and   */
 /* one fp32 scale per tensor                                             */
 /* ------------------------------------------------------------------ */
