@@ -395,6 +395,7 @@ def run_ours(args, rank, world, local_rank):
                                "target": 0.60, "peak": round(fp8_peak, 1)}
         out["quantising_epilogue"] = quantising_epilogue(mx, layers[0])
         out["moe_dispatch"] = moe_dispatch(mx, args, pk["hbm_gbs"])
+        out["ep_dispatch"] = ep_dispatch(mx, pk["hbm_gbs"])
         out["nvfp4"] = nvfp4_measure(mx, layers[0], fp8_peak, pk["hbm_gbs"])
         out["quantiser_sweep"] = quantiser_sweep(mx, pk["hbm_gbs"])
     return out
@@ -672,6 +673,82 @@ def moe_dispatch(mx, args, hbm_gbs, iters=20):
             "permute_quantize_frac": round(pq_bytes / (pq_ms * 1e-3) / 1e9 / hbm_gbs, 4),
             "combine_ms": round(cb_ms, 4), "combine_gbs": round(cb_bytes / (cb_ms * 1e-3) / 1e9, 1),
             "combine_frac": round(cb_bytes / (cb_ms * 1e-3) / 1e9 / hbm_gbs, 4)}
+
+
+def ep_dispatch(mx, hbm_gbs, iters=20):
+    """The expert-parallel exchange's device work for a DeepSeek-V3-671B-like
+    layer split over 8 ranks (16384 tokens, 2048 per rank, hidden 7168, top-8
+    of 256 experts with N(0,1) logits + N(0,0.5) expert bias, 32 experts per
+    rank), on one GPU: one source's plan and quantise-and-pack, one
+    receiver's unpack of what the 8 sources send it (assembled here as the
+    all-to-all delivers it), and the return gather of its expert outputs.
+    The transfer itself is not timed (one GPU per run)."""
+    from mxfp8_grouped_gemm_quantize_b200 import ep
+    P, Tr, k, E, C = 8, 2048, 8, 256, 7168
+    epr = E // P
+    dev = torch.device("cuda", torch.cuda.current_device())
+    rng = np.random.default_rng(4242)
+    bias = rng.normal(0.0, 0.5, E)
+    srcs = []
+    for q in range(P):
+        logits = rng.standard_normal((Tr, E)) + bias[None, :]
+        idx = torch.from_numpy(np.argsort(-logits, axis=1, kind="stable")[:, :k].astype(np.int32)).to(dev)
+        x = wl.normal_bf16((Tr, C), 1.0, 300 + q, device=dev)
+        counts, rec_token, pe, prc, ret_pos, work = mx.mxfp8_ep_plan(idx, E, P)
+        cnt = counts.tolist()
+        R, S = sum(cnt[:P]), sum(cnt[P:])
+        srcs.append((idx, x, cnt, rec_token[:R], pe[:S], prc[:S], work, mx.mxfp8_ep_pack(x, rec_token[:R])))
+
+    def t(fn):
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(iters):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+
+    idx0, x0, cnt0, rt0, _, _, work0, recs0 = srcs[0]
+    plan_ms = t(lambda: mx.mxfp8_ep_plan(idx0, E, P, work=work0))
+    pack_ms = t(lambda: mx.mxfp8_ep_pack(x0, rt0, out=recs0))
+    stride = mx.mxfp8_ep_record_bytes(C)
+    R0, S0 = sum(cnt0[:P]), sum(cnt0[P:])
+
+    def block(c, p):
+        return slice(sum(c[:p]), sum(c[:p + 1]))
+    recs = torch.cat([s[7][block(s[2][:P], 0)] for s in srcs])
+    pe = torch.cat([s[4][block(s[2][P:], 0)] for s in srcs])
+    prc = torch.cat([s[5][block(s[2][P:], 0)] for s in srcs])
+    rc = [s[2][0] for s in srcs] + [s[2][P] for s in srcs]
+    d = ep.Dispatch(recs, pe, prc, rc, cnt0, C)
+    offs, perm, inv, q, sf = ep.receive(d, epr)
+    src_base = torch.tensor(ep.source_bases(rc), dtype=torch.int32, device=dev)
+    unpack_ms = t(lambda: mx.mxfp8_ep_unpack(recs, C, prc, src_base, perm, offs, q, sf))
+    rows = perm.numel()
+    y = wl.normal_bf16((rows, C), 1.0, 333, device=dev)
+    y_ret = torch.empty_like(y)
+    inv_flat = inv.view(-1).contiguous()
+    gather_ms = t(lambda: mx.mxfp8_gather_rows(y, inv_flat, out=y_ret))
+    pack_bytes = R0 * (2 * C + stride)
+    unpack_bytes = rows * 2 * (C + C // 32)
+    gather_bytes = rows * C * 2 * 2
+    wire = R0 * stride + S0 * 8
+    return {"layout": f"{P} ranks x {Tr} tokens, hidden {C}, top-{k} of {E} experts ({epr} per rank)",
+            "records_sent": R0, "pairs_sent": S0,
+            "dispatch_bytes": wire, "dispatch_bytes_bf16_rows": S0 * 2 * C,
+            "dispatch_bytes_ratio": round(wire / (S0 * 2 * C), 4),
+            "plan_ms": round(plan_ms, 4),
+            "pack_ms": round(pack_ms, 4), "pack_gbs": round(pack_bytes / (pack_ms * 1e-3) / 1e9, 1),
+            "pack_frac": round(pack_bytes / (pack_ms * 1e-3) / 1e9 / hbm_gbs, 4),
+            "receiver_rows": rows,
+            "unpack_ms": round(unpack_ms, 4), "unpack_gbs": round(unpack_bytes / (unpack_ms * 1e-3) / 1e9, 1),
+            "unpack_frac": round(unpack_bytes / (unpack_ms * 1e-3) / 1e9 / hbm_gbs, 4),
+            "return_gather_ms": round(gather_ms, 4),
+            "return_gather_gbs": round(gather_bytes / (gather_ms * 1e-3) / 1e9, 1),
+            "note": "device work only; the all-to-all transfer is not measured (one GPU per run)"}
 
 
 def nvfp4_measure(mx, L: Linear, fp8_peak, hbm_gbs, iters=20):

@@ -358,6 +358,92 @@ MXF8_API mxf8_status mxfp8_moe_combine(const uint16_t* yp, int64_t rows, int64_t
                                        const float* w, int64_t num_tokens, int32_t top_k, uint16_t* y,
                                        void* stream);
 
+/* ---------------------------------------------------------------- expert-parallel dispatch */
+/* What an expert-parallel MoE layer sends between GPUs.  Each layer sends
+ * every token to the GPUs holding its experts and brings the expert outputs
+ * back (opensourcebeat.com, "Enabling up to 41% faster pre-training: MXFP8
+ * and DeepEP ...", section "Двухсторонняя атака: MXFP8 и DeepEP"); a token
+ * needed by several experts of one destination crosses the network once and
+ * is copied there (iitak.ru, "NVIDIA в 10 раз ускорила обучение
+ * моделей-«смесей экспертов» на JAX", paragraph on NCCL EP).  These calls
+ * prepare and unpack what travels; the transfer itself is the caller's
+ * (an NCCL all-to-all, split by the counts below).
+ *
+ * Readings (the pages give no format): P ranks own E/P consecutive experts
+ * each (rank p: experts p*E/P .. (p+1)*E/P - 1).  A token travels to each
+ * rank owning one of its experts as one record: its row in rowwise MXFP8 --
+ * byte 32b + n is the E4M3 code of element 32b + n, byte C + b the E8M0 scale
+ * byte of block b (the quantisers' block rule), then zeros up to
+ * mxfp8_ep_record_bytes(C) -- 1 + 1/32 bytes per element instead of bf16's 2.
+ * Each routed (token, slot) pair travels as a pair entry: its local expert
+ * id (e - p*E/P) and its record index, counted from the first record sent to
+ * that rank.  Send order: destination rank, then token, then slot, all
+ * ascending; a receiver concatenates what its sources sent in rank order. */
+
+#define MXF8_EP_MAX_RANKS 256
+#define MXF8_EP_MAX_TOP_K 32
+
+/* Bytes of one record holding a row of `cols` elements (a multiple of 16). */
+MXF8_API int64_t mxfp8_ep_record_bytes(int64_t cols);
+
+/* Workspace of mxfp8_ep_plan in bytes. */
+MXF8_API int64_t mxfp8_ep_plan_workspace_bytes(int64_t num_tokens, int32_t num_ranks);
+
+/* Send plan of a top-k routing over P ranks (no host synchronisation).
+ *   idx          int32 [T, k] global expert ids
+ *   counts       int32 [2P] out: records sent to rank p at [p], pairs at [P + p]
+ *   rec_token    int32 [T * min(k, P)] out: token of record i (the first
+ *                sum(counts[0..P-1]) entries are written)
+ *   pair_expert  int32 [T * k] out: local expert id of pair s
+ *   pair_rec     int32 [T * k] out: record of pair s within its rank's records
+ *   ret_pos      int32 [T, k] out: pair index of slot (t, j) -- the row of
+ *                the returned expert outputs that belongs to it -- or -1
+ * An id outside [0, E) is not sent (ret_pos -1) and sets the device status
+ * (mxfp8_get_status(work)) to MXF8_ERR_BAD_ROUTING.
+ * Errors: INVALID_ARG (null pointers, T < 0, k outside [1, MXF8_EP_MAX_TOP_K],
+ * P outside [1, MXF8_EP_MAX_RANKS], E < 1 or not a multiple of P, T*k >= 2^31,
+ * small workspace), ALIGNMENT (work), UNSUPPORTED, CUDA. */
+MXF8_API mxf8_status mxfp8_ep_plan(const int32_t* idx, int64_t num_tokens, int32_t top_k, int32_t num_experts,
+                                   int32_t num_ranks, int32_t* counts, int32_t* rec_token, int32_t* pair_expert,
+                                   int32_t* pair_rec, int32_t* ret_pos, void* work, int64_t work_bytes,
+                                   void* stream);
+
+/* Quantise and pack: record i = rowwise MXFP8 of x[rec_token[i]] (a token
+ * index outside [0, T) packs an all-zero record).
+ *   x        bf16 [T, cols], cols % 32 == 0, 16-byte aligned
+ *   records  uint8 [num_records, mxfp8_ep_record_bytes(cols)] out, 16-byte aligned
+ * Errors: INVALID_ARG (null pointers, sizes), ALIGNMENT, UNSUPPORTED, CUDA. */
+MXF8_API mxf8_status mxfp8_ep_pack(const uint16_t* x, int64_t num_tokens, int64_t cols, const int32_t* rec_token,
+                                   int64_t num_records, uint8_t* records, void* stream);
+
+/* Receiving side.  R records and `rows` pair entries arrived from P sources,
+ * each source's after those of lower ranks; src_base int32 [2(P + 1)]
+ * (device) holds the first pair of each source at [q] (the total at [P]) and
+ * its first record at [P + 1 + q] (the total at [2P + 1]).  Grouped row r
+ * (rows grouped by local expert with d_offs, e.g. mxfp8_moe_plan of the pair
+ * entries' expert ids) is pair perm[r]; its record is
+ * src_base[P + 1 + q] + pair_rec[perm[r]], q the source whose pairs hold
+ * perm[r].  Writes the grouped rows' rowwise MXFP8 -- codes q [rows, cols]
+ * and scale atoms -- byte for byte what mxfp8_quantize_rowwise writes for
+ * the bf16 rows the records were made from (rowwise blocks lie within one
+ * row, so quantising before the transfer changes nothing).  A pair or record
+ * index out of range gives a zero row.
+ * Errors: INVALID_ARG (null pointers, cols % 32, P outside
+ * [1, MXF8_EP_MAX_RANKS], num_groups < 1, small scale buffer), ALIGNMENT
+ * (records, q, scales), UNSUPPORTED, CUDA. */
+MXF8_API mxf8_status mxfp8_ep_unpack(const uint8_t* records, int64_t num_records, int64_t cols,
+                                     const int32_t* pair_rec, const int32_t* src_base, int32_t num_sources,
+                                     const int32_t* perm, int64_t rows, const int32_t* d_offs, int32_t num_groups,
+                                     uint8_t* q, uint8_t* scales, int64_t scale_bytes, void* stream);
+
+/* dst[i] = src[idx[i]] for rows of row_bytes bytes (a multiple of 16); an
+ * index outside [0, src_rows) gives a zero row.  Used for the return trip:
+ * each received pair's expert output row, in arrival order.
+ * Errors: INVALID_ARG (null pointers, sizes), ALIGNMENT (src, dst),
+ * UNSUPPORTED, CUDA. */
+MXF8_API mxf8_status mxfp8_gather_rows(const void* src, int64_t src_rows, int64_t row_bytes, const int32_t* idx,
+                                       int64_t n, void* dst, void* stream);
+
 /* ---------------------------------------------------------------- NVFP4 */
 /* NVFP4 quantisation: 4-bit E2M1 elements in blocks of 16 that share an E4M3
  * scale, plus one fp32 scale per tensor.  The pages name NVFP4 only as the

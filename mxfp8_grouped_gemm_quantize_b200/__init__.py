@@ -41,7 +41,9 @@ EXPORTED = ("mxfp8_rowwise_scale_bytes", "mxfp8_colwise_pitch", "mxfp8_colwise_s
             "mxfp8_nvfp4_colwise_pitch", "mxfp8_nvfp4_colwise_scale_bytes", "mxfp8_nvfp4_colwise_ld",
             "mxfp8_nvfp4_amax", "mxfp8_nvfp4_quantize_rowwise", "mxfp8_nvfp4_quantize_colwise",
             "mxfp8_nvfp4_grouped_gemm_fwd", "mxfp8_nvfp4_grouped_gemm_dgrad", "mxfp8_nvfp4_grouped_gemm_wgrad",
-            "mxfp8_set_gemm_tiling", "mxfp8_testing_stall_first_stage", "mxfp8_grouped_gemm_fwd_swiglu")
+            "mxfp8_set_gemm_tiling", "mxfp8_testing_stall_first_stage", "mxfp8_grouped_gemm_fwd_swiglu",
+            "mxfp8_ep_record_bytes", "mxfp8_ep_plan_workspace_bytes", "mxfp8_ep_plan", "mxfp8_ep_pack",
+            "mxfp8_ep_unpack", "mxfp8_gather_rows")
 
 
 class MXFP8Error(RuntimeError):
@@ -111,6 +113,18 @@ def lib() -> ctypes.CDLL:
         L.mxfp8_grouped_gemm_fwd_noalloc.restype = _i32
         L.mxfp8_grouped_gemm_fwd_noalloc.argtypes = [_vp, _vp, _i64, _vp, _vp, _i64, _vp, _i32, _i64, _i64, _i64, _vp,
                                                      ctypes.POINTER(_i32), _vp]
+        L.mxfp8_ep_record_bytes.restype = _i64
+        L.mxfp8_ep_record_bytes.argtypes = [_i64]
+        L.mxfp8_ep_plan_workspace_bytes.restype = _i64
+        L.mxfp8_ep_plan_workspace_bytes.argtypes = [_i64, _i32]
+        L.mxfp8_ep_plan.restype = _i32
+        L.mxfp8_ep_plan.argtypes = [_vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
+        L.mxfp8_ep_pack.restype = _i32
+        L.mxfp8_ep_pack.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _vp]
+        L.mxfp8_ep_unpack.restype = _i32
+        L.mxfp8_ep_unpack.argtypes = [_vp, _i64, _i64, _vp, _vp, _i32, _vp, _i64, _vp, _i32, _vp, _vp, _i64, _vp]
+        L.mxfp8_gather_rows.restype = _i32
+        L.mxfp8_gather_rows.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _vp]
         L.mxfp8_get_status.restype = _i32
         L.mxfp8_get_status.argtypes = [_vp, _vp, ctypes.POINTER(_i32)]
         L.mxfp8_status_string.restype = ctypes.c_char_p
@@ -392,6 +406,75 @@ def mxfp8_moe_combine(yp: torch.Tensor, inv: torch.Tensor, w: torch.Tensor, out=
     out = out if out is not None else torch.empty((T, C), dtype=torch.bfloat16, device=yp.device)
     _check(lib().mxfp8_moe_combine(_ptr(yp) if rows else None, rows, C, _ptr(inv), _ptr(w), T, k, _ptr(out),
                                    _stream(stream)), "mxfp8_moe_combine")
+    return out
+
+
+# ------------------------------------------------------------------ expert-parallel dispatch
+def mxfp8_ep_record_bytes(cols: int) -> int:
+    return int(lib().mxfp8_ep_record_bytes(cols))
+
+
+def mxfp8_ep_plan(idx: torch.Tensor, num_experts: int, num_ranks: int, work=None, stream=None):
+    """idx: int32 [T, k] global expert ids -> (counts int32 [2P], rec_token int32 [T*min(k,P)],
+    pair_expert int32 [T*k], pair_rec int32 [T*k], ret_pos int32 [T, k], work); the first
+    sum(counts[:P]) records and sum(counts[P:]) pairs are written."""
+    assert idx.dtype == torch.int32 and idx.dim() == 2
+    T, k = idx.shape
+    dev = idx.device
+    P = num_ranks
+    counts = torch.empty(2 * P, dtype=torch.int32, device=dev)
+    rec_token = torch.empty(max(T * min(k, P), 1), dtype=torch.int32, device=dev)
+    pair_expert = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+    pair_rec = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+    ret_pos = torch.empty((T, k), dtype=torch.int32, device=dev)
+    need = lib().mxfp8_ep_plan_workspace_bytes(T, P)
+    work = work if work is not None else torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib().mxfp8_ep_plan(_ptr(idx) if T else None, T, k, num_experts, P, _ptr(counts), _ptr(rec_token),
+                               _ptr(pair_expert), _ptr(pair_rec), _ptr(ret_pos) if T else None, _ptr(work),
+                               work.numel(), _stream(stream)), "mxfp8_ep_plan")
+    return counts, rec_token, pair_expert, pair_rec, ret_pos, work
+
+
+def mxfp8_ep_pack(x: torch.Tensor, rec_token: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """x: bf16 [T, cols]; rec_token int32 [R] -> records uint8 [R, mxfp8_ep_record_bytes(cols)]."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and rec_token.dtype == torch.int32
+    T, C = x.shape
+    R = rec_token.numel()
+    out = out if out is not None else torch.empty((R, mxfp8_ep_record_bytes(C)), dtype=torch.uint8, device=x.device)
+    _check(lib().mxfp8_ep_pack(_ptr(x) if x.numel() else None, T, C, _ptr(rec_token) if R else None, R,
+                               _ptr(out) if R else None, _stream(stream)), "mxfp8_ep_pack")
+    return out
+
+
+def mxfp8_ep_unpack(records: torch.Tensor, cols: int, pair_rec: torch.Tensor, src_base: torch.Tensor,
+                    perm: torch.Tensor, offs: torch.Tensor, q=None, scales=None, stream=None):
+    """Received records and pair entries -> (q uint8 [rows, cols], scales): the grouped rows'
+    rowwise MXFP8; src_base int32 [2(P+1)] on the device (first pair, then first record, of each source)."""
+    assert records.dtype == torch.uint8 and pair_rec.dtype == torch.int32 and perm.dtype == torch.int32
+    assert src_base.dtype == torch.int32 and src_base.is_cuda
+    R = records.shape[0]
+    rows = perm.numel()
+    G = _groups(offs)
+    P = src_base.numel() // 2 - 1
+    dev = records.device
+    q = q if q is not None else torch.empty((rows, cols), dtype=torch.uint8, device=dev)
+    scales = scales if scales is not None else _u8(mxfp8_rowwise_scale_bytes(rows, cols, G), dev)
+    _check(lib().mxfp8_ep_unpack(_ptr(records) if R else None, R, cols, _ptr(pair_rec) if rows else None,
+                                 _ptr(src_base), P, _ptr(perm) if rows else None, rows, _ptr(offs), G,
+                                 _ptr(q) if rows else None, _ptr(scales), scales.numel(), _stream(stream)),
+           "mxfp8_ep_unpack")
+    return q, scales
+
+
+def mxfp8_gather_rows(src: torch.Tensor, idx: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """out[i] = src[idx[i]] (rows of a 2-D tensor; zero rows for indices out of range)."""
+    assert src.dim() == 2 and idx.dtype == torch.int32
+    n = idx.numel()
+    row_bytes = src.shape[1] * src.element_size()
+    out = out if out is not None else torch.empty((n, src.shape[1]), dtype=src.dtype, device=src.device)
+    _check(lib().mxfp8_gather_rows(_ptr(src) if src.numel() else None, src.shape[0], row_bytes,
+                                   _ptr(idx) if n else None, n, _ptr(out) if n else None, _stream(stream)),
+           "mxfp8_gather_rows")
     return out
 
 

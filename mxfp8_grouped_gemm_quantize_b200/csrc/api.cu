@@ -8,6 +8,7 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "ep_launch.h"
 #include "launch.h"
 #include "mxfp8.h"
 
@@ -427,6 +428,85 @@ mxf8_status mxfp8_moe_combine(const uint16_t* yp, int64_t rows, int64_t cols, co
   cudaError_t e = mxf8::launch_moe_combine(yp, rows, cols, inv, w, num_tokens, top_k, y,
                                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "moe_combine launch");
+}
+
+int64_t mxfp8_ep_record_bytes(int64_t cols) {
+  if (cols <= 0 || cols % 32 != 0) return 0;
+  return mxf8::ep_record_stride(cols);
+}
+
+int64_t mxfp8_ep_plan_workspace_bytes(int64_t num_tokens, int32_t num_ranks) {
+  if (num_tokens < 0 || num_ranks < 1 || num_ranks > MXF8_EP_MAX_RANKS) return 0;
+  // status word | first record of each rank | per-chunk counts (records, pairs per rank)
+  return kWorkspaceBytes + MXF8_EP_MAX_RANKS * 4 + round_up(mxf8::ep_plan_chunks(num_tokens) * 2 * num_ranks * 4, 256);
+}
+
+mxf8_status mxfp8_ep_plan(const int32_t* idx, int64_t num_tokens, int32_t top_k, int32_t num_experts,
+                          int32_t num_ranks, int32_t* counts, int32_t* rec_token, int32_t* pair_expert,
+                          int32_t* pair_rec, int32_t* ret_pos, void* work, int64_t work_bytes, void* stream) {
+  if (num_tokens < 0 || top_k < 1 || top_k > MXF8_EP_MAX_TOP_K) return MXF8_ERR_INVALID_ARG;
+  if (num_ranks < 1 || num_ranks > MXF8_EP_MAX_RANKS || num_experts < 1 || num_experts % num_ranks != 0)
+    return MXF8_ERR_INVALID_ARG;
+  if (num_tokens * top_k >= (int64_t(1) << 31)) return MXF8_ERR_INVALID_ARG;
+  if (!counts || !work || (num_tokens > 0 && (!idx || !rec_token || !pair_expert || !pair_rec || !ret_pos)))
+    return MXF8_ERR_INVALID_ARG;
+  if (work_bytes < mxfp8_ep_plan_workspace_bytes(num_tokens, num_ranks)) return MXF8_ERR_INVALID_ARG;
+  if (!aligned16(work)) return MXF8_ERR_ALIGNMENT;
+  mxf8_status s = check_device();
+  if (s != MXF8_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(work);
+  int32_t* status = reinterpret_cast<int32_t*>(w);
+  int32_t* rec_base = reinterpret_cast<int32_t*>(w + kWorkspaceBytes);
+  int32_t* hist = reinterpret_cast<int32_t*>(w + kWorkspaceBytes + MXF8_EP_MAX_RANKS * 4);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  e = mxf8::launch_ep_plan(idx, num_tokens, top_k, num_experts, num_ranks, counts, rec_token, pair_expert, pair_rec,
+                           ret_pos, status, rec_base, hist, st);
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "ep_plan launch");
+}
+
+mxf8_status mxfp8_ep_pack(const uint16_t* x, int64_t num_tokens, int64_t cols, const int32_t* rec_token,
+                          int64_t num_records, uint8_t* records, void* stream) {
+  if (num_tokens < 0 || num_records < 0 || cols <= 0 || cols % 32 != 0) return MXF8_ERR_INVALID_ARG;
+  if (num_records > (int64_t(1) << 31) - 1 || cols > (int64_t(1) << 30)) return MXF8_ERR_INVALID_ARG;
+  if (num_records > 0 && (!rec_token || !records || (num_tokens > 0 && !x))) return MXF8_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(records)) return MXF8_ERR_ALIGNMENT;
+  mxf8_status s = check_device();
+  if (s != MXF8_OK) return s;
+  cudaError_t e = mxf8::launch_ep_pack(x, num_tokens, cols, rec_token, num_records, records,
+                                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "ep_pack launch");
+}
+
+mxf8_status mxfp8_ep_unpack(const uint8_t* records, int64_t num_records, int64_t cols, const int32_t* pair_rec,
+                            const int32_t* src_base, int32_t num_sources, const int32_t* perm, int64_t rows,
+                            const int32_t* d_offs, int32_t num_groups, uint8_t* q, uint8_t* scales,
+                            int64_t scale_bytes, void* stream) {
+  if (num_records < 0 || num_sources < 1 || num_sources > MXF8_EP_MAX_RANKS) return MXF8_ERR_INVALID_ARG;
+  if (!d_offs || !src_base || (rows > 0 && (!pair_rec || !perm || (num_records > 0 && !records))))
+    return MXF8_ERR_INVALID_ARG;
+  // the rows' codes and scales follow the rowwise quantiser's rules and layout
+  mxf8_status s = check_quant_args(nullptr, 0, cols, num_groups, q, scales, scale_bytes,
+                                   mxfp8_rowwise_scale_bytes(rows, cols, num_groups));
+  if (s != MXF8_OK) return s;
+  if (rows < 0 || rows > (int64_t(1) << 31) - 1 || (rows > 0 && !q)) return MXF8_ERR_INVALID_ARG;
+  if (!aligned16(records)) return MXF8_ERR_ALIGNMENT;
+  if ((s = check_device()) != MXF8_OK) return s;
+  cudaError_t e = mxf8::launch_ep_unpack(records, num_records, cols, pair_rec, src_base, num_sources, perm, rows,
+                                         d_offs, num_groups, q, scales, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "ep_unpack launch");
+}
+
+mxf8_status mxfp8_gather_rows(const void* src, int64_t src_rows, int64_t row_bytes, const int32_t* idx, int64_t n,
+                              void* dst, void* stream) {
+  if (src_rows < 0 || n < 0 || row_bytes <= 0 || row_bytes % 16 != 0) return MXF8_ERR_INVALID_ARG;
+  if (n > 0 && (!idx || !dst || (src_rows > 0 && !src))) return MXF8_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return MXF8_ERR_ALIGNMENT;
+  mxf8_status s = check_device();
+  if (s != MXF8_OK) return s;
+  cudaError_t e = mxf8::launch_gather_rows(src, src_rows, row_bytes, idx, n, dst, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "gather_rows launch");
 }
 
 int64_t mxfp8_nvfp4_rowwise_scale_bytes(int64_t rows, int64_t cols, int32_t num_groups) {

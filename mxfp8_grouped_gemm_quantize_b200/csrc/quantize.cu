@@ -34,39 +34,6 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return r;
 }
 
-// Resolves this CTA's 128-row block (blockIdx.x) to rows of a group.
-// Returns false if the block lies past the last group's blocks.
-struct BlockRows {
-  int64_t row0;     // first input row
-  int nrows;        // real rows in the block (<= 128)
-  int64_t dst0;     // colwise: first code column (P_g + 128*local)
-  int padded;       // colwise: written code columns (multiple of 32, <= 128)
-};
-
-__device__ __forceinline__ bool resolve_block(const int32_t* offs, int32_t G, int64_t rows,
-                                              BlockRows* out) {
-  __shared__ BlockRows s_br;
-  __shared__ int s_ok;
-  if (threadIdx.x < 32) {
-    const GroupBlock gb = warp_find_block(offs, G, rows, blockIdx.x);
-    if (threadIdx.x == 0) {
-      s_ok = gb.g >= 0;
-      if (gb.g >= 0) {
-        const int64_t local = static_cast<int64_t>(blockIdx.x) - gb.rb;
-        const int64_t left = gb.m - 128 * local;
-        const int64_t pad_left = (gb.m + 31) / 32 * 32 - 128 * local;
-        s_br.row0 = gb.lo + 128 * local;
-        s_br.nrows = static_cast<int>(left < 128 ? left : 128);
-        s_br.dst0 = gb.p + 128 * local;
-        s_br.padded = static_cast<int>(pad_left < 128 ? pad_left : 128);
-      }
-    }
-  }
-  __syncthreads();
-  *out = s_br;
-  return s_ok != 0;
-}
-
 // ---------------------------------------------------------------------------
 // Rowwise: thread (rsub = t/16, ch = t%16) handles the 8 elements at columns
 // 8*ch.. of rows rsub + 16*i, i = 0..7; four consecutive lanes form a 32-block.

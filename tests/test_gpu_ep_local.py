@@ -1,6 +1,7 @@
 """The expert-parallel exchange on one GPU with NCCL (one rank): a forward MoE
-layer routed through dispatch / give_back equals the purely local path (plan,
-permute-quantise, grouped GEMM, combine) bit for bit.  Run in a subprocess
+layer routed through dispatch (plan, MXFP8 pack, all-to-all), receive (plan,
+unpack) and give_back equals the purely local path (plan, permute-quantise,
+grouped GEMM, combine) bit for bit.  Run in a subprocess
 with a deadline so that a stuck process group cannot stall the suite."""
 import os
 import socket
@@ -31,23 +32,19 @@ try:
     wq, ws = mx.mxfp8_quantize_rowwise(wl.normal_bf16((E * N, K), 0.05, 7).cuda())
     work = mx.new_workspace(E, T * k, N, K)
 
-    def layer(rows, ids):
-        offs, perm, inv, pw = mx.mxfp8_moe_plan(ids, E)
-        q, s, _, _ = mx.mxfp8_permute_quantize_dual(rows, perm, offs)
-        y = mx.mxfp8_grouped_gemm_fwd(q, s, wq, ws, offs, N, work=work)
-        assert mx.mxfp8_get_status(work) == 0 and mx.mxfp8_get_status(pw) == 0
-        return y, inv
-
-    y_grouped, inv = layer(x, idx)                     # local path
+    offs, perm, inv, pw = mx.mxfp8_moe_plan(idx, E)         # local path
+    q, s, _, _ = mx.mxfp8_permute_quantize_dual(x, perm, offs)
+    y_grouped = mx.mxfp8_grouped_gemm_fwd(q, s, wq, ws, offs, N, work=work)
+    assert mx.mxfp8_get_status(work) == 0 and mx.mxfp8_get_status(pw) == 0
     y_a = mx.mxfp8_moe_combine(y_grouped, inv, w)
 
-    rows, le, ex = ep.dispatch(x, idx, E)              # through the exchange
-    y_grouped_b, inv_b = layer(rows, le.view(-1, 1))
-    ones = torch.ones((rows.shape[0], 1), dtype=torch.float32, device="cuda")
-    y_rows = mx.mxfp8_moe_combine(y_grouped_b, inv_b, ones)
-    y_pairs = ep.give_back(y_rows, ex)
-    pairs = torch.arange(T * k, dtype=torch.int32, device="cuda").view(T, k)
-    y_b = mx.mxfp8_moe_combine(y_pairs, pairs, w)
+    d = ep.dispatch(x, idx, E)                               # through the exchange: MXFP8 records
+    assert d.records.dtype == torch.uint8 and d.records.shape[1] == mx.mxfp8_ep_record_bytes(K)
+    offs_b, perm_b, inv_b, q_b, s_b = ep.receive(d, E)
+    assert torch.equal(offs_b, offs) and torch.equal(q_b, q)
+    y_grouped_b = mx.mxfp8_grouped_gemm_fwd(q_b, s_b, wq, ws, offs_b, N, work=work)
+    y_back = ep.give_back(y_grouped_b, inv_b, d)
+    y_b = mx.mxfp8_moe_combine(y_back, d.ret_pos, w)
     torch.cuda.synchronize()
     assert torch.equal(y_a.view(torch.int16), y_b.view(torch.int16)), "exchange path differs"
     print("ok")
