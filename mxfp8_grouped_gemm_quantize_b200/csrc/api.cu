@@ -437,8 +437,9 @@ int64_t mxfp8_ep_record_bytes(int64_t cols) {
 
 int64_t mxfp8_ep_plan_workspace_bytes(int64_t num_tokens, int32_t num_ranks) {
   if (num_tokens < 0 || num_ranks < 1 || num_ranks > MXF8_EP_MAX_RANKS) return 0;
-  // status word | first record of each rank | per-chunk counts (records, pairs per rank)
-  return kWorkspaceBytes + MXF8_EP_MAX_RANKS * 4 + round_up(mxf8::ep_plan_chunks(num_tokens) * 2 * num_ranks * 4, 256);
+  // status word | first record and first pair of each rank | per-chunk counts (records, pairs per rank)
+  return kWorkspaceBytes + 2 * MXF8_EP_MAX_RANKS * 4 +
+         round_up(mxf8::ep_plan_chunks(num_tokens) * 2 * num_ranks * 4, 256);
 }
 
 mxf8_status mxfp8_ep_plan(const int32_t* idx, int64_t num_tokens, int32_t top_k, int32_t num_experts,
@@ -457,12 +458,12 @@ mxf8_status mxfp8_ep_plan(const int32_t* idx, int64_t num_tokens, int32_t top_k,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(work);
   int32_t* status = reinterpret_cast<int32_t*>(w);
-  int32_t* rec_base = reinterpret_cast<int32_t*>(w + kWorkspaceBytes);
-  int32_t* hist = reinterpret_cast<int32_t*>(w + kWorkspaceBytes + MXF8_EP_MAX_RANKS * 4);
+  int32_t* bases = reinterpret_cast<int32_t*>(w + kWorkspaceBytes);
+  int32_t* hist = reinterpret_cast<int32_t*>(w + kWorkspaceBytes + 2 * MXF8_EP_MAX_RANKS * 4);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   e = mxf8::launch_ep_plan(idx, num_tokens, top_k, num_experts, num_ranks, counts, rec_token, pair_expert, pair_rec,
-                           ret_pos, status, rec_base, hist, st);
+                           ret_pos, status, bases, hist, st);
   return e == cudaSuccess ? MXF8_OK : cuda_fail(e, "ep_plan launch");
 }
 

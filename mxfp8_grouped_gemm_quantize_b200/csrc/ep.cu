@@ -14,11 +14,12 @@
 // pair entry (local expert id, record index within the records sent to that
 // rank).  Send order: destination rank, token, slot, all ascending.
 //
-// Plan (three launches, no host round trip): (1) one thread per chunk of 32
-// tokens counts its records and pairs per destination; (2) one CTA turns the
-// counts into per-chunk start positions (an exclusive scan over chunks, then
-// over ranks); (3) every chunk thread walks its tokens again and places its
-// records, pairs and return positions.
+// Plan (three launches, no host round trip): (1) one warp per chunk of 32
+// tokens (a lane per token) counts the chunk's records and pairs per
+// destination with ballots and warp sums; (2) one CTA turns the counts into
+// per-chunk start positions (warp scans over chunks, then over ranks); (3)
+// every chunk warp places its records, pairs and return positions, lane
+// order giving token order.
 // Pack: one thread per 32-element block of a record encodes it with the same
 // block rule as the rowwise quantiser.  Unpack: one CTA per 128-row x
 // 128-column tile of the receiver's grouped rows, like the rowwise quantiser,
@@ -35,119 +36,134 @@
 namespace mxf8 {
 namespace {
 
-constexpr int kEpChunk = 32;   // tokens walked by one plan thread
+constexpr int kEpChunk = 32;   // tokens of one plan warp (one per lane)
 constexpr int kPlanThreads = 128;
+constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ int32_t owner_of(int32_t e, int32_t E, int32_t epr) {
   return (e >= 0 && e < E) ? e / epr : -1;
 }
 
-// Pass 1.  hist[c][p]: records chunk c sends to rank p; hist[c][P + p]: pairs.
+__device__ __forceinline__ int32_t warp_incl_sum(int32_t v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int32_t n = __shfl_up_sync(kFull, v, d);
+    if (lane >= d) v += n;
+  }
+  return v;
+}
+
+// Loads a lane's token's expert ids and owners (a lane past T has none).
+__device__ __forceinline__ bool load_slots(const int32_t* __restrict__ idx, int64_t t, int64_t T, int32_t k,
+                                           int32_t E, int32_t epr, int32_t (&eid)[MXF8_EP_MAX_TOP_K],
+                                           int32_t (&own)[MXF8_EP_MAX_TOP_K]) {
+  bool bad = false;
+  for (int32_t j = 0; j < k; ++j) {
+    const int32_t e = t < T ? __ldg(idx + t * k + j) : -1;
+    eid[j] = e;
+    own[j] = t < T ? owner_of(e, E, epr) : -1;
+    bad = bad || (t < T && own[j] < 0);
+  }
+  return bad;
+}
+
+// Pass 1 (one warp per chunk of 32 tokens).  hist[p][c]: records chunk c
+// sends to rank p; hist[P + p][c]: pairs.
 __global__ void __launch_bounds__(kPlanThreads) ep_count_kernel(const int32_t* __restrict__ idx, int64_t T,
                                                                  int32_t k, int32_t E, int32_t P,
-                                                                 int32_t* __restrict__ hist,
+                                                                 int32_t* __restrict__ hist, int64_t chunks,
                                                                  int32_t* __restrict__ status) {
-  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t chunks = (T + kEpChunk - 1) / kEpChunk;
-  if (c >= chunks) return;
-  int32_t* h = hist + c * 2 * P;
-  for (int32_t p = 0; p < 2 * P; ++p) h[p] = 0;
-  const int32_t epr = E / P;
-  const int64_t t1 = min(T, (c + 1) * kEpChunk);
-  bool bad = false;
-  int32_t own[MXF8_EP_MAX_TOP_K];
-  for (int64_t t = c * kEpChunk; t < t1; ++t) {
-    for (int32_t j = 0; j < k; ++j) {
-      const int32_t p = owner_of(__ldg(idx + t * k + j), E, epr);
-      own[j] = p;
-      if (p < 0) {
-        bad = true;
-        continue;
-      }
-      bool first = true;
-      for (int32_t jj = 0; jj < j; ++jj) first = first && own[jj] != p;
-      h[p] += first ? 1 : 0;
-      h[P + p] += 1;
+  const int64_t c = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (c >= chunks) return;   // whole warps only
+  int32_t eid[MXF8_EP_MAX_TOP_K], own[MXF8_EP_MAX_TOP_K];
+  if (load_slots(idx, c * kEpChunk + lane, T, k, E, E / P, eid, own))
+    atomicCAS(status, 0, static_cast<int32_t>(MXF8_ERR_BAD_ROUTING));
+  for (int32_t p = 0; p < P; ++p) {
+    int32_t n = 0;
+    for (int32_t j = 0; j < k; ++j) n += own[j] == p ? 1 : 0;
+    const unsigned bal = __ballot_sync(kFull, n > 0);
+    const int32_t tot = bal ? __reduce_add_sync(kFull, n) : 0;
+    if (lane == 0) {
+      hist[static_cast<int64_t>(p) * chunks + c] = __popc(bal);
+      hist[static_cast<int64_t>(P + p) * chunks + c] = tot;
     }
   }
-  if (bad) atomicCAS(status, 0, static_cast<int32_t>(MXF8_ERR_BAD_ROUTING));
 }
 
-// Pass 2 (one CTA of MXF8_EP_MAX_RANKS threads): hist entries become the
-// first record / pair position of each chunk for each rank; counts and the
-// first record of each rank (rec_base) are written.
-__global__ void __launch_bounds__(MXF8_EP_MAX_RANKS) ep_scan_kernel(int32_t* __restrict__ hist, int64_t chunks,
-                                                                    int32_t P, int32_t* __restrict__ counts,
-                                                                    int32_t* __restrict__ rec_base) {
-  __shared__ int32_t tr[MXF8_EP_MAX_RANKS], tp[MXF8_EP_MAX_RANKS];
-  const int p = threadIdx.x;
-  int32_t nr = 0, np = 0;
-  if (p < P) {
-    for (int64_t c = 0; c < chunks; ++c) {
-      int32_t* h = hist + c * 2 * P;
-      const int32_t a = h[p], b = h[P + p];
-      h[p] = nr;
-      h[P + p] = np;
-      nr += a;
-      np += b;
+// Pass 2 (one CTA): every hist row becomes its exclusive prefix over chunks
+// (one warp per row); bases[p] = first record of rank p, bases[MAX + p] =
+// its first pair; counts as documented.
+__global__ void __launch_bounds__(1024) ep_scan_kernel(int32_t* __restrict__ hist, int64_t chunks, int32_t P,
+                                                      int32_t* __restrict__ counts, int32_t* __restrict__ bases) {
+  __shared__ int32_t tot[2 * MXF8_EP_MAX_RANKS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int row = warp; row < 2 * P; row += 32) {
+    int32_t* h = hist + static_cast<int64_t>(row) * chunks;
+    int32_t carry = 0;
+    for (int64_t c0 = 0; c0 < chunks; c0 += 32) {
+      const int64_t c = c0 + lane;
+      const int32_t v = c < chunks ? h[c] : 0;
+      const int32_t incl = warp_incl_sum(v);
+      if (c < chunks) h[c] = carry + incl - v;
+      carry += __shfl_sync(kFull, incl, 31);
     }
+    if (lane == 0) tot[row] = carry;
   }
-  tr[p] = p < P ? nr : 0;
-  tp[p] = p < P ? np : 0;
   __syncthreads();
-  for (int d = 1; d < MXF8_EP_MAX_RANKS; d <<= 1) {   // inclusive scans over ranks
-    const int32_t a = p >= d ? tr[p - d] : 0, b = p >= d ? tp[p - d] : 0;
-    __syncthreads();
-    tr[p] += a;
-    tp[p] += b;
-    __syncthreads();
-  }
-  if (p < P) {
-    const int32_t r0 = p > 0 ? tr[p - 1] : 0, s0 = p > 0 ? tp[p - 1] : 0;
-    counts[p] = nr;
-    counts[P + p] = np;
-    rec_base[p] = r0;
-    for (int64_t c = 0; c < chunks; ++c) {
-      int32_t* h = hist + c * 2 * P;
-      h[p] += r0;
-      h[P + p] += s0;
+  if (warp < 2) {   // warp 0: records, warp 1: pairs -- exclusive scans over ranks
+    int32_t carry = 0;
+    for (int p0 = 0; p0 < P; p0 += 32) {
+      const int p = p0 + lane;
+      const int32_t v = p < P ? tot[warp * P + p] : 0;
+      const int32_t incl = warp_incl_sum(v);
+      if (p < P) {
+        bases[warp * MXF8_EP_MAX_RANKS + p] = carry + incl - v;
+        counts[warp * P + p] = v;
+      }
+      carry += __shfl_sync(kFull, incl, 31);
     }
   }
 }
 
-// Pass 3: placement, in token and slot order within each chunk.
+// Pass 3 (one warp per chunk): placement.  Lane L's record for rank p comes
+// after the chunk's records of lanes < L for p; its pairs for p after theirs,
+// in slot order.
 __global__ void __launch_bounds__(kPlanThreads) ep_place_kernel(
-    const int32_t* __restrict__ idx, int64_t T, int32_t k, int32_t E, int32_t P, int32_t* __restrict__ hist,
-    const int32_t* __restrict__ rec_base, int32_t* __restrict__ rec_token, int32_t* __restrict__ pair_expert,
-    int32_t* __restrict__ pair_rec, int32_t* __restrict__ ret_pos) {
-  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t chunks = (T + kEpChunk - 1) / kEpChunk;
+    const int32_t* __restrict__ idx, int64_t T, int32_t k, int32_t E, int32_t P, const int32_t* __restrict__ hist,
+    int64_t chunks, const int32_t* __restrict__ bases, int32_t* __restrict__ rec_token,
+    int32_t* __restrict__ pair_expert, int32_t* __restrict__ pair_rec, int32_t* __restrict__ ret_pos) {
+  const int64_t c = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
   if (c >= chunks) return;
-  int32_t* h = hist + c * 2 * P;
   const int32_t epr = E / P;
-  const int64_t t1 = min(T, (c + 1) * kEpChunk);
-  int32_t own[MXF8_EP_MAX_TOP_K], rec[MXF8_EP_MAX_TOP_K];
-  for (int64_t t = c * kEpChunk; t < t1; ++t) {
-    for (int32_t j = 0; j < k; ++j) {
-      const int32_t e = __ldg(idx + t * k + j);
-      const int32_t p = owner_of(e, E, epr);
-      own[j] = p;
-      if (p < 0) {
-        ret_pos[t * k + j] = -1;
-        continue;
+  const int64_t t = c * kEpChunk + lane;
+  int32_t eid[MXF8_EP_MAX_TOP_K], own[MXF8_EP_MAX_TOP_K];
+  load_slots(idx, t, T, k, E, epr, eid, own);
+  if (t < T)
+    for (int32_t j = 0; j < k; ++j)
+      if (own[j] < 0) ret_pos[t * k + j] = -1;
+  const unsigned below = (1u << lane) - 1u;
+  for (int32_t p = 0; p < P; ++p) {
+    int32_t n = 0;
+    for (int32_t j = 0; j < k; ++j) n += own[j] == p ? 1 : 0;
+    const unsigned bal = __ballot_sync(kFull, n > 0);
+    if (bal == 0) continue;   // uniform across the warp
+    const int32_t excl = warp_incl_sum(n) - n;
+    if (n > 0) {
+      const int32_t rb = __ldg(bases + p);
+      const int32_t ri = rb + __ldg(hist + static_cast<int64_t>(p) * chunks + c) + __popc(bal & below);
+      rec_token[ri] = static_cast<int32_t>(t);
+      int32_t s = __ldg(bases + MXF8_EP_MAX_RANKS + p) + __ldg(hist + static_cast<int64_t>(P + p) * chunks + c) +
+                  excl;
+      for (int32_t j = 0; j < k; ++j) {
+        if (own[j] != p) continue;
+        pair_expert[s] = eid[j] - p * epr;
+        pair_rec[s] = ri - rb;
+        ret_pos[t * k + j] = s;
+        ++s;
       }
-      int32_t ri = -1;
-      for (int32_t jj = 0; jj < j; ++jj)
-        if (ri < 0 && own[jj] == p) ri = rec[jj];
-      if (ri < 0) {
-        ri = h[p]++;
-        rec_token[ri] = static_cast<int32_t>(t);
-      }
-      rec[j] = ri;
-      const int32_t s = h[P + p]++;
-      pair_expert[s] = e - p * epr;
-      pair_rec[s] = ri - __ldg(rec_base + p);
-      ret_pos[t * k + j] = s;
     }
   }
 }
@@ -272,18 +288,19 @@ int64_t ep_plan_chunks(int64_t T) { return (T + kEpChunk - 1) / kEpChunk; }
 
 cudaError_t launch_ep_plan(const int32_t* idx, int64_t T, int32_t k, int32_t E, int32_t P, int32_t* counts,
                            int32_t* rec_token, int32_t* pair_expert, int32_t* pair_rec, int32_t* ret_pos,
-                           int32_t* status, int32_t* rec_base, int32_t* hist, cudaStream_t stream) {
+                           int32_t* status, int32_t* bases, int32_t* hist, cudaStream_t stream) {
   const int64_t chunks = ep_plan_chunks(T);
-  const unsigned blocks = static_cast<unsigned>((chunks + kPlanThreads - 1) / kPlanThreads);
+  const int64_t warps_per_cta = kPlanThreads / 32;
+  const unsigned blocks = static_cast<unsigned>((chunks + warps_per_cta - 1) / warps_per_cta);
   if (chunks > 0) {
-    ep_count_kernel<<<blocks, kPlanThreads, 0, stream>>>(idx, T, k, E, P, hist, status);
+    ep_count_kernel<<<blocks, kPlanThreads, 0, stream>>>(idx, T, k, E, P, hist, chunks, status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  ep_scan_kernel<<<1, MXF8_EP_MAX_RANKS, 0, stream>>>(hist, chunks, P, counts, rec_base);
+  ep_scan_kernel<<<1, 1024, 0, stream>>>(hist, chunks, P, counts, bases);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || chunks == 0) return e;
-  ep_place_kernel<<<blocks, kPlanThreads, 0, stream>>>(idx, T, k, E, P, hist, rec_base, rec_token, pair_expert,
+  ep_place_kernel<<<blocks, kPlanThreads, 0, stream>>>(idx, T, k, E, P, hist, chunks, bases, rec_token, pair_expert,
                                                       pair_rec, ret_pos);
   return cudaGetLastError();
 }

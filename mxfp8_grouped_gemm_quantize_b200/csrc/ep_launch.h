@@ -11,7 +11,7 @@ int64_t ep_plan_chunks(int64_t T);
 int64_t ep_record_stride(int64_t C);
 cudaError_t launch_ep_plan(const int32_t* idx, int64_t T, int32_t k, int32_t E, int32_t P, int32_t* counts,
                            int32_t* rec_token, int32_t* pair_expert, int32_t* pair_rec, int32_t* ret_pos,
-                           int32_t* status, int32_t* rec_base, int32_t* hist, cudaStream_t stream);
+                           int32_t* status, int32_t* bases, int32_t* hist, cudaStream_t stream);
 cudaError_t launch_ep_pack(const uint16_t* x, int64_t T, int64_t C, const int32_t* rec_token, int64_t R,
                            uint8_t* records, cudaStream_t stream);
 cudaError_t launch_ep_unpack(const uint8_t* records, int64_t R, int64_t C, const int32_t* pair_rec,
