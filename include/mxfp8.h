@@ -288,10 +288,11 @@ MXF8_API mxf8_status mxfp8_grouped_gemm_fwd_noalloc(const uint8_t* xq, const uin
 MXF8_API mxf8_status mxfp8_set_gemm_tiling(int32_t cta_pair, int32_t stage_k);
 
 /* Test switch for the bounded pipeline waits: while enabled (enable != 0),
- * every grouped GEMM launch leaves its first pipeline stage unfilled, so the
- * MMA warp's wait on it runs out after the 2 s limit; the kernel drains what
- * it issued, frees tensor memory and returns with MXF8_ERR_TIMEOUT in the
- * workspace status.  Off by default; meant only for tests of that path. */
+ * every grouped GEMM launch (1-CTA tiles and CTA pairs alike) leaves its
+ * first pipeline stage unfilled, so the wait on it runs out after the 2 s
+ * limit; the kernel drains what it issued, frees tensor memory and returns
+ * with MXF8_ERR_TIMEOUT in the workspace status.  Off by default; meant only
+ * for tests of that path. */
 MXF8_API void mxfp8_testing_stall_first_stage(int32_t enable);
 
 /* ---------------------------------------------------------------- MoE dispatch / combine */

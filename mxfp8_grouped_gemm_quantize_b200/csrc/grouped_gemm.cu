@@ -61,7 +61,7 @@ constexpr int round_up_c(int a, int b) { return (a + b - 1) / b * b; }
 
 // Pipeline shape: CG CTAs per MMA, KS 128-wide K blocks per stage.  The ring
 // takes as many stages as shared memory holds: 1 CTA: 4 x 128-deep or
-// 2 x 256-deep; pair: 5 x 128-deep or 3 x 256-deep.  Deeper stages amortise
+// 2 x 256-deep; pair: 6 x 128-deep or 3 x 256-deep.  Deeper stages amortise
 // the fixed cost of a stage hand-off (barrier round trip, copy issue) over
 // twice the MMAs.
 // FP4 (NVFP4 operands): a 128-byte K block holds 256 elements = four MMAs of
@@ -126,7 +126,7 @@ struct Params {
   int64_t out_ld;                      // output row stride (elements)
   int32_t* status;
   uint64_t timeout_ns;
-  int32_t inject_skip_stage;           // test hook: the producer leaves stage 0 unfilled (1-CTA only)
+  int32_t inject_skip_stage;           // test hook: the producers leave stage 0 unfilled
   // Quantising epilogue (fwd/dgrad): MXFP8 copies of the bf16 output, in the
   // quantisers' layouts with the GEMM's groups.  Null pointers skip a layout.
   uint8_t* qr;                         // rowwise codes [M, out_ld]
@@ -437,9 +437,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       uint32_t it = 0, s = 0, ph = 0;
       int32_t eh = 0;
       bool failed = false;
-      // Test hook: stage 0 gets neither its copies nor its arrival, so the MMA
-      // warp's bounded wait on it runs out; the drain below skips it.
-      const bool skip0 = CG == 1 && p.inject_skip_stage != 0;
+      // Test hook: stage 0 gets neither its copies nor its arrival (in both
+      // CTAs of a pair), so the MMA warp's bounded wait on it runs out; the
+      // drain below skips it.
+      const bool skip0 = p.inject_skip_stage != 0;
       for (int32_t t = unit0; t < total && !failed; t += nunits) {
         eh = advance_group(sc, p.E, t, eh);
         const Tile tl = decode_tile<CG, FP4, SG>(p, sc, t, eh, rank);
