@@ -86,6 +86,15 @@ def gemm_sources_sha256() -> str:
     return h.hexdigest()
 
 
+def step_peak(pk, timed_ms: float):
+    """FP8 peak for kernels timed inside the step: the sustained figure once the
+    timed region is a seconds-long loop (>= 0.5 s, where the power cap sets in),
+    else the burst figure.  Returns (TFLOP/s, 'sustained' | 'burst')."""
+    if timed_ms >= 500.0 and pk.get("bf16_sust"):
+        return pk["bf16_sust"] * FP8_OVER_BF16, "sustained"
+    return pk["bf16"] * FP8_OVER_BF16, "burst"
+
+
 def gemm_traffic():
     """(bytes per GEMM launch, workload it was captured on), or (None, None)
     when no capture exists for the current kernel sources."""
@@ -347,7 +356,8 @@ def run_ours(args, rank, world, local_rank):
     value = whole_job_tflops(step_flops, ms_step, world)
 
     pk = peaks()
-    fp8_peak = pk["bf16"] * FP8_OVER_BF16
+    fp8_peak = pk["bf16"] * FP8_OVER_BF16              # burst: kernels timed alone
+    in_step_peak, peak_kind = step_peak(pk, ms_total)  # kernels timed inside the step loop
     traffic, traffic_wl = gemm_traffic()
     gemm_ms = sum(sum(v) for k, v in per_kind.items() if k.startswith("gemm")) / K
     gemm_launches = sum(len(v) for k, v in per_kind.items() if k.startswith("gemm"))
@@ -365,14 +375,16 @@ def run_ours(args, rank, world, local_rank):
         "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)", "data": "synthetic",
         "config": workload_config(w, args.quantiser, world),
-        "fraction_of_fp8_peak": round(value / world / fp8_peak, 4),
+        "fraction_of_fp8_peak": round(value / world / in_step_peak, 4),
         "roofline": {"kernel": "grouped_gemm_kernel (fwd+dgrad+wgrad launches)", "bound": "tensor",
-                     "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(gemm_tflops / fp8_peak, 4), "traffic": traffic,
+                     "achieved": round(gemm_tflops, 1), "peak": round(in_step_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(gemm_tflops / in_step_peak, 4),
+                     "frac_of_burst_peak": round(gemm_tflops / fp8_peak, 4), "traffic": traffic,
                      "traffic_source": (f"ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, mean over the "
                                         f"fwd, dgrad and wgrad launches of {traffic_wl}" if traffic is not None else
                                         "no ncu capture of the current kernel sources"),
-                     "peak_source": f"{pk['src']} bf16 burst x {FP8_OVER_BF16} (nominal FP8/BF16)",
+                     "peak_source": (f"{pk['src']} bf16 {peak_kind} x {FP8_OVER_BF16} (nominal FP8/BF16); "
+                                     f"timed region {ms_total:.0f} ms"),
                      "launches_timed": gemm_launches},
         "quantiser": {"achieved_gbs": round(quant_gbs, 1), "peak_gbs": pk["hbm_gbs"],
                       "frac": round(quant_gbs / pk["hbm_gbs"], 4), "ms_per_step": round(quant_ms, 4)},

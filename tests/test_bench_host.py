@@ -105,3 +105,10 @@ def test_the_headline_is_the_671b_like_layer():
     assert c["workload"] == "ds-v3-671b-like MoE layer" and c["routed_rows"] == 16384 and c["experts"] == 32
     assert c["layers"] == [{"name": "gate_up", "N": 4096, "K": 7168}, {"name": "down", "N": 7168, "K": 2048}]
     assert "Zipf" in c["routing"]
+
+
+def test_in_step_kernels_are_held_to_the_sustained_peak_in_long_runs():
+    pk = {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sust": 1400.0, "src": "fallback"}
+    assert bench.step_peak(pk, 1300.0) == (2800.0, "sustained")
+    assert bench.step_peak(pk, 80.0) == (3180.0, "burst")
+    assert bench.step_peak(dict(pk, bf16_sust=None), 1300.0) == (3180.0, "burst")
