@@ -187,7 +187,7 @@ def test_distinct_block_scales_pin_the_scale_layout(mx, tile_config):
 
 @pytest.mark.parametrize("counts,N,K", [([1], 128, 32), ([0, 0, 5], 128, 64), ([300], 128, 160),
                                         ([3, 0, 0, 0], 256, 1024), ([129, 127], 512, 96),
-                                        ([40, 0, 260], 384, 544)])
+                                        ([40, 0, 260], 384, 544), ([256, 512, 3], 256, 128)])
 def test_edge_shapes(mx, tile_config, counts, N, K):
     run_all_and_compare(make_case(mx, counts, N, K, seed=sum(counts)))
 
