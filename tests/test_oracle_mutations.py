@@ -220,3 +220,58 @@ def test_nvfp4_restatement_passes_and_mutants_fail_the_golden_blocks():
     assert not _nvfp4_golden_ok(lambda v, S: _nvfp4_block(v, S, div=4.0))           # wrong E2M1 max in sf
     assert not _nvfp4_golden_ok(lambda v, S: _nvfp4_block(v, S, tie_even=False))    # ties away from zero
     assert not _nvfp4_golden_ok(lambda v, S: _nvfp4_block(v, 1.0))                  # tensor scale ignored
+
+
+# ---------------------------------------------------------------- expert-parallel dispatch plan
+def _ep_plan_restated(idx, E, P, owner=None, dedup=True, rec_relative=True, slot_major=False):
+    """A loop restatement of the EP send plan with optional planted mistakes:
+    owner(e) other than e // (E/P), one record per pair instead of per
+    (token, rank), record indices counted from the start of the send buffer
+    instead of the destination's first record, or pairs ordered slot-major."""
+    T, k = idx.shape
+    epr = E // P
+    owner = owner or (lambda e: e // epr)
+    counts = [0] * (2 * P)
+    rec_token, pair_expert, pair_rec = [], [], []
+    ret = -np.ones((T, k), dtype=np.int64)
+    for p in range(P):
+        rec0 = len(rec_token)
+        order = [(t, j) for j in range(k) for t in range(T)] if slot_major else \
+                [(t, j) for t in range(T) for j in range(k)]
+        mine = {}
+        for t, j in order:
+            e = int(idx[t, j])
+            if not (0 <= e < E) or owner(e) != p:
+                continue
+            if t not in mine or not dedup:
+                mine[t] = len(rec_token) - (rec0 if rec_relative else 0)
+                rec_token.append(t)
+            ret[t, j] = len(pair_expert)
+            pair_expert.append(e % epr)
+            pair_rec.append(mine[t])
+        counts[p] = len(rec_token) - rec0
+        counts[P + p] = sum(1 for t, j in order if 0 <= int(idx[t, j]) < E and owner(int(idx[t, j])) == p)
+    return counts, rec_token, pair_expert, pair_rec, ret
+
+
+def _ep_plan_agrees(plan, idx, E, P):
+    from tests.test_oracle_ep import brute_plan
+    counts, rec_token, pe, prc, ret = brute_plan(idx, E, P)
+    c2, rt2, pe2, prc2, ret2 = plan
+    return counts == c2 and rec_token == rt2 and pe == pe2 and prc == prc2 and np.array_equal(ret, ret2)
+
+
+@pytest.mark.parametrize("name,kw", [("owner by modulo", {"owner": "mod"}), ("no dedup", {"dedup": False}),
+                                     ("absolute record index", {"rec_relative": False}),
+                                     ("slot-major order", {"slot_major": True})])
+def test_ep_plan_mutants_fail_the_brute_force_pin(name, kw):
+    E, P = 12, 3
+    idx = np.array([[0, 1, 5], [11, 4, 3], [7, 8, 2], [6, 9, 10], [1, 0, 4]], dtype=np.int32)
+    # the restatement without mistakes and the oracle agree with the pin
+    assert _ep_plan_agrees(_ep_plan_restated(idx, E, P), idx, E, P)
+    pl = oracle.ep_plan(idx, E, P)
+    assert _ep_plan_agrees((pl.counts.tolist(), pl.rec_token.tolist(), pl.pair_expert.tolist(),
+                            pl.pair_rec.tolist(), pl.ret_pos), idx, E, P)
+    if kw.get("owner") == "mod":
+        kw = {"owner": lambda e: e % P}
+    assert not _ep_plan_agrees(_ep_plan_restated(idx, E, P, **kw), idx, E, P), name
