@@ -254,3 +254,20 @@ def test_workload_full_size_sampled(mx, name):
     for layer in w.layers:
         X, W, dY = wl.layer_tensors(w, layer)
         _sampled_check(Case(mx, X, W, dY, w.offsets, check_quant=False), rng)
+
+
+def test_the_largest_group_count(mx, tile_config):
+    """MXF8_GEMM_MAX_GROUPS experts, most of them empty or tiny: the on-device
+    schedule's prefix runs over eight warps' worth of groups and the wgrad
+    longest-first ranking over all of them (ties between equal counts)."""
+    rng = np.random.default_rng(256)
+    counts = rng.choice([0, 0, 1, 3, 17, 40, 129, 260], size=mx.MXF8_GEMM_MAX_GROUPS).tolist()
+    run_all_and_compare(make_case(mx, counts, 128, 96, seed=256))
+
+
+def test_more_groups_than_the_limit_are_rejected(mx):
+    E = mx.MXF8_GEMM_MAX_GROUPS + 1
+    c = make_case(mx, [1] * 4, 128, 64, check_quant=False)
+    od = torch.arange(E + 1, dtype=torch.int32, device="cuda").clamp(max=4)
+    with pytest.raises(mx.MXFP8Error):
+        mx.mxfp8_grouped_gemm_fwd(c.xq, c.xs, c.wq, c.ws, od, 128, work=mx.new_workspace(E, 4, 128, 64))
