@@ -80,3 +80,39 @@ def test_missing_library_is_an_error(monkeypatch, tmp_path):
     monkeypatch.setattr(mx, "LIB_PATH", str(tmp_path / "libmxfp8.so"))
     with pytest.raises(RuntimeError, match="missing"):
         mx.lib()
+
+
+@pytest.mark.parametrize("C", [32, 64, 96, 1408, 2048, 7168])
+def test_ep_record_size_agrees_with_the_format(lib, C):
+    import mxfp8_grouped_gemm_quantize_b200 as m
+    assert m.mxfp8_ep_record_bytes(C) == oracle.ep_record_bytes(C)
+    assert m.mxfp8_ep_record_bytes(C) % 16 == 0 and m.mxfp8_ep_record_bytes(C) >= C + C // 32
+    assert lib.mxfp8_ep_record_bytes(0) == 0 and lib.mxfp8_ep_record_bytes(48) == 0   # cols % 32 != 0
+
+
+def test_ep_plan_workspace_grows_with_tokens_and_ranks(lib):
+    w = lib.mxfp8_ep_plan_workspace_bytes
+    assert w(0, 1) > 0 and w(0, 1) % 16 == 0
+    assert w(4096, 8) >= w(2048, 8) >= w(2048, 2)
+    assert w(10, 0) == 0 and w(10, 257) == 0 and w(-1, 2) == 0
+
+
+def test_tiling_switch_accepts_the_documented_values_only(lib):
+    try:
+        for cta_pair in (-1, 0, 1):
+            for stage_k in (-1, 1, 2):
+                assert lib.mxfp8_set_gemm_tiling(cta_pair, stage_k) == 0
+        for bad in ((2, -1), (-2, -1), (0, 0), (0, 3), (1, -2)):
+            assert lib.mxfp8_set_gemm_tiling(*bad) == 1   # MXF8_ERR_INVALID_ARG
+    finally:
+        lib.mxfp8_set_gemm_tiling(-1, -1)
+
+
+def test_argument_errors_are_reported_before_any_device_call(lib):
+    """Host-side validation needs no GPU: invalid sizes and null pointers are
+    rejected with MXF8_ERR_INVALID_ARG before the library touches a device."""
+    assert lib.mxfp8_quantize_rowwise(None, 4, 48, None, 1, None, None, 0, None) == 1      # cols % 32
+    assert lib.mxfp8_moe_plan(None, 4, 0, 8, None, None, None, None, 0, None) == 1           # top_k < 1
+    assert lib.mxfp8_ep_plan(None, 4, 2, 5, 2, None, None, None, None, None, None, 0, None) == 1   # E % P
+    assert lib.mxfp8_ep_pack(None, 4, 48, None, 1, None, None) == 1                            # cols % 32
+    assert lib.mxfp8_gather_rows(None, 4, 24, None, 1, None, None) == 1                        # row bytes % 16
