@@ -17,7 +17,10 @@
 //     (cta_group::2).  Each CTA stages its own 128 rows of A, half of B's 256
 //     rows and all 256 rows of B's scales; the pair computes a 256x256 output
 //     tile, 128 rows in each CTA's tensor memory.  Per CTA this moves 2/3 of
-//     the operand bytes per FLOP of a 1-CTA 128x256 tile.
+//     the operand bytes per FLOP of a 1-CTA 128x256 tile.  In fwd/dgrad a
+//     group's ragged last tile (r < 256 rows) runs with the operand roles
+//     swapped: 256 B rows x round_up(r, 32) tokens, so pairs pad a group to
+//     32 rows rather than 256.
 //   CG = 1: 128x256x32 MMAs (cta_group::1), one CTA per tile.
 // Roles per CTA (192 threads): warp 0 TMA producer; warp 1 allocates the 512
 // tensor-memory columns, and (in the leader CTA) one thread copies scale
@@ -165,6 +168,9 @@ struct Tile {
   int32_t q_rb;          // fwd/dgrad: RB_e + row block, the output's rowwise scale atom row
                          //            and colwise scale atom column
   int32_t q_p;           // fwd/dgrad: P_e + 128 * row block, the output's colwise code column
+  bool swapped;          // CTA pairs, fwd/dgrad: a group's ragged last tile with the operand roles
+                         // swapped (A = the B operand's 256 rows, B = the group's last tokens)
+  int32_t ntok;          // swapped: MMA N = the tile's tokens rounded up to 32
 };
 
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
@@ -196,7 +202,17 @@ __device__ __forceinline__ int32_t advance_group(const Sched& s, int32_t E, int3
 // SG (SwiGLU, fwd only): output tile nt covers columns 128nt..128nt+127 of
 // h [M, N/2]; its B rows are gate rows e*N + 128nt.. and up rows
 // e*N + N/2 + 128nt.. (CTA pairs: rank 0 stages the gate rows, rank 1 the up rows).
-template <int CG, bool FP4 = false, bool SG = false>
+//
+// ST (CTA pairs, fwd/dgrad): a group whose row count is not a multiple of 256
+// ends in a tile of r < 256 rows.  Padded to 256 rows it would cost a whole
+// pair tile; instead the pair computes its transpose, Y_tail^T = W_half X_tail^T:
+// A = the 256 B-operand rows of the output-column block (each CTA stages its
+// 128, exactly as it would stage them as B), B = the tail's r tokens rounded
+// up to 32 (MMA N, each CTA staging half), with the scale maps exchanged the
+// same way.  The accumulator then holds output columns in its lanes and
+// tokens in its columns, and the epilogue writes it back transposed.  The
+// tensor work of the tile shrinks from 256 to round_up(r, 32) rows.
+template <int CG, bool FP4 = false, bool SG = false, bool ST = false>
 __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int32_t t, int32_t si, uint32_t rank) {
   // K blocks are 128 bytes of codes: 128 E4M3 or 256 E2M1 elements; MMA steps
   // take 32 (E4M3) or 64 (E2M1) elements.  TMA x coordinates count bytes.
@@ -260,6 +276,31 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int
   tl.sfa_atom = sfa_row * p.sfa_pitch + sfa_col;
   tl.sfb_atom0 = sfb_row * p.sfb_pitch + sfb_col;
   tl.sfb_atom1 = sfb_row1 * p.sfb_pitch + sfb_col;
+  tl.swapped = false;
+  tl.ntok = 0;
+  if constexpr (ST) {
+    const int32_t mp = local % munits;   // the pair's 256-row block
+    if (p.mode != kWgrad && mp == munits - 1 && (m & 255) != 0) {
+      const int32_t r = m - 256 * mp;
+      tl.swapped = true;
+      tl.ntok = (r + 31) & ~31;
+      // A slot <- this CTA's 128 B-operand rows (the B staging of a normal pair tile)
+      tl.a_x = tl.b_x;
+      tl.a_y = tl.b_y;
+      // B slot <- this CTA's half of the tail tokens (rows of the A operand)
+      tl.b_x = 0;
+      tl.b_y = row0 + 256 * mp + static_cast<int32_t>(rank) * (tl.ntok / 2);
+      // A scales: the atom of this CTA's B-operand half; B scales: the tail's two atom rows
+      tl.sfa_atom = (rank == 0 ? tl.sfb_atom0 : tl.sfb_atom1);
+      tl.sfb_atom0 = int64_t(s.rb[e] + 2 * mp) * p.sfa_pitch;
+      tl.sfb_atom1 = tl.sfb_atom0 + p.sfa_pitch;
+      tl.out_row = int64_t(row0) + 256 * mp;
+      tl.rows = r;
+      tl.out_col = int64_t(BN) * nt + 128 * static_cast<int32_t>(rank);
+      tl.cols = static_cast<int32_t>(min64(128, out_cols - tl.out_col));
+      if (tl.cols < 0) tl.cols = 0;
+    }
+  }
   return tl;
 }
 
@@ -371,6 +412,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const __grid_constant__ CUtensorMap tmOut, const Params p) {
   using C = Cfg<CG, KS, FP4>;
   constexpr int STAGES = C::STAGES;
+  constexpr bool ST = CG == 2 && !QE && !FP4 && !SG;   // swapped ragged last tiles (see decode_tile)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -443,7 +485,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const bool skip0 = p.inject_skip_stage != 0;
       for (int32_t t = unit0; t < total && !failed; t += nunits) {
         eh = advance_group(sc, p.E, t, eh);
-        const Tile tl = decode_tile<CG, FP4, SG>(p, sc, t, eh, rank);
+        const Tile tl = decode_tile<CG, FP4, SG, ST>(p, sc, t, eh, rank);
         for (int32_t kb0 = 0; kb0 < tl.kblocks; kb0 += C::KS) {
           if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, lim)) {
             record_error(p.status, MXF8_ERR_TIMEOUT, abort_flag);
@@ -477,8 +519,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const uint32_t sb = smem_addr(smem + C::OFF_B + q * C::B_TILE);
             const int32_t kx = BK * (kb0 + h);
             if constexpr (CG == 2) {
-              tma_load_2d_pair(sa, &tmA, tl.a_x + kx, tl.a_y, fb);
-              tma_load_2d_pair(sb, &tmB, tl.b_x + kx, tl.b_y, fb);
+              // a swapped tile stages the B operand's rows in the A slot and its
+              // tokens (a whole 128-row box, of which the MMA reads ntok / 2) in the B slot
+              tma_load_2d_pair(sa, tl.swapped ? &tmB : &tmA, tl.a_x + kx, tl.a_y, fb);
+              tma_load_2d_pair(sb, tl.swapped ? &tmA : &tmB, tl.b_x + kx, tl.b_y, fb);
             } else if constexpr (SG) {
               // gate rows, then the up rows N/2 further (two 128-row boxes)
               tma_load_2d(sa, &tmA, tl.a_x + kx, tl.a_y, fb);
@@ -490,9 +534,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
           }
           if constexpr (CG == 2) {
-            tma_load_2d_pair(ssa, &tmSFA, 0, ya, fb);
-            tma_load_2d_pair(ssb, &tmSFB, 0, yb0, fb);
-            tma_load_2d_pair(ssb + C::KS * C::APK * 512, &tmSFB, 0, yb1, fb);
+            const CUtensorMap* msa = tl.swapped ? &tmSFB : &tmSFA;
+            const CUtensorMap* msb = tl.swapped ? &tmSFA : &tmSFB;
+            tma_load_2d_pair(ssa, msa, 0, ya, fb);
+            tma_load_2d_pair(ssb, msb, 0, yb0, fb);
+            tma_load_2d_pair(ssb + C::KS * C::APK * 512, msb, 0, yb1, fb);
           } else {
             tma_load_2d(ssa, &tmSFA, 0, ya, fb);
             tma_load_2d(ssb, &tmSFB, 0, yb0, fb);
@@ -544,6 +590,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       bool failed = false;
       for (int32_t t = unit0; t < total && !failed; t += nunits) {
         int32_t kblocks = kb_fixed, ksteps_last = ks_fixed;
+        uint32_t idesc_t = idesc0;
+        if constexpr (ST) {
+          if (p.mode != kWgrad) {
+            // a group's ragged last pair tile runs swapped with N = its tokens rounded up to 32
+            eh = advance_group(sc, p.E, t, eh);
+            const int32_t e = sc.slot[eh];
+            const int32_t m = sc.off[e + 1] - sc.off[e];
+            const int32_t munits = group_m_units<CG>(p, m);
+            if ((t - sc.tile0[eh]) % munits == munits - 1 && (m & 255) != 0) {
+              const uint32_t ntok = static_cast<uint32_t>((m - 256 * (munits - 1) + 31) & ~31);
+              idesc_t = (idesc0 & ~(0x3Fu << 17)) | ((ntok >> 3) << 17);
+            }
+          }
+        }
         if (p.mode == kWgrad) {
           eh = advance_group(sc, p.E, t, eh);
           const int32_t e = sc.slot[eh];
@@ -608,7 +668,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             for (int k = 0; k < 4; ++k) {
               if (FULL || k < nk) {
                 // +2 per step: the start-address field counts 16-byte units, one step is 32 bytes of K
-                const uint32_t idesc = idesc0 | (uint32_t(k) << 4) | (uint32_t(k) << 29);
+                const uint32_t idesc = idesc_t | (uint32_t(k) << 4) | (uint32_t(k) << 29);
                 if constexpr (CG == 2)
                   tc_mma_mxf8_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, sfa_t | (uint32_t(k) << 30),
                                    sfb_t | (uint32_t(k) << 30), acc);
@@ -671,7 +731,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     for (int32_t t = unit0; t < total; t += nunits) {
       eh = advance_group(sc, p.E, t, eh);
-      const Tile tl = decode_tile<CG, FP4, SG>(p, sc, t, eh, rank);
+      const Tile tl = decode_tile<CG, FP4, SG, ST>(p, sc, t, eh, rank);
       const int32_t vr = max(0, min(32, tl.rows - row_base));       // valid rows of this warp's slice
       uint16_t* out_tile = p.out + tl.out_row * p.out_ld + tl.out_col;
       if (tl.kblocks == 0) {
@@ -811,6 +871,56 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           }
         }
       };
+      if constexpr (ST) {
+        if (tl.swapped) {
+          // Swapped tile: lane n of this warp's quarter is output column
+          // out_col + 32 * quarter + n, accumulator column i is token i.  Each
+          // 32-token chunk goes through the warp's stage as a [32 tokens][32
+          // columns] bf16 block, then out as 64-byte row segments (tokens past
+          // the group are not written).  Chunks shared with the other
+          // accumulator are drained first (buffer 0: the high ones, buffer 1:
+          // the low ones), then the accumulator is released.
+          const int nch = tl.ntok / 32;
+          const int ov_lo = buf == 0 ? static_cast<int>(C::ACC_STRIDE / 32) : 0;
+          const int ov_hi = buf == 0 ? 8 : static_cast<int>((256 - C::ACC_STRIDE) / 32);
+          const int n_ov = max(0, min(nch, ov_hi) - ov_lo);
+          if (n_ov == 0) release();
+          int done_ov = 0;
+          uint16_t* stg16 = reinterpret_cast<uint16_t*>(stage_base);
+          const uint4* stg4 = reinterpret_cast<const uint4*>(stage_base);
+          if (lane == 0) bulk_wait_read<0>();   // an earlier tile's TMA store has read the stage
+          __syncwarp();
+          const bool col_ok = tl.cols > 32 * static_cast<int32_t>(quarter);
+          uint16_t* out_q = p.out + tl.out_row * p.out_ld + tl.out_col + 32 * quarter;
+#pragma unroll 1
+          for (int i = 0; i < nch; ++i) {
+            const int jc = buf == 0 ? nch - 1 - i : i;
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tbase + 32 * jc, v);
+            tmem_wait_regs(v);
+            if (jc >= ov_lo && jc < ov_hi && ++done_ov == n_ov) release();
+            if (col_ok) {
+#pragma unroll
+              for (int k = 0; k < 16; ++k) {
+                const uint32_t pk = cvt_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                stg16[(2 * k) * 32 + lane] = static_cast<uint16_t>(pk & 0xFFFFu);
+                stg16[(2 * k + 1) * 32 + lane] = static_cast<uint16_t>(pk >> 16);
+              }
+              __syncwarp();
+#pragma unroll
+              for (int it = 0; it < 4; ++it) {
+                const int row = 8 * it + (lane >> 2), q = lane & 3;
+                const int32_t tok = 32 * jc + row;
+                if (tok < tl.rows)
+                  *reinterpret_cast<uint4*>(out_q + int64_t(tok) * p.out_ld + 8 * q) = stg4[row * 4 + q];
+              }
+              __syncwarp();
+            }
+          }
+          ++j;
+          continue;
+        }
+      }
       if constexpr (SG) {
         // SwiGLU: accumulator columns 0-127 hold the gate, 128-255 the up
         // projection of the same 128 output columns; output chunk cc pairs
@@ -961,18 +1071,22 @@ cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** detail) {
   // Tile configuration, from sizes the host knows (the group sizes stay on
-  // the device): fwd/dgrad over long contractions (>= 40 K blocks) of groups
-  // averaging >= 768 rows run CTA pairs with 256-deep stages -- pairs move
-  // 2/3 of the operand bytes per FLOP and their 256-row padding is then a
-  // small share; everything else runs 1-CTA 128x256 tiles with 128-deep
-  // stages (on B200 these won every other pass of the three MoE layers).
+  // the device).  Plain fwd/dgrad over long contractions (>= 32 K blocks) run
+  // CTA pairs with 256-deep stages: pairs move 2/3 of the operand bytes per
+  // FLOP, and each group's ragged last tile runs swapped with N = its tokens
+  // rounded up to 32, so the padding stays small.  The quantising and SwiGLU
+  // epilogues have no swapped tile (their pair tiles pad groups to 256 rows),
+  // so they take pairs only where groups average >= 768 rows over >= 40 K
+  // blocks.  Everything else runs 1-CTA 128x256 tiles with 128-deep stages
+  // (on B200 these won every other pass of the three MoE layers).
   // mxfp8_set_gemm_tiling overrides either choice.
   int force_cg = -1, force_ks = -1;
   gemm_tiling_override(&force_cg, &force_ks);
   int cg = 1, ks = 1;
-  if (a.mode != kWgrad) {
+  if (a.mode != kWgrad && !a.fp4) {
     const int64_t kblocks = ((a.mode == kFwd ? a.K : a.N) + BK - 1) / BK;
-    if (kblocks >= 40 && a.M >= int64_t(768) * a.E) { cg = 2; ks = 2; }
+    const bool epilogue_extra = a.swiglu || a.qr != nullptr || a.qc != nullptr;
+    if (epilogue_extra ? (kblocks >= 40 && a.M >= int64_t(768) * a.E) : kblocks >= 32) { cg = 2; ks = 2; }
   }
   if (force_cg == 0 || force_cg == 1) cg = force_cg == 1 ? 2 : 1;
   if (force_ks == 1 || force_ks == 2) ks = force_ks;
