@@ -165,6 +165,21 @@ def test_small_integer_operands_exact(mx, tile_config):
     run_all_and_compare(Case(mx, X, W, dY, offs), exact=True)
 
 
+def test_ragged_tails_of_every_pair_shape_exact(mx, tile_config):
+    """CTA pairs compute a group's last r < 256 rows as a swapped tile of
+    round_up(r, 32) tokens; tails r = 31, 32, 33, 64, ..., 224, 225, 255 (and
+    groups of exactly 256) cover every token-chunk count, both rounding cases
+    and tails behind full 256-row blocks.  Integer operands make every pass
+    exact; N = 640 leaves half of the last output-column block empty."""
+    counts = [32, 64 + 256, 96, 128, 160 + 512, 192, 224, 31, 33, 225, 255, 256]
+    offs = wl.offsets_from_counts(counts)
+    M, E, N, K = int(offs[-1]), len(counts), 640, 256
+    X = wl.integer_bf16((M, K), -14, 14, 11)
+    W = wl.integer_bf16((E, N, K), -14, 14, 12)
+    dY = wl.integer_bf16((M, N), -14, 14, 13)
+    run_all_and_compare(Case(mx, X, W, dY, offs), exact=True)
+
+
 def test_distinct_block_scales_pin_the_scale_layout(mx, tile_config):
     """Every 32-block gets its own power-of-two magnitude, so a scale read
     from the wrong row or block breaks parity."""
