@@ -74,7 +74,7 @@ constexpr int round_up_c(int a, int b) { return (a + b - 1) / b * b; }
 template <int CG, int KS_, bool FP4 = false>
 struct Cfg {
   static constexpr int KS = KS_;
-  static constexpr int STAGES = FP4 ? 3 : (CG == 2 ? (KS == 2 ? 3 : 6) : (KS == 2 ? 2 : 4));
+  static constexpr int STAGES = FP4 ? (CG == 2 ? 5 : 3) : (CG == 2 ? (KS == 2 ? 3 : 6) : (KS == 2 ? 2 : 4));
   static constexpr int APK = FP4 ? 4 : 1;              // scale atoms per K block and 128 rows
   static constexpr int SFA_T = SFA_TILE * APK, SFB_T = SFB_TILE * APK;
   static constexpr int SLOTS = STAGES * KS;            // 128-wide K-block slots in the ring
@@ -412,7 +412,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const __grid_constant__ CUtensorMap tmOut, const Params p) {
   using C = Cfg<CG, KS, FP4>;
   constexpr int STAGES = C::STAGES;
-  constexpr bool ST = CG == 2 && !QE && !FP4 && !SG;   // swapped ragged last tiles (see decode_tile)
+  constexpr bool ST = CG == 2 && !QE && !SG;   // swapped ragged last tiles (see decode_tile)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -636,16 +636,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             for (int i = 0; i < 4; ++i) {
               if (FULL || i < nk) {
                 const uint32_t sfa_t = set0 + SF_STRIDE * i, sfb_t = sfa_t + 4;
-                tc_cp_32x128b_x4(sfa_t, dsa + (512 >> 4) * i);
-                tc_cp_32x128b_x4(sfb_t, dsb + (512 >> 4) * i);
-                tc_cp_32x128b_x4(sfb_t + 4, dsb + (512 >> 4) * (C::KS * C::APK + i));
+                if constexpr (CG == 2) {
+                  tc_cp_32x128b_x4_pair(sfa_t, dsa + (512 >> 4) * i);
+                  tc_cp_32x128b_x4_pair(sfb_t, dsb + (512 >> 4) * i);
+                  tc_cp_32x128b_x4_pair(sfb_t + 4, dsb + (512 >> 4) * (C::KS * C::APK + i));
+                } else {
+                  tc_cp_32x128b_x4(sfa_t, dsa + (512 >> 4) * i);
+                  tc_cp_32x128b_x4(sfb_t, dsb + (512 >> 4) * i);
+                  tc_cp_32x128b_x4(sfb_t + 4, dsb + (512 >> 4) * (C::KS * C::APK + i));
+                }
               }
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               if (FULL || i < nk) {
                 const uint32_t sfa_t = set0 + SF_STRIDE * i, sfb_t = sfa_t + 4;
-                tc_mma_nvf4(d_tmem, da + 2 * i, db + 2 * i, idesc0, sfa_t, sfb_t, acc);
+                if constexpr (CG == 2)
+                  tc_mma_nvf4_pair(d_tmem, da + 2 * i, db + 2 * i, idesc_t, sfa_t, sfb_t, acc);
+                else
+                  tc_mma_nvf4(d_tmem, da + 2 * i, db + 2 * i, idesc_t, sfa_t, sfb_t, acc);
                 acc = 1;
               }
             }
@@ -902,7 +911,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (col_ok) {
 #pragma unroll
               for (int k = 0; k < 16; ++k) {
-                const uint32_t pk = cvt_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                float f0 = __uint_as_float(v[2 * k]), f1 = __uint_as_float(v[2 * k + 1]);
+                if constexpr (FP4) { f0 = __fmul_rn(f0, oscale); f1 = __fmul_rn(f1, oscale); }
+                const uint32_t pk = cvt_bf16x2(f0, f1);
                 stg16[(2 * k) * 32 + lane] = static_cast<uint16_t>(pk & 0xFFFFu);
                 stg16[(2 * k + 1) * 32 + lane] = static_cast<uint16_t>(pk >> 16);
               }
@@ -1090,7 +1101,12 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   }
   if (force_cg == 0 || force_cg == 1) cg = force_cg == 1 ? 2 : 1;
   if (force_ks == 1 || force_ks == 2) ks = force_ks;
-  if (a.fp4) { cg = 1; ks = 1; }   // NVFP4: one configuration (1-CTA, 3 x 128-byte stages)
+  // NVFP4: 128-byte K blocks (256 elements) in single-block stages: 1-CTA tiles
+  // (3 stages) unless mxfp8_set_gemm_tiling asks for CTA pairs (5 stages).
+  // Pairs halve the operand bytes per FLOP but not the scale-factor copies
+  // each SM receives (three per K = 64 MMA), which bound this kernel: on
+  // B200 they measured 0.80-0.88x of the 1-CTA tiles on every pass.
+  if (a.fp4) { ks = 1; cg = force_cg == 1 ? 2 : 1; }
   const uint32_t sf_box_rows = 4 * ks * (a.fp4 ? 4 : 1);
   const int64_t out_rows = a.mode == kWgrad ? int64_t(a.E) * a.N : a.M;
   const int64_t out_cols = a.mode == kFwd ? (a.swiglu ? a.N / 2 : a.N) : a.K;
@@ -1132,7 +1148,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   p.qr = a.qr; p.sr = a.sr; p.qc = a.qc; p.sc = a.sc;
   p.qc_ld = a.qc_ld; p.sc_pitch = a.sc_pitch;
   p.amax_a = a.amax_a; p.amax_b = a.amax_b;
-  if (a.fp4) return launch_cg<1, 1, false, true>(p, maps, stream);
+  if (a.fp4) return cg == 2 ? launch_cg<2, 1, false, true>(p, maps, stream) : launch_cg<1, 1, false, true>(p, maps, stream);
   if (a.swiglu) {
     if (cg == 2) return ks == 2 ? launch_cg<2, 2, true, false, true>(p, maps, stream)
                                 : launch_cg<2, 1, true, false, true>(p, maps, stream);

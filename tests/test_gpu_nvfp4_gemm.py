@@ -24,6 +24,15 @@ def mx():
     return m
 
 
+@pytest.fixture(params=["default", "pair"])
+def fp4_tiling(mx, request):
+    """The NVFP4 GEMM in its default 1-CTA tiles and in CTA pairs (each group's
+    ragged last tile swapped)."""
+    mx.mxfp8_set_gemm_tiling(1 if request.param == "pair" else -1, -1)
+    yield request.param
+    mx.mxfp8_set_gemm_tiling(-1, -1)
+
+
 class Fp4Case:
     def __init__(self, mx, X, W, dY, offs):
         self.mx, self.offs = mx, np.asarray(offs, dtype=np.int32)
@@ -80,11 +89,11 @@ def check(mx, counts, N, K, seed=0):
             assert_gemm_close(gdw[e], rdw[e], f"nvfp4 wgrad expert {e}")
 
 
-def test_tiny(mx):
+def test_tiny(mx, fp4_tiling):
     check(mx, [0, 7, 21, 36], 128, 256)
 
 
-def test_ragged_multi_tile(mx):
+def test_ragged_multi_tile(mx, fp4_tiling):
     """Several tiles per group, ragged tails, an empty expert, a partial output
     tile (N = 384) and a partial K block (K = 448: one full 256-element block
     and one of three MMAs)."""
@@ -93,8 +102,15 @@ def test_ragged_multi_tile(mx):
 
 @pytest.mark.parametrize("counts,N,K", [([1], 128, 64), ([0, 0, 5], 128, 128), ([300], 256, 320),
                                         ([129, 127], 512, 192), ([70, 0, 33, 200], 256, 1024)])
-def test_edge_shapes(mx, counts, N, K):
+def test_edge_shapes(mx, fp4_tiling, counts, N, K):
     check(mx, counts, N, K, seed=sum(counts))
+
+
+def test_ragged_tails_of_every_pair_shape(mx, fp4_tiling):
+    """Group tails r = 31..255 around the multiples of 32 (the swapped tiles of
+    CTA pairs have N = round_up(r, 32)), groups of exactly 256 rows and a half
+    empty last output-column block (N = 640)."""
+    check(mx, [32, 64 + 256, 96, 128, 160 + 512, 192, 224, 31, 33, 225, 255, 256], 640, 512, seed=21)
 
 
 def test_full_size_sampled_ds_v3_16b(mx):
