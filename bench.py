@@ -63,7 +63,7 @@ def parse():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the measurements outside the step (e2e, per-config passes, quantising epilogue, MoE "
                          "dispatch, NVFP4, quantiser sweep)")
-    ap.add_argument("--per-config-iters", type=int, default=10)
+    ap.add_argument("--per-config-iters", type=int, default=20)
     return ap.parse_args()
 
 
@@ -414,8 +414,9 @@ def run_ours(args, rank, world, local_rank):
 
 
 def timed_alone(fn, flush, iters):
-    """Median CUDA-event time (ms) of one launch with L2 flushed before it."""
-    for _ in range(2):
+    """Median CUDA-event time (ms) of one launch with L2 flushed before it,
+    after five warm-up launches."""
+    for _ in range(5):
         fn()
     ts = []
     for _ in range(iters):
@@ -851,7 +852,7 @@ def _cpu_sample(w: wl.Workload, budget_s: float):
     return flops, secs, desc
 
 
-def quantiser_sweep(mx, hbm_gbs, iters=10):
+def quantiser_sweep(mx, hbm_gbs, iters=20):
     """The quantiser sweep: M in {4096, 16384, 65536} x K in {2048, 5120, 7168},
     one group, N(0,1) with 0.1 % outliers x1000 and 1 % of aligned 32x32 tiles
     zeroed.  Rowwise, colwise and dual kernels, each launch timed alone with L2
@@ -860,18 +861,7 @@ def quantiser_sweep(mx, hbm_gbs, iters=10):
     flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
 
     def t(fn):
-        for _ in range(3):
-            fn()
-        tot = 0.0
-        for _ in range(iters):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            tot += a.elapsed_time(b)
-        return tot / iters
+        return timed_alone(fn, flush, iters)
 
     rows = []
     for M, K in wl.quantiser_sweep():
@@ -890,6 +880,7 @@ def quantiser_sweep(mx, hbm_gbs, iters=10):
         del x, q, sf, qT, sfT
     torch.cuda.empty_cache()
     return {"input": "N(0,1), 0.1 % outliers x1000, 1 % of aligned 32x32 tiles zeroed; one group",
+            "method": f"each launch alone, L2 flushed before it, five warm-ups, median of {iters}",
             "peak_gbs": hbm_gbs, "sizes": rows}
 
 
