@@ -295,6 +295,8 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, const Sched& s, int
       tl.sfb_atom0 = int64_t(s.rb[e] + 2 * mp) * p.sfa_pitch;
       tl.sfb_atom1 = tl.sfb_atom0 + p.sfa_pitch;
       tl.out_row = int64_t(row0) + 256 * mp;
+      tl.q_rb = s.rb[e] + 2 * mp;            // the tail's first 128-row scale block
+      tl.q_p = s.p[e] + 256 * mp;            // and its first colwise code column
       tl.rows = r;
       tl.out_col = int64_t(BN) * nt + 128 * static_cast<int32_t>(rank);
       tl.cols = static_cast<int32_t>(min64(128, out_cols - tl.out_col));
@@ -412,7 +414,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const __grid_constant__ CUtensorMap tmOut, const Params p) {
   using C = Cfg<CG, KS, FP4>;
   constexpr int STAGES = C::STAGES;
-  constexpr bool ST = CG == 2 && !QE && !SG;   // swapped ragged last tiles (see decode_tile)
+  constexpr bool ST = CG == 2 && !SG;   // swapped ragged last tiles (see decode_tile)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -885,22 +887,50 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           // Swapped tile: lane n of this warp's quarter is output column
           // out_col + 32 * quarter + n, accumulator column i is token i.  Each
           // 32-token chunk goes through the warp's stage as a [32 tokens][32
-          // columns] bf16 block, then out as 64-byte row segments (tokens past
-          // the group are not written).  Chunks shared with the other
+          // columns] bf16 block (neighbouring lanes pair their columns with a
+          // shuffle, so each lane stores 4-byte words; the 16-byte chunk q of
+          // token row j sits at chunk q ^ (j / 2 % 4), which keeps both the
+          // stores and the 16-byte row reads free of bank conflicts), then
+          // out as 64-byte row segments (tokens past the group are not written).  Chunks shared with the other
           // accumulator are drained first (buffer 0: the high ones, buffer 1:
           // the low ones), then the accumulator is released.
+          // Quantising epilogue: a lane's 32 tokens of one column are that
+          // column's colwise 32-block (encoded from registers; tokens past the
+          // group are pad: out of the amax, code 0), and a stage row is one
+          // token's rowwise 32-block (encoded by the lane that reads it back).
+          // Every scale byte of the 128-token blocks the tile covers is
+          // written, zero for pad tokens and blocks.
           const int nch = tl.ntok / 32;
           const int ov_lo = buf == 0 ? static_cast<int>(C::ACC_STRIDE / 32) : 0;
           const int ov_hi = buf == 0 ? 8 : static_cast<int>((256 - C::ACC_STRIDE) / 32);
           const int n_ov = max(0, min(nch, ov_hi) - ov_lo);
           if (n_ov == 0) release();
           int done_ov = 0;
-          uint16_t* stg16 = reinterpret_cast<uint16_t*>(stage_base);
+          uint32_t* stg32 = reinterpret_cast<uint32_t*>(stage_base);
           const uint4* stg4 = reinterpret_cast<const uint4*>(stage_base);
+          auto swz = [](int row, int q) { return row * 4 + (q ^ ((row >> 1) & 3)); };   // 16-byte chunk index
           if (lane == 0) bulk_wait_read<0>();   // an earlier tile's TMA store has read the stage
           __syncwarp();
           const bool col_ok = tl.cols > 32 * static_cast<int32_t>(quarter);
-          uint16_t* out_q = p.out + tl.out_row * p.out_ld + tl.out_col + 32 * quarter;
+          const int64_t col_q = tl.out_col + 32 * quarter;   // this warp's first output column
+          const int64_t n_col = col_q + lane;                 // this lane's output column
+          const int64_t pitch_r = (p.out_ld + 127) / 128;     // rowwise atoms per atom row
+          const bool atoms = tl.out_col / 128 < pitch_r;      // this CTA's columns own scale atoms
+          // Scale bytes of token chunk jc: rowwise (token 32 jc + lane, block
+          // `quarter` of this CTA's atom column), colwise (column n_col, 32-token
+          // sub-block jc % 4).
+          auto put_scales = [&](int jc, uint32_t rs, uint32_t cs) {
+            if constexpr (QE) {
+              if (!atoms) return;
+              const int64_t rb = tl.q_rb + jc / 4;
+              if (p.sr != nullptr)
+                p.sr[512 * (rb * pitch_r + tl.out_col / 128) + lane * 16 + (jc & 3) * 4 + quarter] =
+                    static_cast<uint8_t>(rs);
+              if (p.sc != nullptr)
+                p.sc[512 * ((n_col / 128) * p.sc_pitch + rb) + lane * 16 + quarter * 4 + (jc & 3)] =
+                    static_cast<uint8_t>(cs);
+            }
+          };
 #pragma unroll 1
           for (int i = 0; i < nch; ++i) {
             const int jc = buf == 0 ? nch - 1 - i : i;
@@ -908,25 +938,76 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             tmem_ld_32x32b_x32(tbase + 32 * jc, v);
             tmem_wait_regs(v);
             if (jc >= ov_lo && jc < ov_hi && ++done_ov == n_ov) release();
+            uint32_t rs = 0, cs = 0;
             if (col_ok) {
+              uint32_t pk[16];   // bf16 tokens 2k (low half) and 2k + 1 of this lane's column
+              const bool odd = lane & 1;
 #pragma unroll
               for (int k = 0; k < 16; ++k) {
                 float f0 = __uint_as_float(v[2 * k]), f1 = __uint_as_float(v[2 * k + 1]);
                 if constexpr (FP4) { f0 = __fmul_rn(f0, oscale); f1 = __fmul_rn(f1, oscale); }
-                const uint32_t pk = cvt_bf16x2(f0, f1);
-                stg16[(2 * k) * 32 + lane] = static_cast<uint16_t>(pk & 0xFFFFu);
-                stg16[(2 * k + 1) * 32 + lane] = static_cast<uint16_t>(pk >> 16);
+                pk[k] = cvt_bf16x2(f0, f1);
+                // even lane: token 2k of columns (lane, lane + 1); odd lane: token 2k + 1 of (lane - 1, lane)
+                const uint32_t other = __shfl_xor_sync(0xffffffffu, pk[k], 1);
+                const uint32_t word = odd ? __byte_perm(other, pk[k], 0x7632) : __byte_perm(pk[k], other, 0x5410);
+                const int row = 2 * k + (odd ? 1 : 0), w = lane >> 1;
+                stg32[swz(row, w >> 2) * 4 + (w & 3)] = word;
+              }
+              if constexpr (QE) {
+                if (p.qc != nullptr) {
+                  const int valid = min(32, tl.rows - 32 * jc);   // real tokens of this 32-block
+#pragma unroll
+                  for (int k = 0; k < 16; ++k) {
+                    if (2 * k >= valid) pk[k] = 0u;
+                    else if (2 * k + 1 >= valid) pk[k] &= 0xFFFFu;
+                  }
+                  uint32_t a = 0;
+#pragma unroll
+                  for (int u = 0; u < 4; ++u)
+                    a = max(a, amax_bits8(make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3])));
+                  cs = scale_byte(a);
+                  uint32_t o[8];
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) {
+                    const uint2 w = encode8(make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]), cs);
+                    o[2 * u] = cs == 0xFFu ? nan_codes4(2 * u, valid) : w.x;
+                    o[2 * u + 1] = cs == 0xFFu ? nan_codes4(2 * u + 1, valid) : w.y;
+                  }
+                  uint4* qcol = reinterpret_cast<uint4*>(p.qc + n_col * p.qc_ld + tl.q_p + 32 * jc);
+                  qcol[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                  qcol[1] = make_uint4(o[4], o[5], o[6], o[7]);
+                }
               }
               __syncwarp();
+              if (p.out != nullptr) {
+                uint16_t* out_q = p.out + tl.out_row * p.out_ld + col_q;
 #pragma unroll
-              for (int it = 0; it < 4; ++it) {
-                const int row = 8 * it + (lane >> 2), q = lane & 3;
-                const int32_t tok = 32 * jc + row;
-                if (tok < tl.rows)
-                  *reinterpret_cast<uint4*>(out_q + int64_t(tok) * p.out_ld + 8 * q) = stg4[row * 4 + q];
+                for (int it = 0; it < 4; ++it) {
+                  const int row = 8 * it + (lane >> 2), q = lane & 3;
+                  const int32_t tok = 32 * jc + row;
+                  if (tok < tl.rows)
+                    *reinterpret_cast<uint4*>(out_q + int64_t(tok) * p.out_ld + 8 * q) = stg4[swz(row, q)];
+                }
+              }
+              if constexpr (QE) {
+                const int32_t tok = 32 * jc + lane;
+                if (p.qr != nullptr && tok < tl.rows) {
+                  const uint4 r0 = stg4[swz(lane, 0)], r1 = stg4[swz(lane, 1)], r2 = stg4[swz(lane, 2)],
+                              r3 = stg4[swz(lane, 3)];
+                  rs = scale_byte(max(max(amax_bits8(r0), amax_bits8(r1)), max(amax_bits8(r2), amax_bits8(r3))));
+                  const uint2 w0 = encode8(r0, rs), w1 = encode8(r1, rs), w2 = encode8(r2, rs), w3 = encode8(r3, rs);
+                  uint4* qrow = reinterpret_cast<uint4*>(p.qr + (tl.out_row + tok) * p.out_ld + col_q);
+                  qrow[0] = make_uint4(w0.x, w0.y, w1.x, w1.y);
+                  qrow[1] = make_uint4(w2.x, w2.y, w3.x, w3.y);
+                }
               }
               __syncwarp();
             }
+            put_scales(jc, rs, cs);
+          }
+          if constexpr (QE) {
+            // the rest of the last 128-token block: pad tokens, zero scales
+            for (int jc = nch; jc < (nch + 3) / 4 * 4; ++jc) put_scales(jc, 0u, 0u);
           }
           ++j;
           continue;
@@ -1082,22 +1163,20 @@ cudaError_t launch_cg(const Params& p, const CUtensorMap (&maps)[5], cudaStream_
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** detail) {
   // Tile configuration, from sizes the host knows (the group sizes stay on
-  // the device).  Plain fwd/dgrad over long contractions (>= 32 K blocks) run
-  // CTA pairs with 256-deep stages: pairs move 2/3 of the operand bytes per
-  // FLOP, and each group's ragged last tile runs swapped with N = its tokens
-  // rounded up to 32, so the padding stays small.  The quantising and SwiGLU
-  // epilogues have no swapped tile (their pair tiles pad groups to 256 rows),
-  // so they take pairs only where groups average >= 768 rows over >= 40 K
-  // blocks.  Everything else runs 1-CTA 128x256 tiles with 128-deep stages
-  // (on B200 these won every other pass of the three MoE layers).
-  // mxfp8_set_gemm_tiling overrides either choice.
+  // the device).  fwd/dgrad over long contractions (>= 32 K blocks) run CTA
+  // pairs with 256-deep stages: pairs move 2/3 of the operand bytes per FLOP,
+  // and each group's ragged last tile runs swapped with N = its tokens rounded
+  // up to 32, so the padding stays small.  The SwiGLU epilogue has no swapped
+  // tile (its pair tiles pad groups to 256 rows), so it takes pairs only where
+  // groups average >= 768 rows over >= 40 K blocks.  Everything else runs
+  // 1-CTA 128x256 tiles with 128-deep stages (on B200 these won every other
+  // pass of the three MoE layers).  mxfp8_set_gemm_tiling overrides either choice.
   int force_cg = -1, force_ks = -1;
   gemm_tiling_override(&force_cg, &force_ks);
   int cg = 1, ks = 1;
   if (a.mode != kWgrad && !a.fp4) {
     const int64_t kblocks = ((a.mode == kFwd ? a.K : a.N) + BK - 1) / BK;
-    const bool epilogue_extra = a.swiglu || a.qr != nullptr || a.qc != nullptr;
-    if (epilogue_extra ? (kblocks >= 40 && a.M >= int64_t(768) * a.E) : kblocks >= 32) { cg = 2; ks = 2; }
+    if (a.swiglu ? (kblocks >= 40 && a.M >= int64_t(768) * a.E) : kblocks >= 32) { cg = 2; ks = 2; }
   }
   if (force_cg == 0 || force_cg == 1) cg = force_cg == 1 ? 2 : 1;
   if (force_ks == 1 || force_ks == 2) ks = force_ks;
