@@ -891,9 +891,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           // shuffle, so each lane stores 4-byte words; the 16-byte chunk q of
           // token row j sits at chunk q ^ (j / 2 % 4), which keeps both the
           // stores and the 16-byte row reads free of bank conflicts), then
-          // out as 64-byte row segments (tokens past the group are not written).  Chunks shared with the other
-          // accumulator are drained first (buffer 0: the high ones, buffer 1:
-          // the low ones), then the accumulator is released.
+          // leaves as 64-byte row segments (tokens past the group are not
+          // written).  Chunks shared with the other accumulator are drained
+          // first (buffer 0: the high ones, buffer 1: the low ones), then the
+          // accumulator is released.
           // Quantising epilogue: a lane's 32 tokens of one column are that
           // column's colwise 32-block (encoded from registers; tokens past the
           // group are pad: out of the amax, code 0), and a stage row is one

@@ -110,7 +110,7 @@ def test_quantising_epilogue(mx, tile_config, name, mode):
 
 
 @pytest.mark.parametrize("mode", ["fwd", "dgrad"])
-def test_distinct_block_magnitudes_and_overflow(mx, mode):
+def test_distinct_block_magnitudes_and_overflow(mx, tile_config, mode):
     """Rows of X and dY scaled by powers of two from 2^-30 to 2^40 give
     output blocks over a wide scale range; a few rows scaled by 2^120 make
     the fp32 accumulators overflow, so their blocks take the NaN-scale path."""
@@ -130,8 +130,9 @@ def test_distinct_block_magnitudes_and_overflow(mx, mode):
 
 
 @pytest.mark.parametrize("mode", ["fwd", "dgrad"])
-def test_each_output_alone(mx, mode):
-    """Any subset of {bf16, rowwise, colwise} gives the same bytes."""
+def test_each_output_alone(mx, tile_config, mode):
+    """Any subset of {bf16, rowwise, colwise} gives the same bytes (in CTA
+    pairs the groups' ragged tiles run swapped, with their own drain)."""
     c = make_case(mx, [0, 1, 129, 300, 77, 255], 384, 416, seed=7)
     y_all, r_all, c_all = fused(mx, c, mode)
     _, r_only, _ = fused(mx, c, mode, out=False, colwise=False)
