@@ -281,15 +281,19 @@ MXF8_API mxf8_status mxfp8_grouped_gemm_fwd_noalloc(const uint8_t* xq, const uin
 /* ---------------------------------------------------------------- tuning and testing switches */
 
 /* Overrides, for the calling process, the tile configuration the grouped
- * GEMMs (MXFP8) choose per pass.  The pages fix no tiling; these are this
- * library's own pipeline shapes.
+ * GEMMs choose per pass.  The pages fix no tiling; these are this library's
+ * own pipeline shapes.
  *   cta_pair  -1 = the library's rule, 0 = 1-CTA 128x256 tiles,
- *             1 = CTA-pair 256x256 tiles (cta_group::2)
+ *             1 = CTA-pair 256x256 tiles (cta_group::2; in fwd/dgrad each
+ *             group's ragged last tile runs with the operand roles swapped)
  *   stage_k   -1 = the library's rule, 1 = 128-deep K stages, 2 = 256-deep
- * Results are the same under every setting (same products, same fp32
- * accumulation order within a 32-element step); only speed changes.  Returns
- * MXF8_ERR_INVALID_ARG for any other value.  Not thread-safe against
- * concurrent GEMM calls. */
+ *             (MXFP8 only; the NVFP4 GEMMs take cta_pair and always use
+ *             single 128-byte K blocks per stage)
+ * Every setting computes the same exact products in fp32 and meets the same
+ * tolerance; the hardware's summation order inside a tile may differ between
+ * shapes, so results can differ in the last bits.  Only speed is meant to
+ * change.  Returns MXF8_ERR_INVALID_ARG for any other value.  Not
+ * thread-safe against concurrent GEMM calls. */
 MXF8_API mxf8_status mxfp8_set_gemm_tiling(int32_t cta_pair, int32_t stage_k);
 
 /* Test switch for the bounded pipeline waits: while enabled (enable != 0),
