@@ -413,14 +413,20 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
-def timed_alone(fn, flush, iters):
+def timed_alone(fn, flush, iters, clean=False):
     """Median CUDA-event time (ms) of one launch with L2 flushed before it,
-    after five warm-up launches."""
+    after five warm-up launches.  The flush writes a buffer twice the size of
+    L2; clean=True also reads it back, so L2 is left holding clean lines
+    instead of up to a full L2 of dirty ones that the timed launch would have
+    to write back to HBM on its first misses (which charges a bandwidth-bound
+    kernel for traffic that is not its own)."""
     for _ in range(5):
         fn()
     ts = []
     for _ in range(iters):
         flush.zero_()
+        if clean:
+            flush.sum()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         fn()
@@ -445,7 +451,7 @@ def per_config(mx, args, fp8_peak, hbm_gbs, dev, device_index):
             w = wl.WORKLOADS[name]()
             cfg = {"routing": ROUTING[name], "experts": w.E, "routed_rows": w.M, "linears": {}}
             tot = {p: [0.0, 0.0] for p in ("fwd", "dgrad", "wgrad")}
-            q_bytes, q_ms = 0.0, 0.0
+            q_bytes, q_ms, q_ms_dirty = 0.0, 0.0, 0.0
             for layer in w.layers:
                 L = Linear(mx, w, layer, dev, "dual")
                 for fn in L.dual_quantisations():
@@ -461,7 +467,8 @@ def per_config(mx, args, fp8_peak, hbm_gbs, dev, device_index):
                 if mx.mxfp8_get_status(L.work) != 0:
                     raise SystemExit(f"bench: device status error in the {name} {layer.name} passes")
                 for fn in L.dual_quantisations():
-                    q_ms += timed_alone(fn, flush, it)
+                    q_ms += timed_alone(fn, flush, it, clean=True)
+                    q_ms_dirty += timed_alone(fn, flush, it)
                 q_bytes += L.quant_bytes()
                 cfg["linears"][layer.name] = r
                 del L
@@ -472,13 +479,17 @@ def per_config(mx, args, fp8_peak, hbm_gbs, dev, device_index):
             cfg["all_passes"] = {"tflops": round(f_all / (ms_all * 1e-3) / 1e12, 1),
                                  "frac": round(f_all / (ms_all * 1e-3) / 1e12 / fp8_peak, 4)}
             gbs = q_bytes / (q_ms * 1e-3) / 1e9
+            gbs_dirty = q_bytes / (q_ms_dirty * 1e-3) / 1e9
             cfg["quantiser"] = {"kernel": "quantize_dual_kernel (X, W, dY of both linears)", "ms": round(q_ms, 4),
-                                "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4)}
+                                "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4),
+                                "flush": "written, then read back (L2 left clean)",
+                                "write_only_flush": {"ms": round(q_ms_dirty, 4), "gbs": round(gbs_dirty, 1),
+                                                     "frac": round(gbs_dirty / hbm_gbs, 4)}}
             res[name] = cfg
     del flush
     torch.cuda.empty_cache()
-    res["method"] = (f"each launch alone, L2 flushed before it ({2 * max(l2, 64 << 20) >> 20} MiB written), "
-                     f"median of {it}")
+    res["method"] = (f"each launch alone, L2 flushed before it ({2 * max(l2, 64 << 20) >> 20} MiB written; the "
+                     f"quantisers' flush also reads it back), five warm-ups, median of {it}")
     res["clocks"] = clk.summary()
     return res
 
@@ -860,8 +871,8 @@ def quantiser_sweep(mx, hbm_gbs, iters=20):
     2 + 1 + 1/32 B per element, dual: 2 + 2 (1 + 1/32))."""
     flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
 
-    def t(fn):
-        return timed_alone(fn, flush, iters)
+    def t(fn, clean=True):
+        return timed_alone(fn, flush, iters, clean)
 
     rows = []
     for M, K in wl.quantiser_sweep():
@@ -873,14 +884,16 @@ def quantiser_sweep(mx, hbm_gbs, iters=20):
                               ("colwise", lambda: mx.mxfp8_quantize_colwise(x, None, qT=qT, scales=sfT), 3.03125),
                               ("dual", lambda: mx.mxfp8_quantize_dual(x, None, q=q, scales=sf, qT=qT, scalesT=sfT),
                                4.0625)):
-            ms = t(fn)
-            gbs = M * K * bpe / (ms * 1e-3) / 1e9
-            r[name] = {"us": round(ms * 1e3, 1), "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4)}
+            ms, ms_dirty = t(fn), t(fn, clean=False)
+            gbs, gbs_dirty = M * K * bpe / (ms * 1e-3) / 1e9, M * K * bpe / (ms_dirty * 1e-3) / 1e9
+            r[name] = {"us": round(ms * 1e3, 1), "gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4),
+                       "write_only_flush": {"us": round(ms_dirty * 1e3, 1), "frac": round(gbs_dirty / hbm_gbs, 4)}}
         rows.append(r)
         del x, q, sf, qT, sfT
     torch.cuda.empty_cache()
     return {"input": "N(0,1), 0.1 % outliers x1000, 1 % of aligned 32x32 tiles zeroed; one group",
-            "method": f"each launch alone, L2 flushed before it, five warm-ups, median of {iters}",
+            "method": (f"each launch alone, L2 flushed before it (a 256 MiB buffer written, then read back, so L2 "
+                       f"holds clean lines; write_only_flush: written only), five warm-ups, median of {iters}"),
             "peak_gbs": hbm_gbs, "sizes": rows}
 
 
