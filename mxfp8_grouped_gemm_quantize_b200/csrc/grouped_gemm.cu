@@ -10,7 +10,9 @@
 // Every operand is K-major E4M3 with E8M0 scales per 32 elements along K
 // (MXFP8: opensourcebeat.com, "Enabling up to 41% faster pre-training ...",
 // FAQ), so one block-scaled MMA instruction (kind::mxf8f6f4, K = 32) applies
-// the scales in hardware and accumulates in fp32 tensor memory.
+// the scales in hardware and accumulates in fp32 tensor memory.  The NVFP4
+// variant (FP4) takes E2M1 operands with E4M3 scales per 16 elements
+// (kind::mxf4nvf4, K = 64) through the same pipeline.
 //
 // One kernel template, CG = CTAs per MMA:
 //   CG = 2: CTA pairs (clusters of 2) issue 256x256x32 MMAs
@@ -26,12 +28,13 @@
 // tensor-memory columns, and (in the leader CTA) one thread copies scale
 // atoms to tensor memory and issues the MMAs; warps 2-5 drain the
 // accumulator: tcgen05.ld -> bf16 -> 128-byte-swizzled shared stage -> TMA
-// bulk-tensor store (plain masked stores only for a group's ragged slice).
+// bulk-tensor store (plain masked stores only for a group's ragged slice and
+// for the row segments of a swapped tile).
 // Two 128x256 fp32 accumulators overlap in 64 or 128 columns (0..255 and
 // 192..447, or 128..383 when more pipeline stages need more scale columns);
 // the epilogue drains the shared columns first and releases the accumulator,
 // so the next tile's MMAs overlap the rest of the drain.  The columns after
-// accumulator 1 hold one scale-factor set per pipeline stage.
+// accumulator 1 hold the scale-factor sets (see Cfg).
 // The tile schedule is built on the device from the group offsets at kernel
 // start (no host synchronisation); tiles are dealt round-robin.  Every wait is
 // bounded: on timeout the kernel records MXF8_ERR_TIMEOUT, drains its
