@@ -271,6 +271,21 @@ def test_workload_full_size_sampled(mx, name):
         _sampled_check(Case(mx, X, W, dY, w.offsets, check_quant=False), rng)
 
 
+@pytest.mark.parametrize("seed", range(8))
+def test_random_shapes(mx, tile_config, seed):
+    """Seeded random problems: 1-24 experts with counts from 0 to 700 (a few
+    empty), N a multiple of 128 up to 640, K a multiple of 32 up to 1024 -- so
+    every tile shape meets full, ragged and swapped tiles, partial output
+    blocks and partial K blocks in combinations no hand-picked case covers."""
+    rng = np.random.default_rng(1000 + seed)
+    E = int(rng.integers(1, 25))
+    counts = rng.integers(0, 701, size=E)
+    counts[rng.random(E) < 0.15] = 0
+    N = 128 * int(rng.integers(1, 6))
+    K = 32 * int(rng.integers(1, 33))
+    run_all_and_compare(make_case(mx, counts.tolist(), N, K, seed=seed))
+
+
 def test_the_largest_group_count(mx, tile_config):
     """MXF8_GEMM_MAX_GROUPS experts, most of them empty or tiny: the on-device
     schedule's prefix runs over eight warps' worth of groups and the wgrad

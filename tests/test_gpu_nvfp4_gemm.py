@@ -106,6 +106,18 @@ def test_edge_shapes(mx, fp4_tiling, counts, N, K):
     check(mx, counts, N, K, seed=sum(counts))
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_random_shapes(mx, fp4_tiling, seed):
+    """Seeded random problems (1-16 experts, counts 0-600 with some empty,
+    N a multiple of 128 up to 512, K a multiple of 64 up to 1024) in both
+    tile shapes."""
+    rng = np.random.default_rng(2000 + seed)
+    E = int(rng.integers(1, 17))
+    counts = rng.integers(0, 601, size=E)
+    counts[rng.random(E) < 0.15] = 0
+    check(mx, counts.tolist(), 128 * int(rng.integers(1, 5)), 64 * int(rng.integers(1, 17)), seed=seed)
+
+
 def test_ragged_tails_of_every_pair_shape(mx, fp4_tiling):
     """Group tails r = 31..255 around the multiples of 32 (the swapped tiles of
     CTA pairs have N = round_up(r, 32)), groups of exactly 256 rows and a half
