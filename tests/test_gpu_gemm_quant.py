@@ -110,6 +110,20 @@ def test_quantising_epilogue(mx, tile_config, name, mode):
 
 
 @pytest.mark.parametrize("mode", ["fwd", "dgrad"])
+@pytest.mark.parametrize("seed", range(3))
+def test_quantising_epilogue_random_shapes(mx, tile_config, seed, mode):
+    """Seeded random problems: 1-16 experts, counts 0-600 (some empty), N a
+    multiple of 128 up to 640, K a multiple of 32 up to 768 -- partial scale
+    atoms, ragged and swapped tiles in every tile shape."""
+    rng = np.random.default_rng(4000 + seed)
+    E = int(rng.integers(1, 17))
+    counts = rng.integers(0, 601, size=E)
+    counts[rng.random(E) < 0.15] = 0
+    N, K = 128 * int(rng.integers(1, 6)), 32 * int(rng.integers(1, 25))
+    check_mode(mx, make_case(mx, counts.tolist(), N, K, seed=seed, check_quant=False), mode)
+
+
+@pytest.mark.parametrize("mode", ["fwd", "dgrad"])
 def test_distinct_block_magnitudes_and_overflow(mx, tile_config, mode):
     """Rows of X and dY scaled by powers of two from 2^-30 to 2^40 give
     output blocks over a wide scale range; a few rows scaled by 2^120 make

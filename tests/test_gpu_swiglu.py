@@ -124,6 +124,17 @@ def test_swiglu_epilogue(mx, tile_config, counts, N, K):
     check(mx, _op(mx, counts, N, K, seed=N + K))
 
 
+@pytest.mark.parametrize("seed", range(3))
+def test_swiglu_random_shapes(mx, tile_config, seed):
+    """Seeded random problems: 1-16 experts, counts 0-600 (some empty), N a
+    multiple of 256 up to 1024, K a multiple of 32 up to 768."""
+    rng = np.random.default_rng(3000 + seed)
+    E = int(rng.integers(1, 17))
+    counts = rng.integers(0, 601, size=E)
+    counts[rng.random(E) < 0.15] = 0
+    check(mx, _op(mx, counts.tolist(), 256 * int(rng.integers(1, 5)), 32 * int(rng.integers(1, 25)), seed=seed))
+
+
 def test_each_output_alone(mx):
     """Any subset of {bf16 h, rowwise, colwise} gives the same bytes, and a
     skipped layout is not touched."""
