@@ -155,6 +155,72 @@ def test_full_size_sampled_ds_v3_16b(mx):
     assert np.all(np.isfinite(f64(dx)[r[:16]])) and np.all(np.isfinite(f64(dw)[:, cn[:8], :][:, :, ck[:8]]))
 
 
+def _nvfp4_rows(q, sf, C, row0, atom_row0, n, S):
+    """Rows row0 .. row0 + n - 1 of a rowwise NVFP4 operand (their scale rows
+    start at 128-row atom row atom_row0), dequantised: fp64 [n, C]."""
+    pitch = oracle.nvfp4_rowwise_pitch(C)
+    nb = (n + 127) // 128
+    atoms = np.ascontiguousarray(sf[atom_row0 * pitch * 512:(atom_row0 + nb) * pitch * 512])
+    return oracle.nvfp4_dequantize_rowwise(np.ascontiguousarray(q[row0:row0 + n]), atoms, S)
+
+
+def _nvfp4_cols(qT, sfT, pitch, col0, atom_col0, n, S):
+    """Logical rows col0 .. col0 + n - 1 of a colwise NVFP4 operand (codes
+    from element column col0 of qT, an even number; scales from 64-row atom
+    column atom_col0 of every 128-row atom row), dequantised: fp64 [n, C]."""
+    C = qT.shape[0]
+    ld = oracle.nvfp4_colwise_ld(n, 1) // 2
+    sub = np.zeros((C, ld), dtype=np.uint8)
+    nbytes = (n + 1) // 2
+    sub[:, :nbytes] = qT[:, col0 // 2:col0 // 2 + nbytes]
+    rb, na = (C + 127) // 128, (n + 63) // 64
+    atoms = np.asarray(sfT[:rb * pitch * 512]).reshape(rb, pitch, 512)[:, atom_col0:atom_col0 + na]
+    return oracle.nvfp4_dequantize_colwise(sub, np.ascontiguousarray(atoms).reshape(-1), n, S)
+
+
+def test_whole_tensors_ds_v3_671b_gate_up(mx):
+    """The DeepSeek-V3-671B-like gate/up linear at full size in the default
+    launch configuration: every output element of fwd, dgrad and wgrad,
+    expert by expert, against the oracle's fp64 product of the GPU's own
+    NVFP4 bytes (zero dW for an expert without rows)."""
+    w = wl.WORKLOADS["ds-v3-671b"]()
+    L = w.layers[0]
+    X, W, dY = wl.layer_tensors(w, L)
+    c = Fp4Case(mx, X, W, dY, w.offsets)
+    del X, W, dY
+    y, dx, dw = c.run()
+    o = np.asarray(c.offs, np.int64)
+    m = np.diff(o)
+    E, N, K, M = c.E, c.N, c.K, c.M
+    RB = np.concatenate([[0], np.cumsum((m + 127) // 128)])
+    Q = np.concatenate([[0], np.cumsum((m + 63) // 64)])
+    P = np.concatenate([[0], np.cumsum((m + 31) // 32 * 32)])
+    xq, xs, wq, ws = np_u8(c.xq), np_u8(c.xs), np_u8(c.wq), np_u8(c.ws)
+    dyq, dys, wqT, wsT = np_u8(c.dyq), np_u8(c.dys), np_u8(c.wqT), np_u8(c.wsT)
+    pitch_w = oracle.nvfp4_colwise_pitch(E * N, 1)
+    for e in range(E):
+        lo, hi = int(o[e]), int(o[e + 1])
+        if hi == lo:
+            continue
+        We = _nvfp4_rows(wq, ws, K, e * N, e * N // 128, N, c.Sw)
+        Xe = _nvfp4_rows(xq, xs, K, lo, int(RB[e]), hi - lo, c.Sx)
+        assert_gemm_close(f64(y[lo:hi]), Xe @ We.T, f"nvfp4 fwd expert {e}")
+        dYe = _nvfp4_rows(dyq, dys, N, lo, int(RB[e]), hi - lo, c.Sdy)
+        WeT = _nvfp4_cols(wqT, wsT, pitch_w, e * N, e * N // 64, N, c.Sw)
+        assert_gemm_close(f64(dx[lo:hi]), dYe @ WeT, f"nvfp4 dgrad expert {e}")
+    del xq, xs, wq, ws, dyq, dys, wqT, wsT
+    dyqT, dysT, xqT, xsT = np_u8(c.dyqT), np_u8(c.dysT), np_u8(c.xqT), np_u8(c.xsT)
+    pitch = oracle.nvfp4_colwise_pitch(M, E)
+    for e in range(E):
+        got = f64(dw[e])
+        if m[e] == 0:
+            assert np.all(got == 0.0), f"nvfp4 wgrad: empty expert {e} is not zero"
+            continue
+        dYc = _nvfp4_cols(dyqT, dysT, pitch, int(P[e]), int(Q[e]), int(m[e]), c.Sdy)
+        Xc = _nvfp4_cols(xqT, xsT, pitch, int(P[e]), int(Q[e]), int(m[e]), c.Sx)
+        assert_gemm_close(got, dYc.T @ Xc, f"nvfp4 wgrad expert {e}")
+
+
 def _row_scales(sf, row, offs, C):
     """The scale atom bytes of one row, re-packed as a single-row buffer in the
     same layout (row 0 of a one-group matrix)."""
